@@ -1,0 +1,379 @@
+#!/usr/bin/env python3
+"""Benchmark of the KDA layer core on B200.
+
+One step = one prefill call of the 8K-token workload (prefill_bf16_T8192_H32:
+1 sequence x 8192 tokens x 32 heads x d=128, bf16 q/k/v, fp32 log-decay and
+beta, zero initial state, final state returned) through the library's C ABI.
+The decode step of the 256-sequence x 34-layer workload (one layer per call,
+rotating over the 34 state slabs) is timed the same way and reported in the
+``decode`` object.  Inputs are synthetic and seeded (gated_delta_rule_152_b200.inputs).
+
+Multi-GPU: one process per GPU (torchrun).  Sequences and heads are
+independent, so every rank runs its own replica of the workload (weak
+scaling) with no collective on the data path; the timed region is bracketed by
+a barrier and the max over ranks is reported.
+
+``--impl reference`` times the fp64 CPU oracle (the only reference that
+exists for this method) on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gated_delta_rule_152_b200 import inputs as kin  # noqa: E402
+
+METRIC = "KDA prefill tokens/s and decode seq-steps/s per layer on 1 B200; % of roofline"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+TF32_OVER_BF16 = 1.1 / 2.25          # nominal dense tf32 : bf16 tensor-core ratio
+D = 128
+# Algorithmic HBM bytes per token-head of the prefill: q, k, v bf16 (3 x 256),
+# g fp32 (512), beta (4), o fp32 (512).  Per (sequence, head) add the final
+# state write (64 KiB) and, when given, the initial state read (64 KiB).
+PREFILL_BYTES_PER_TOKEN_HEAD = 3 * 2 * D + 4 * D + 4 + 4 * D
+STATE_BYTES = 4 * D * D
+# Dense contraction flops per token-head of the 64-token chunk form:
+# 5 x (2 C^2 d) + 3 x (2 C d^2) + C^3 / 3 per chunk of C = 64 tokens.
+PREFILL_FLOPS_PER_TOKEN_HEAD = (5 * 2 * 64 * 64 * D + 3 * 2 * 64 * D * D + 64 ** 3 // 3) // 64
+# Decode: state read + write, plus q, k, v (bf16), g (fp32), beta, o (fp32).
+DECODE_BYTES_PER_SEQ_HEAD = 2 * STATE_BYTES + 3 * 2 * D + 4 * D + 4 + 4 * D
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, 1400.0, "fallback"
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.out = None
+        try:
+            props = torch.cuda.get_device_properties(device_index)
+            bus = getattr(props, "pci_bus_id", None)
+            dom = getattr(props, "pci_domain_id", 0)
+            devn = getattr(props, "pci_device_id", 0)
+            self.target = f"{dom:08x}:{bus:02x}:{devn:02x}.0" if bus is not None else str(device_index)
+        except Exception:
+            self.target = str(device_index)
+
+    def start(self):
+        try:
+            self.out = open(os.devnull, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.target, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            text, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            text = ""
+        sms, maxs, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in text.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sms.append(float(parts[0]))
+                maxs.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sms:
+            return None
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxs), "reasons": sorted(reasons),
+                "samples": len(sms)}
+
+
+# ---------------------------------------------------------------- distributed
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- CPU baseline
+def oracle_prefill_sample(x: kin.PrefillInputs, tokens: int, threads: int = 0):
+    """Run the fp64 oracle on the first `tokens` tokens of the workload (all
+    heads); returns (seconds, tokens)."""
+    import oracle
+    sl = slice(0, tokens)
+    t0 = time.perf_counter()
+    oracle.kda_forward(x.q[sl], x.k[sl], x.v[sl], x.g[sl], x.beta[sl], [0, tokens], None, threads=threads)
+    return time.perf_counter() - t0, tokens
+
+
+def cpu_baseline(x: kin.PrefillInputs, target_s: float = 10.0):
+    import oracle
+    cores = oracle.max_threads()
+    probe_tokens = 256
+    dt, _ = oracle_prefill_sample(x, probe_tokens)
+    tokens = int(min(x.total_T, max(probe_tokens, probe_tokens * target_s / max(dt, 1e-6))))
+    tokens = max(64, (tokens // 64) * 64)
+    dt, tokens = oracle_prefill_sample(x, tokens)
+    return {"value": tokens / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"first {tokens} of 8192 tokens x 32 heads of prefill_bf16_T8192_H32, fp64, "
+                      f"{cores} OpenMP threads over (sequence, head) pairs, {dt:.1f} s"}
+
+
+# ---------------------------------------------------------------- GPU arm
+def bench_gpu(args, world, rank, local):
+    from gated_delta_rule_152_b200 import kda
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    hbm, bf16, bf16_sus, peak_src = load_peaks()
+    stream = torch.cuda.current_stream(dev)
+
+    # ---------------- prefill (8K-token workload) --------------------------
+    x = kin.make_prefill(kin.PREFILL_8K)
+    xd = x.to(dev)
+    T, H = x.total_T, x.heads
+    o = torch.empty(T, H, D, device=dev)
+    sT = torch.empty(1, H, D, D, device=dev)
+    ws = torch.empty(max(kda.kda_chunk_fwd_workspace_size(1, T, H), 256), dtype=torch.uint8, device=dev)
+
+    def step():
+        kda.kda_chunk_fwd(xd.q, xd.k, xd.v, xd.g, xd.beta, xd.cu_seqlens, initial_state=None,
+                          final_state=sT, o=o, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clk = clocks.stop()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    prefill_tok_s = world * T / (ms / 1e3)
+    bytes_per_launch = T * H * PREFILL_BYTES_PER_TOKEN_HEAD + H * STATE_BYTES
+    achieved_gbs = bytes_per_launch / (ms / 1e3) / 1e9
+    flops_per_launch = T * H * PREFILL_FLOPS_PER_TOKEN_HEAD
+    tf32_peak = bf16 * TF32_OVER_BF16
+    achieved_tflops = flops_per_launch / (ms / 1e3) / 1e12
+
+    # end to end: pinned host inputs -> device, call, o + final state -> host
+    pin = lambda t: t.pin_memory()
+    hq, hk, hv, hg, hb, hcu = (pin(t) for t in (x.q, x.k, x.v, x.g, x.beta, x.cu_seqlens))
+    ho = torch.empty(T, H, D).pin_memory()
+    hs = torch.empty(1, H, D, D).pin_memory()
+    dq, dk, dv, dg, db, dcu = (torch.empty_like(t, device=dev) for t in (hq, hk, hv, hg, hb, hcu))
+
+    def e2e_step():
+        for d_, h_ in ((dq, hq), (dk, hk), (dv, hv), (dg, hg), (db, hb), (dcu, hcu)):
+            d_.copy_(h_, non_blocking=True)
+        kda.kda_chunk_fwd(dq, dk, dv, dg, db, dcu, final_state=sT, o=o, workspace=ws, stream=stream)
+        ho.copy_(o, non_blocking=True)
+        hs.copy_(sT, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hg, hb, hcu))
+    d2h = ho.numel() * 4 + hs.numel() * 4
+    del xd, dq, dk, dv, dg, db
+    torch.cuda.empty_cache()
+
+    # ---------------- decode (256 seq x 34 layers) -------------------------
+    spec = kin.DECODE_256x34
+    L = spec.layers if not args.quick else 4
+    N = spec.n_seqs
+    states = torch.empty(L, N, spec.heads, D, D, device=dev)
+
+    def fill(layer):   # each layer slab has its own seed; drawn on the host in parallel
+        states[layer].copy_(kin.make_decode_state(spec, layer))
+        return layer
+
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as pool:
+        list(pool.map(fill, range(L)))
+    torch.cuda.synchronize(dev)
+    toks = [kin.make_decode_tokens(spec, layer).to(dev) for layer in range(L)]
+    od = torch.empty(N, spec.heads, D, device=dev)
+
+    def dstep(i):
+        t = toks[i % L]
+        kda.kda_decode_step(t.q, t.k, t.v, t.g, t.beta, states[i % L], o=od, stream=stream)
+
+    dsteps = max(args.steps, L)
+    for i in range(max(args.warmup, 3)):
+        dstep(i)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for i in range(dsteps):
+        dstep(i)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    dms = max_over_ranks(e0.elapsed_time(e1) / dsteps, world)
+    dec_rate = world * N / (dms / 1e3)
+    dec_bytes = N * spec.heads * DECODE_BYTES_PER_SEQ_HEAD
+    dec_gbs = dec_bytes / (dms / 1e3) / 1e9
+    del states
+    torch.cuda.empty_cache()
+
+    line = {
+        "metric": METRIC,
+        "value": prefill_tok_s,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "tf32",
+        "data": "synthetic (seeded; no dataset or weights involved)",
+        "config": {"workload": kin.PREFILL_8K.name, "sequences": 1, "tokens": T, "heads": H, "d": D,
+                   "qkv_dtype": "bf16", "o_dtype": "fp32", "parallelism": f"replicas x{world}",
+                   "l2": "inputs 471 MB > 126 MB L2, no flush"},
+        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved_gbs / hbm, "traffic": None,
+                     "peak_source": f"{peak_src} hbm_gbs",
+                     "bytes_per_launch": bytes_per_launch,
+                     "tensor": {"achieved_tflops": achieved_tflops, "peak_tflops_tf32": tf32_peak,
+                                "frac": achieved_tflops / tf32_peak,
+                                "flops_per_launch": flops_per_launch}},
+        "decode": {"workload": spec.name, "value": dec_rate, "unit": "seq-steps/s/layer",
+                   "ms_per_call": dms, "layers_rotated": L,
+                   "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": hbm, "unit": "GB/s",
+                                "frac": dec_gbs / hbm, "bytes_per_launch": dec_bytes}},
+        "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps * 2 + dsteps,
+        "clocks": clk,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(x)
+    return line
+
+
+def bench_reference(args, world, rank):
+    """The reference arm: the fp64 oracle on the host cores, same metric."""
+    if rank != 0:
+        return None
+    import oracle
+    x = kin.make_prefill(kin.PREFILL_8K)
+    tokens = args.ref_tokens
+    for _ in range(args.warmup):
+        oracle_prefill_sample(x, 64)
+    t_total = 0.0
+    for _ in range(args.steps):
+        dt, _ = oracle_prefill_sample(x, tokens)
+        t_total += dt
+    rate = tokens * args.steps / t_total
+    cores = oracle.max_threads()
+    sample = (f"first {tokens} of 8192 tokens x 32 heads of prefill_bf16_T8192_H32 per step, fp64, "
+              f"{cores} OpenMP threads")
+    return {
+        "impl": "reference", "metric": METRIC, "value": rate, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)",
+        "config": {"workload": kin.PREFILL_8K.name, "sequences": 1, "tokens": 8192, "heads": 32, "d": D},
+        "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--ref-tokens", type=int, default=1024)
+    ap.add_argument("--quick", action="store_true", help="decode over 4 layer slabs instead of 34")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    world, rank, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            line = bench_reference(args, world, rank)
+        else:
+            line = bench_gpu(args, world, rank, local)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -122,14 +122,17 @@ def _gen(seed: int) -> torch.Generator:
 
 
 def _decay(x32: torch.Tensor, kind: str) -> torch.Tensor:
-    x = x32.double()
-    if kind == "logsigmoid":
-        g = torch.nn.functional.logsigmoid(x)
-    elif kind == "neg_softplus":
-        g = -torch.nn.functional.softplus(x)
-    else:
+    """g from its fp32 source draw, evaluated in fp64 and rounded to fp32, in
+    place and in slices so large workloads do not need an fp64 copy."""
+    if kind not in ("logsigmoid", "neg_softplus"):
         raise ValueError(f"unknown decay distribution {kind!r}")
-    return g.float()
+    flat = x32.view(-1)
+    step = 1 << 24
+    for s in range(0, flat.numel(), step):
+        x = flat[s:s + step].double()
+        g = torch.nn.functional.logsigmoid(x) if kind == "logsigmoid" else -torch.nn.functional.softplus(x)
+        flat[s:s + step] = g.float()
+    return x32
 
 
 def _decay_source(shape, kind: str, gen: torch.Generator) -> torch.Tensor:

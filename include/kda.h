@@ -1,0 +1,147 @@
+/*
+ * kda.h -- C ABI of the Kimi Delta Attention (KDA) layer core for NVIDIA B200
+ * (sm_100a).  Library: gated_delta_rule_152_b200/libkda.so.
+ *
+ * The operation (page "GLM-5.3-FLASH", dimsnsums.com/models/glm-5-3-flash/
+ * attention, section "How can a layer remember without rereading?", the
+ * displayed update rule): every (sequence, head) carries a d x d state S
+ * (d = 128, rows = key channels, columns = value channels) updated per token as
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *
+ * with a per-channel decay alpha_t = exp(g_t) in (0,1]^d and write strength
+ * beta_t, and emits o_t = scale * S_t^T q_t from the updated state.  With
+ * KDA_FLAG_L2NORM_QK, q_t and k_t are first divided by sqrt(sum(x^2) + 1e-6)
+ * over the head's d channels.  Sequences and heads are independent.
+ *
+ * Conventions shared by every call:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     allocates and frees nothing.  Every pointer must be 16-byte aligned.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and is asynchronous: a KDA_OK return means the launch was
+ *     accepted, not that the kernel finished.
+ *   - Layouts are row-major and contiguous:
+ *       q, k, v, g : [tokens, H, d]      (token, head, channel)
+ *       beta       : [tokens, H]
+ *       o          : [tokens, H, d]      fp32
+ *       states     : [N, H, d, d] fp32   (sequence, head, key row, value col)
+ *   - q, k, v share one dtype (kda_dtype); g, beta, states and o are fp32.
+ *   - g = log(alpha) must be finite and <= 0.  Within one 64-token chunk the
+ *     decay a channel accumulates (-sum g) must stay below 80 for the
+ *     tensor-core path; larger decay is still finite but loses accuracy there
+ *     (use KDA_FLAG_RECURRENT, which has no such limit).
+ *   - Only d == 128 is supported (KDA_ERR_UNSUPPORTED otherwise).
+ *   - Returns KDA_OK (0) or a negative kda_status.  Host-side checks run
+ *     before anything is enqueued; on an error nothing is launched.
+ */
+#ifndef KDA_H
+#define KDA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KDA_API __attribute__((visibility("default")))
+#else
+#define KDA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *kda_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = -1, /* NULL required pointer, negative size, bad cu_seqlens length */
+    KDA_ERR_UNSUPPORTED = -2, /* d != 128, unsupported dtype or flag, device not sm_100 */
+    KDA_ERR_MISALIGNED = -3,  /* a pointer is not 16-byte aligned */
+    KDA_ERR_WORKSPACE = -4,   /* workspace NULL or smaller than kda_chunk_fwd_workspace_size() */
+    KDA_ERR_CUDA = -5         /* a CUDA runtime call or kernel launch failed */
+} kda_status;
+
+typedef enum { KDA_DTYPE_BF16 = 0, KDA_DTYPE_FP32 = 1 } kda_dtype;
+
+enum {
+    /* L2-normalise q and k per token and head inside the kernel. */
+    KDA_FLAG_L2NORM_QK = 1u,
+    /* Force the token-by-token fp32 kernel for prefill (default for FP32
+     * inputs; for BF16 inputs the chunked tensor-core kernel is the default). */
+    KDA_FLAG_RECURRENT = 2u
+};
+
+/* Device-side error bits, OR-ed into the first 32-bit word of the workspace by
+ * kda_chunk_fwd and readable with kda_workspace_error(). */
+enum {
+    KDA_DEVERR_CU_SEQLENS = 1u, /* cu_seqlens not non-decreasing in [0, total_T]; the
+                                   offending sequences were treated as empty */
+    KDA_DEVERR_TIMEOUT = 2u     /* a bounded wait inside a kernel gave up; outputs of the
+                                   affected (sequence, head) are undefined */
+};
+
+/*
+ * Bytes of device workspace kda_chunk_fwd needs for these sizes (the
+ * error word plus the sequence schedule).  Returns 0 for invalid sizes.
+ */
+KDA_API size_t kda_chunk_fwd_workspace_size(int32_t N, int64_t total_T, int32_t H, int32_t d,
+                                    kda_dtype dt);
+
+/*
+ * Prefill over N packed variable-length sequences (the chunked form of the
+ * update rule above; the page gives only the per-token rule, the 64-token
+ * chunking is this library's and reproduces the per-token result).
+ *
+ *   q, k, v       [total_T, H, d]  dtype dt
+ *   g             [total_T, H, d]  fp32, log(alpha), finite, <= 0
+ *   beta          [total_T, H]     fp32
+ *   cu_seqlens    [N + 1] int32 DEVICE array: cu[0] = 0, non-decreasing,
+ *                 cu[N] = total_T; sequence n is tokens cu[n] .. cu[n+1]-1.
+ *                 Not checked on the host; an inconsistent array sets
+ *                 KDA_DEVERR_CU_SEQLENS in the workspace and the offending
+ *                 sequences are skipped.
+ *   scale         o = scale * S^T q.
+ *   flags         KDA_FLAG_*.
+ *   initial_state [N, H, d, d] fp32 or NULL (= zeros).
+ *   final_state   [N, H, d, d] fp32 or NULL (not written).  May alias
+ *                 initial_state (in-place continuation).  A zero-length
+ *                 sequence gets final = initial.
+ *   o             [total_T, H, d] fp32, written for every token.
+ *   workspace     device scratch of at least
+ *                 kda_chunk_fwd_workspace_size(...) bytes; its first word is
+ *                 cleared by this call and receives KDA_DEVERR_* bits.  Calls
+ *                 that share a workspace must be stream-ordered.
+ */
+KDA_API int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g,
+                  const float *beta, const int32_t *cu_seqlens, int32_t N, int64_t total_T,
+                  int32_t H, int32_t d, kda_dtype dt, float scale, uint32_t flags,
+                  const float *initial_state, float *final_state, float *o, void *workspace,
+                  size_t workspace_bytes, kda_stream_t stream);
+
+/*
+ * One decode step for N sequences: each (sequence, head) state advances by
+ * exactly one token, in place, and o receives that token's output
+ * (o = scale * S_new^T q).  Same rule as above with T = 1.
+ *
+ *   q, k, v  [N, H, d] dtype dt      g [N, H, d] fp32      beta [N, H] fp32
+ *   state    [N, H, d, d] fp32, read and overwritten
+ *   o        [N, H, d] fp32
+ */
+KDA_API int kda_decode_step(const void *q, const void *k, const void *v, const float *g,
+                    const float *beta, float *state, float *o, int32_t N, int32_t H,
+                    int32_t d, kda_dtype dt, float scale, uint32_t flags,
+                    kda_stream_t stream);
+
+/*
+ * Copy the device error word of a workspace used by kda_chunk_fwd to *out
+ * (synchronises `stream`).  Returns KDA_OK or KDA_ERR_*.
+ */
+KDA_API int kda_workspace_error(const void *workspace, uint32_t *out, kda_stream_t stream);
+
+/* Static English description of a kda_status value. */
+KDA_API const char *kda_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KDA_H */

@@ -1,0 +1,105 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+declared in include/kda.h, and rejects bad arguments on the host before any
+CUDA call (fake, never-dereferenced pointers are enough for that)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_delta_rule_152_b200 import kda
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kda.h")
+
+A = 0x10000          # a fake 16-byte-aligned device address
+MIS = 0x10008        # misaligned
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^[A-Za-z_][\w\s\*]*?\b(kda_\w+)\s*\(", text, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from gated_delta_rule_152_b200 import build
+    build.build()
+    return kda.load_library()
+
+
+def test_library_exports_every_declared_function(lib):
+    names = header_functions()
+    assert set(names) >= {"kda_chunk_fwd", "kda_decode_step", "kda_chunk_fwd_workspace_size",
+                          "kda_status_string", "kda_workspace_error"}
+    for name in names:
+        assert hasattr(lib, name), name
+    assert set(kda.EXPORTED) <= set(names)
+
+
+def test_status_strings(lib):
+    assert kda.kda_status_string(0) == "ok"
+    for s in range(-5, 0):
+        assert kda.kda_status_string(s) not in ("ok", "unknown status")
+    assert kda.kda_status_string(-99) == "unknown status"
+
+
+def test_workspace_size(lib):
+    assert lib.kda_chunk_fwd_workspace_size(16, 1000, 32, 128, 0) >= 256 + 64
+    assert lib.kda_chunk_fwd_workspace_size(16, 1000, 32, 64, 0) == 0
+    assert lib.kda_chunk_fwd_workspace_size(-1, 1000, 32, 128, 0) == 0
+
+
+def _chunk(lib, **kw):
+    args = dict(q=A, k=A, v=A, g=A, beta=A, cu=A, N=2, T=100, H=4, d=128, dt=0, scale=1.0, flags=1,
+                s0=None, sT=None, o=A, ws=A, wsb=4096, stream=None)
+    args.update(kw)
+    return lib.kda_chunk_fwd(args["q"], args["k"], args["v"], args["g"], args["beta"], args["cu"],
+                             args["N"], args["T"], args["H"], args["d"], args["dt"], args["scale"],
+                             args["flags"], args["s0"], args["sT"], args["o"], args["ws"], args["wsb"],
+                             args["stream"])
+
+
+def test_chunk_fwd_host_validation(lib):
+    assert _chunk(lib, d=64) == kda.KDA_ERR_UNSUPPORTED
+    assert _chunk(lib, dt=7) == kda.KDA_ERR_UNSUPPORTED
+    assert _chunk(lib, flags=0x80) == kda.KDA_ERR_UNSUPPORTED
+    assert _chunk(lib, N=-1) == kda.KDA_ERR_INVALID_ARG
+    assert _chunk(lib, H=0) == kda.KDA_ERR_INVALID_ARG
+    assert _chunk(lib, T=1 << 31) == kda.KDA_ERR_INVALID_ARG
+    assert _chunk(lib, cu=None) == kda.KDA_ERR_INVALID_ARG
+    assert _chunk(lib, q=None) == kda.KDA_ERR_INVALID_ARG
+    assert _chunk(lib, o=None) == kda.KDA_ERR_INVALID_ARG
+    assert _chunk(lib, g=MIS) == kda.KDA_ERR_MISALIGNED
+    assert _chunk(lib, s0=MIS) == kda.KDA_ERR_MISALIGNED
+    assert _chunk(lib, ws=None) == kda.KDA_ERR_WORKSPACE
+    assert _chunk(lib, wsb=16) == kda.KDA_ERR_WORKSPACE
+
+
+def test_decode_host_validation(lib):
+    def dec(**kw):
+        a = dict(q=A, k=A, v=A, g=A, beta=A, s=A, o=A, N=4, H=2, d=128, dt=0, scale=1.0, flags=1)
+        a.update(kw)
+        return lib.kda_decode_step(a["q"], a["k"], a["v"], a["g"], a["beta"], a["s"], a["o"], a["N"],
+                                   a["H"], a["d"], a["dt"], a["scale"], a["flags"], None)
+    assert dec(d=100) == kda.KDA_ERR_UNSUPPORTED
+    assert dec(flags=2) == kda.KDA_ERR_UNSUPPORTED   # the recurrent flag is prefill-only
+    assert dec(N=-3) == kda.KDA_ERR_INVALID_ARG
+    assert dec(s=None) == kda.KDA_ERR_INVALID_ARG
+    assert dec(o=MIS) == kda.KDA_ERR_MISALIGNED
+    assert dec(N=0) == kda.KDA_OK                    # nothing to do, nothing launched
+
+
+def test_valid_call_without_gpu_reports_cuda_error(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("has a GPU")
+    assert _chunk(lib) in (kda.KDA_ERR_CUDA, kda.KDA_ERR_UNSUPPORTED)
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+    x = torch.zeros(4, 2, 128)
+    with pytest.raises(ValueError):
+        kda.kda_chunk_fwd(x, x, x, x, torch.zeros(4, 2), torch.tensor([0, 4], dtype=torch.int32))

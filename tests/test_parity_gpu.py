@@ -1,0 +1,219 @@
+"""GPU parity: the CUDA library against the fp64 oracle, element by element.
+
+Bar (both o and the final state, separately): max|gpu - oracle| <= tol x
+RMS(oracle), tol = 1e-4 for fp32 q/k/v and 2e-2 for bf16 q/k/v.  Small cases
+span several 64-token chunks and ragged tails; the five named workloads run at
+full size on the GPU and are compared on every output the oracle can afford
+(all of them, or a subset of heads for the two 130K-token workloads).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_delta_rule_152_b200 import inputs as kin
+from gated_delta_rule_152_b200 import kda
+
+pytestmark = pytest.mark.gpu
+
+TOL_FP32 = 1e-4
+TOL_BF16 = 2e-2
+
+
+def err_ratio(gpu: torch.Tensor, ref: np.ndarray) -> float:
+    g = gpu.detach().double().cpu().numpy()
+    rms = float(np.sqrt(np.mean(ref * ref)))
+    return float(np.abs(g - ref).max()) / max(rms, 1e-300)
+
+
+def assert_close(gpu, ref, tol, what):
+    r = err_ratio(gpu, ref)
+    assert np.isfinite(gpu.detach().cpu().numpy()).all(), f"{what}: non-finite output"
+    assert r <= tol, f"{what}: max|err| = {r:.3e} x RMS(ref) > {tol:g}"
+    return r
+
+
+def run_both(x: kin.PrefillInputs, recurrent=False, scale=1.0, l2norm=True, heads=None):
+    dev = torch.device("cuda")
+    xd = x.to(dev)
+    o, sT = kda.kda_chunk_fwd(xd.q, xd.k, xd.v, xd.g, xd.beta, xd.cu_seqlens, scale=scale,
+                              l2norm=l2norm, initial_state=xd.initial_state, recurrent=recurrent)
+    torch.cuda.synchronize()
+    sel = slice(None) if heads is None else list(heads)
+    s0 = None if x.initial_state is None else x.initial_state[:, sel].contiguous()
+    o_ref, s_ref = oracle.kda_forward(x.q[:, sel].contiguous(), x.k[:, sel].contiguous(),
+                                      x.v[:, sel].contiguous(), x.g[:, sel].contiguous(),
+                                      x.beta[:, sel].contiguous(), x.cu_seqlens, s0, scale=scale,
+                                      l2norm=l2norm)
+    return o[:, sel], sT[:, sel], o_ref, s_ref
+
+
+def test_tiny_fp32_workload_full():
+    x = kin.make_prefill(kin.TINY_FP32)
+    o, s, o_ref, s_ref = run_both(x)
+    assert_close(o, o_ref, TOL_FP32, "o")
+    assert_close(s, s_ref, TOL_FP32, "final state")
+
+
+@pytest.mark.parametrize("lengths", [[1], [63], [64], [65], [200], [0, 5, 64, 130, 1, 257]])
+def test_recurrent_kernel_bf16(lengths):
+    x = kin.make_custom_prefill(11, lengths, heads=3, init_state_std=0.02)
+    o, s, o_ref, s_ref = run_both(x, recurrent=True, scale=0.75)
+    assert_close(o, o_ref, TOL_FP32 if sum(lengths) else TOL_FP32, "o")   # fp32 arithmetic throughout
+    assert_close(s, s_ref, TOL_FP32, "final state")
+
+
+@pytest.mark.parametrize("lengths", [[1], [63], [64], [65], [200], [1000]])
+def test_chunk_kernel_single_sequence(lengths):
+    x = kin.make_custom_prefill(21, lengths, heads=2, init_state_std=0.02)
+    o, s, o_ref, s_ref = run_both(x)
+    assert_close(o, o_ref, TOL_BF16, "o")
+    assert_close(s, s_ref, TOL_BF16, "final state")
+
+
+def test_chunk_kernel_varlen_with_empty_and_ragged():
+    x = kin.make_custom_prefill(22, [0, 5, 64, 130, 1, 257, 0, 128], heads=3, init_state_std=0.05)
+    o, s, o_ref, s_ref = run_both(x, scale=0.5)
+    assert_close(o, o_ref, TOL_BF16, "o")
+    assert_close(s, s_ref, TOL_BF16, "final state")
+    # empty sequences: final state equals the initial state exactly
+    for n in (0, 6):
+        assert torch.equal(s[n].cpu(), x.initial_state[n])
+
+
+def test_chunk_kernel_without_l2norm():
+    x = kin.make_custom_prefill(23, [150, 70], heads=2, init_state_std=0.02)
+    # keep |k| near 1 so the un-normalised recurrence stays bounded
+    x.q = (x.q.float() / 11.3).to(torch.bfloat16)
+    x.k = (x.k.float() / 11.3).to(torch.bfloat16)
+    o, s, o_ref, s_ref = run_both(x, l2norm=False)
+    assert_close(o, o_ref, TOL_BF16, "o")
+    assert_close(s, s_ref, TOL_BF16, "final state")
+
+
+def test_chunk_kernel_strong_decay():
+    # per-chunk decay per channel around 40 nats (inside the tensor-core path's range)
+    x = kin.make_custom_prefill(24, [300], heads=2, init_state_std=0.02)
+    x.g = x.g * 8.0
+    o, s, o_ref, s_ref = run_both(x)
+    assert_close(o, o_ref, TOL_BF16, "o")
+    assert_close(s, s_ref, TOL_BF16, "final state")
+
+
+def test_chunk_kernel_in_place_state():
+    x = kin.make_custom_prefill(25, [100, 33], heads=2, init_state_std=0.02)
+    dev = torch.device("cuda")
+    xd = x.to(dev)
+    state = xd.initial_state.clone()
+    o, s = kda.kda_chunk_fwd(xd.q, xd.k, xd.v, xd.g, xd.beta, xd.cu_seqlens,
+                             initial_state=state, final_state=state)
+    torch.cuda.synchronize()
+    o_ref, s_ref = oracle.kda_forward(x.q, x.k, x.v, x.g, x.beta, x.cu_seqlens, x.initial_state)
+    assert s.data_ptr() == state.data_ptr()
+    assert_close(state, s_ref, TOL_BF16, "in-place final state")
+    assert_close(o, o_ref, TOL_BF16, "o")
+
+
+def test_chunk_kernel_split_resume_matches_single_call():
+    x = kin.make_custom_prefill(26, [400], heads=2, init_state_std=0.02)
+    dev = torch.device("cuda")
+    xd = x.to(dev)
+    o_full, s_full = kda.kda_chunk_fwd(xd.q, xd.k, xd.v, xd.g, xd.beta, xd.cu_seqlens,
+                                       initial_state=xd.initial_state)
+    cut = 150
+    cu1 = torch.tensor([0, cut], dtype=torch.int32, device=dev)
+    cu2 = torch.tensor([0, 400 - cut], dtype=torch.int32, device=dev)
+    o1, s1 = kda.kda_chunk_fwd(xd.q[:cut], xd.k[:cut], xd.v[:cut], xd.g[:cut], xd.beta[:cut], cu1,
+                               initial_state=xd.initial_state)
+    o2, s2 = kda.kda_chunk_fwd(xd.q[cut:].contiguous(), xd.k[cut:].contiguous(), xd.v[cut:].contiguous(),
+                               xd.g[cut:].contiguous(), xd.beta[cut:].contiguous(), cu2, initial_state=s1)
+    torch.cuda.synchronize()
+    o_ref, s_ref = oracle.kda_forward(x.q, x.k, x.v, x.g, x.beta, x.cu_seqlens, x.initial_state)
+    assert_close(torch.cat([o1, o2]), o_ref, TOL_BF16, "split o")
+    assert_close(s2, s_ref, TOL_BF16, "split final state")
+
+
+def test_zero_tokens_copies_initial_state():
+    dev = torch.device("cuda")
+    H = 2
+    s0 = torch.randn(3, H, 128, 128, device=dev)
+    e = torch.empty(0, H, 128, device=dev, dtype=torch.bfloat16)
+    cu = torch.zeros(4, dtype=torch.int32, device=dev)
+    o, s = kda.kda_chunk_fwd(e, e, e, e.float(), torch.empty(0, H, device=dev), cu, initial_state=s0)
+    torch.cuda.synchronize()
+    assert o.numel() == 0 and torch.equal(s, s0)
+
+
+def test_bad_cu_seqlens_flags_error_and_skips_only_that_sequence():
+    x = kin.make_custom_prefill(27, [40, 30, 50], heads=2)
+    dev = torch.device("cuda")
+    xd = x.to(dev)
+    bad = torch.tensor([0, 40, 20, 120], dtype=torch.int32, device=dev)   # sequence 1 decreasing
+    ws = torch.zeros(1024, dtype=torch.uint8, device=dev)
+    o = torch.zeros(120, 2, 128, device=dev)
+    o, s = kda.kda_chunk_fwd(xd.q, xd.k, xd.v, xd.g, xd.beta, bad, o=o, workspace=ws)
+    assert kda.kda_workspace_error(ws) & kda.KDA_DEVERR_CU_SEQLENS
+    o_ref, _ = oracle.kda_forward(x.q[:40], x.k[:40], x.v[:40], x.g[:40], x.beta[:40], [0, 40])
+    assert_close(o[:40], o_ref, TOL_BF16, "o of the valid sequence")
+    ws.zero_()
+    kda.kda_chunk_fwd(xd.q, xd.k, xd.v, xd.g, xd.beta, xd.cu_seqlens, workspace=ws)
+    assert kda.kda_workspace_error(ws) == 0
+
+
+def test_prefill_8k_workload_full():
+    x = kin.make_prefill(kin.PREFILL_8K)
+    o, s, o_ref, s_ref = run_both(x)
+    assert_close(o, o_ref, TOL_BF16, "o")
+    assert_close(s, s_ref, TOL_BF16, "final state")
+
+
+def test_prefill_8k_recurrent_path_matches_oracle():
+    x = kin.make_prefill(kin.PREFILL_8K, heads=4)
+    o, s, o_ref, s_ref = run_both(x, recurrent=True)
+    assert_close(o, o_ref, TOL_FP32, "o")
+    assert_close(s, s_ref, TOL_FP32, "final state")
+
+
+def test_prefill_128k_workload_sampled_heads():
+    x = kin.make_prefill(kin.PREFILL_128K)
+    o, s, o_ref, s_ref = run_both(x, heads=[0, 13, 31])
+    assert_close(o, o_ref, TOL_BF16, "o")
+    assert_close(s, s_ref, TOL_BF16, "final state")
+
+
+def test_varlen_16_workload_sampled_heads():
+    x = kin.make_prefill(kin.VARLEN_16)
+    o, s, o_ref, s_ref = run_both(x, heads=[0, 7, 31])
+    assert_close(o, o_ref, TOL_BF16, "o")
+    assert_close(s, s_ref, TOL_BF16, "final state")
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_decode_small(dtype):
+    spec = kin.DecodeSpec("small", 77, 5, 1, 3, dtype)
+    tok = kin.make_decode_tokens(spec, 0)
+    st = kin.make_decode_state(spec, 0)
+    dev = torch.device("cuda")
+    td = tok.to(dev)
+    sd = st.to(dev)
+    o = kda.kda_decode_step(td.q, td.k, td.v, td.g, td.beta, sd, scale=0.9)
+    torch.cuda.synchronize()
+    o_ref, s_ref = oracle.kda_decode(tok.q, tok.k, tok.v, tok.g, tok.beta, st, scale=0.9)
+    assert_close(o, o_ref, TOL_FP32, "o")
+    assert_close(sd, s_ref, TOL_FP32, "state")
+
+
+def test_decode_workload_full_layer_two_steps():
+    spec = kin.DECODE_256x34
+    dev = torch.device("cuda")
+    st = kin.make_decode_state(spec, 5)
+    sd = st.to(dev)
+    ref_state = st
+    for step in range(2):
+        tok = kin.make_decode_tokens(spec, 5 + 100 * step)
+        td = tok.to(dev)
+        o = kda.kda_decode_step(td.q, td.k, td.v, td.g, td.beta, sd)
+        torch.cuda.synchronize()
+        o_ref, ref_state = oracle.kda_decode(tok.q, tok.k, tok.v, tok.g, tok.beta, ref_state)
+        assert_close(o, o_ref, TOL_BF16, f"o step {step}")
+        assert_close(sd, ref_state, TOL_BF16, f"state step {step}")
