@@ -10,34 +10,34 @@
 // (rows = key channels), Gamma_r = g_0 + ... + g_r per channel and
 // Gamma_C = Gamma_{L-1} (L = tokens in the chunk):
 //     E_r = exp(Gamma_r - Gamma_C) (>= 1),   F_r = exp(Gamma_C - Gamma_r) (<= 1)
-//     Kt = k_r E_r,  Qt = scale q_r E_r,  Kb = k_r F_r                 (prep)
-//     [A ; P] = [Kt ; Qt] Kb^T   (A_ri = sum_c k_rc k_ic e^{Gamma_rc - Gamma_ic})
-//     M = strict_lower(diag(beta) A),  T' = (I + M)^-1 diag(beta)   (UT transform)
-//     P = lower_incl(P)
-//     U = T' V,  W' = T' Kt                                          (WY products)
+//     Kt = k_r E_r,  Qt = scale q_r E_r,  Kb = k_r F_r                  (prep)
 //     St = Diag(exp(Gamma_C)) S                     (state decayed to chunk end)
-//     delta = U - W' St,  O = Qt St + P delta,  S_next = St + Kb^T delta
-// Unrolling the per-token rule inside the chunk gives (I + M) delta =
-// diag(beta)(V - K~ S) with K~_r = k_r exp(Gamma_r) = Kt_r exp(Gamma_C), which
-// is the triangular system above; O and S_next follow the same way.  Every
-// exponent is taken relative to the chunk end, so all factors are finite as
-// long as a channel's decay inside one chunk, -sum(g), stays below ~87.
+//     [A ; P] = [Kt ; Qt] Kb^T   (A_ri = sum_c k_rc k_ic e^{Gamma_rc - Gamma_ic})
+//     [Y ; Z] = [Kt ; Qt] St     (Y_r = k_r^T Diag(e^{Gamma_r}) S, Z_r likewise for q)
+//     M = strict_lower(diag(beta) A),  T' = (I + M)^-1 diag(beta)   (UT transform)
+//     delta = T' (V - Y),   O = Z + lower_incl(P) delta,   S_next = St + Kb^T delta
+// Unrolling the per-token rule inside the chunk gives the triangular system
+// (I + M) delta = diag(beta) (V - Y) for the rank-one corrections delta_r,
+// from which the outputs and the end state follow.  Every exponent is taken
+// relative to the chunk end, so all factors are finite as long as a channel's
+// decay inside one chunk, -sum(g), stays below ~87.
 //
 // Precision: operands are rounded to tf32 (10-bit mantissa) and accumulated in
 // fp32.  bf16 operands were measured (CPU emulation against the fp64 oracle)
 // to exceed a 2e-2 x RMS max-error budget on the 8K-token workload; tf32 stays
-// near 5e-3.  The state stays fp32 between chunks.
+// near 5e-3.  The state stays fp32 between chunks (in tensor memory).
 //
 // Work decomposition: one CTA per (sequence, head, 32-column value slice); the
 // value columns of S evolve independently, so four CTAs share a head and each
-// recomputes the head-level chunk quantities (A, P, T', W').  Every MMA is
-// M = 128 by stacking two 64-row operands:
-//     [Kt ; Qt] x Kb^T      -> A (lanes 0-63), P (lanes 64-127)
-//     [T' ; P]  x V         -> U (lanes 0-63; lanes 64-127 unused)
-//     [T' ; P]  x Kt        -> W' (lanes 0-63; lanes 64-127 unused)
-//     [-W' ; Qt] x St       -> -W' St (lanes 0-63), Qt St (lanes 64-127)
-//     [T' ; P]  x delta     -> accumulated onto the previous: lanes 64-127 = O
-//     Kb^T      x delta     -> accumulated onto St in TMEM: S_next
+// recomputes the head-level chunk quantities (A, P, T').  Every MMA is
+// M = 128 (two 64-row operands stacked) with both operands K-major in shared
+// memory:
+//     [Kt ; Qt] x Kb^T     -> A (lanes 0-63), P (lanes 64-127)
+//     [Kt ; Qt] x St       -> Y (lanes 0-63), Z (lanes 64-127)
+//     [T' ; P]  x V        -> T'V (lanes 0-63; lanes 64-127 unused)
+//     [T' ; P]  x (-Y)     -> accumulated: lanes 0-63 = delta
+//     [T' ; P]  x delta    -> accumulated onto [Y ; Z]: lanes 64-127 = O
+//     Kb^T      x delta    -> accumulated onto St in TMEM: S_next
 // Block: 256 threads (8 warps); thread 0 issues TMA and MMA.  A warp may only
 // touch tensor-memory lanes 32*(warp%4) .. +31.
 #include "kda_common.cuh"
@@ -54,68 +54,68 @@ constexpr int kNV = 32;         // value columns per CTA
 constexpr int kSplit = kD / kNV;
 constexpr int kThreads = 256;
 
-// Shared memory (byte offsets from a 1024-aligned base).  All MMA operand
-// tiles use 128-byte rows with the 128-byte swizzle (see sm100.cuh).
-constexpr uint32_t OFF_XQ = 0;        // 64 KB: 4 K-blocks (channels 32kb..) x 128 rows:
-                                      //   rows 0-63 Kt (later -W'), rows 64-127 Qt
-constexpr uint32_t OFF_KB = 65536;    // 32 KB: 4 K-blocks x 64 rows: Kb
-constexpr uint32_t OFF_TP = 98304;    // 32 KB: 2 K-blocks (tokens 32kb..) x 128 rows:
-                                      //   rows 0-63 T (fp32 while solving, then T'), rows 64-127 P
-constexpr uint32_t OFF_SB = 131072;   // 16 KB: 128 rows (key channel) x 32 value cols: St;
-                                      //   during the triangular solve: M (64 x 64 fp32)
-constexpr uint32_t OFF_DL = 147456;   // 8 KB: 64 rows (token) x 32 value cols: delta;
-                                      //   during prep: Gamma exchange; during the solve: temps
-constexpr uint32_t OFF_VB = 155648;   // 8 KB: 64 rows (token) x 32 value cols: V slice
-constexpr uint32_t OFF_RQ = 163840;   // 16 KB: raw q [64][128] bf16 (TMA destination)
-constexpr uint32_t OFF_RK = 180224;   // 16 KB: raw k
-constexpr uint32_t OFF_MISC = 196608; // beta[64], exp(Gamma_C)[128], barriers, TMEM address
+// Shared memory (byte offsets from a 1024-aligned base).  Every MMA operand
+// is K-major with 128-byte rows (32 tf32 elements of K) and the 128-byte
+// swizzle (sm100.cuh); further K elements live in further "K-blocks".
+constexpr uint32_t OFF_XQ = 0;         // 64 KB: [Kt ; Qt], 128 rows (token, token) x 128 channels
+                                       //   = 4 K-blocks x 16 KB.  After the first MMA pair it is
+                                       //   dead and holds the triangular solve's scratch.
+constexpr uint32_t OFF_KB = 65536;     // 32 KB: Kb, 64 rows (token) x 128 channels = 4 K-blocks x 8 KB.
+                                       //   Also the TMA destination of the next chunk's raw q, k.
+constexpr uint32_t OFF_KBT = 98304;    // 32 KB: Kb^T, 128 rows (channel) x 64 tokens = 2 K-blocks x 16 KB
+constexpr uint32_t OFF_TP = 131072;    // 32 KB: [T' ; P], 128 rows x 64 tokens = 2 K-blocks x 16 KB
+constexpr uint32_t OFF_ST = 163840;    // 16 KB: St^T, 32 rows (value col) x 128 channels = 4 x 4 KB
+constexpr uint32_t OFF_VT = 180224;    // 8 KB: V^T, 32 rows x 64 tokens = 2 x 4 KB
+constexpr uint32_t OFF_YT = 188416;    // 8 KB: (-Y)^T, later delta^T; during prep the Gamma exchange
+constexpr uint32_t OFF_MISC = 196608;  // beta[64], exp(Gamma_C)[128], barriers, TMEM address
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 1024 + 1024;   // + alignment slack
 
-constexpr uint32_t KB_XQ = 16384;     // K-block strides
+constexpr uint32_t KB_XQ = 16384;      // K-block strides
 constexpr uint32_t KB_KB = 8192;
+constexpr uint32_t KB_KBT = 16384;
 constexpr uint32_t KB_TP = 16384;
+constexpr uint32_t KB_ST = 4096;
+constexpr uint32_t KB_VT = 4096;
+
+// Scratch of the triangular solve inside the dead XQ region.
+constexpr uint32_t OFF_M = OFF_XQ;             // M, 64 x 64 fp32 (row-swizzled)
+constexpr uint32_t OFF_TMP = OFF_XQ + 16384;   // block-merge temporaries, 6 KB
 
 // Tensor-memory columns (fp32 accumulators, 128 lanes each).
 constexpr uint32_t TM_AP = 0;     // 64 cols: A | P
-constexpr uint32_t TM_U = 64;     // 32 cols: U
-constexpr uint32_t TM_X = 96;     // 32 cols: -W'St | QtSt (+P delta = O)
-constexpr uint32_t TM_W = 128;    // 128 cols: W'
-constexpr uint32_t TM_S = 256;    // 32 cols: state slice (key rows x 32 value cols)
-constexpr uint32_t TM_COLS = 512;
+constexpr uint32_t TM_X = 64;     // 32 cols: Y | Z, then Z + P delta = O in lanes 64-127
+constexpr uint32_t TM_U = 96;     // 32 cols: T'V, then delta in lanes 0-63
+constexpr uint32_t TM_S = 128;    // 32 cols: state slice (key rows x 32 value cols)
+constexpr uint32_t TM_COLS = 256;
 
-constexpr uint32_t ID_AP = idesc_tf32(128, 64, false, false);
-constexpr uint32_t ID_U = idesc_tf32(128, 32, false, true);
-constexpr uint32_t ID_W = idesc_tf32(128, 128, false, true);
-constexpr uint32_t ID_X = idesc_tf32(128, 32, false, true);
-constexpr uint32_t ID_S = idesc_tf32(128, 32, true, true);
+constexpr uint32_t ID_N64 = idesc_tf32(128, 64, false, false);
+constexpr uint32_t ID_N32 = idesc_tf32(128, 32, false, false);
 
-// fp32 scratch addressing inside the swizzled regions -----------------------
-// M (64 x 64 fp32) in the St region: 16 float4 chunks per row, chunk position
-// XOR-ed with the row so column-wise accesses of 32 rows hit distinct banks.
+// M (64 x 64 fp32): 16 float4 chunks per row, chunk position XOR-ed with the
+// row so that 32 rows written at the same column hit distinct banks.
 __device__ __forceinline__ float* M_at(uint8_t* smem, int r, int i) {
-    return reinterpret_cast<float*>(smem + OFF_SB) + r * 64 + ((((i >> 2) ^ (r & 15))) << 2) + (i & 3);
+    return reinterpret_cast<float*>(smem + OFF_M) + r * 64 + (((i >> 2) ^ (r & 15)) << 2) + (i & 3);
 }
-// T / T' (rows 0-63 of the [T' ; P] operand, K-major, tokens along K).
+// T / T' in rows 0-63 of the [T' ; P] operand (tokens along K).
 __device__ __forceinline__ float* T_at(uint8_t* smem, int r, int i) {
     return reinterpret_cast<float*>(smem + OFF_TP + (i >> 5) * KB_TP + sw128_off(r, (i & 31) >> 2)) + (i & 3);
+}
+// Element (row, k) of a K-major operand tile at `base` with K-block stride `kb`.
+__device__ __forceinline__ float* K_at(uint8_t* smem, uint32_t base, uint32_t kb, int row, int k) {
+    return reinterpret_cast<float*>(smem + base + (k >> 5) * kb + sw128_off(row, (k & 31) >> 2)) + (k & 3);
 }
 
 __device__ __forceinline__ void st_tf32x4(uint8_t* smem, uint32_t off, float a, float b, float c, float d) {
     *reinterpret_cast<float4*>(smem + off) = make_float4(to_tf32(a), to_tf32(b), to_tf32(c), to_tf32(d));
 }
 
-// Store 32 consecutive fp32 values (one thread's TMEM row) as tf32 into the
-// 8 chunks of swizzled row `row` of a region at byte offset `base`.
-__device__ __forceinline__ void st_row32(uint8_t* smem, uint32_t base, int row, const float (&v)[32],
-                                         float sign = 1.f) {
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-        st_tf32x4(smem, base + sw128_off(row, j), sign * v[4 * j], sign * v[4 * j + 1],
-                  sign * v[4 * j + 2], sign * v[4 * j + 3]);
-}
-
 __device__ __forceinline__ uint32_t tm_lane(uint32_t tmem, int quarter, uint32_t col) {
     return tmem + (static_cast<uint32_t>(32 * quarter) << 16) + col;
+}
+
+// K-major SW128 descriptor of K step s (8 tf32 = 32 bytes) of a tile.
+__device__ __forceinline__ uint64_t kdesc(uint32_t sb, uint32_t base, uint32_t kb_stride, int s) {
+    return sdesc_sw128(sb + base + (s >> 2) * kb_stride + (s & 3) * 32, 16, 1024);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -204,35 +204,47 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         breg = 0.f;
         if (tid < L) breg = __ldg(beta + (size_t)(t0 + tid) * H + h);
     };
+    // raw q and k tiles (64 tokens x 128 channels, bf16) into the Kb region
     auto issue_load = [&](int64_t t0) {
         mbar_arrive_expect_tx(bar_load, 2u * kC * kD * 2u);
-        tma_load_3d(smem + OFF_RQ, &tm_q, bar_load, 0, h, static_cast<int32_t>(t0));
-        tma_load_3d(smem + OFF_RK, &tm_k, bar_load, 0, h, static_cast<int32_t>(t0));
+        tma_load_3d(smem + OFF_KB, &tm_q, bar_load, 0, h, static_cast<int32_t>(t0));
+        tma_load_3d(smem + OFF_KB + kC * kD * 2, &tm_k, bar_load, 0, h, static_cast<int32_t>(t0));
     };
 
     bool ok = true;
-    uint32_t mma_phase = 0;
+    uint32_t mma_phase = 0, load_parity = 0;
     bool load_pending = false, mma_pending = false;
-    uint32_t load_parity = 0;
     if (nchunks > 0) {
         if (tid == 0) issue_load(bos);
         load_pending = true;
-        prefetch(bos, static_cast<int>((len < kC ? len : (int64_t)kC)));
+        prefetch(bos, static_cast<int>(len < kC ? len : (int64_t)kC));
     }
     tc_fence_before();
     __syncthreads();
 
     for (int c = 0; c < nchunks; ++c) {
         const int64_t t0 = bos + (int64_t)c * kC;
-        const int L = static_cast<int>((eos - t0 < kC ? eos - t0 : (int64_t)kC));
+        const int L = static_cast<int>(eos - t0 < kC ? eos - t0 : (int64_t)kC);
 
         ok = !__syncthreads_or(!mbar_wait_bounded(bar_load, c & 1));
         if (!ok) break;
         load_pending = false;
 
-        // ---------------------------------------------------------- prep
+        // ================================================== prep
         {
-            float* xch = reinterpret_cast<float*>(smem + OFF_DL);   // [8 warps][128]
+            // raw q, k of the thread's 8 rows x 4 channels into registers first:
+            // the tiles written below overwrite the raw staging area
+            uint2 qraw[8], kraw[8];
+            const uint8_t* rq = smem + OFF_KB;
+            const uint8_t* rk = smem + OFF_KB + kC * kD * 2;
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                const int r = 8 * warp + m;
+                qraw[m] = *reinterpret_cast<const uint2*>(rq + r * kD * 2 + lane * 8);
+                kraw[m] = *reinterpret_cast<const uint2*>(rk + r * kD * 2 + lane * 8);
+            }
+            // Gamma (log2 units): prefix over the thread's 8 rows, then over warps
+            float* xch = reinterpret_cast<float*>(smem + OFF_YT);   // [8 warps][128]
             float G[8][4];
 #pragma unroll
             for (int x = 0; x < 4; ++x) {
@@ -244,7 +256,7 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 }
                 xch[warp * 128 + 4 * lane + x] = run;
             }
-            __syncthreads();
+            __syncthreads();   // also: every thread has its raw q, k in registers
             float off[4] = {0.f, 0.f, 0.f, 0.f}, GC[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int w = 0; w < 8; ++w) {
@@ -258,14 +270,14 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
             if (tid < kC) beta_s[tid] = breg;
 
-            const __nv_bfloat16* rq = reinterpret_cast<const __nv_bfloat16*>(smem + OFF_RQ);
-            const __nv_bfloat16* rk = reinterpret_cast<const __nv_bfloat16*>(smem + OFF_RK);
 #pragma unroll
             for (int m = 0; m < 8; ++m) {
                 const int r = 8 * warp + m;
                 float qv[4], kv[4];
-                load4(rq + r * kD + 4 * lane, qv);
-                load4(rk + r * kD + 4 * lane, kv);
+                qv[0] = __uint_as_float(qraw[m].x << 16); qv[1] = __uint_as_float(qraw[m].x & 0xFFFF0000u);
+                qv[2] = __uint_as_float(qraw[m].y << 16); qv[3] = __uint_as_float(qraw[m].y & 0xFFFF0000u);
+                kv[0] = __uint_as_float(kraw[m].x << 16); kv[1] = __uint_as_float(kraw[m].x & 0xFFFF0000u);
+                kv[2] = __uint_as_float(kraw[m].y << 16); kv[3] = __uint_as_float(kraw[m].y & 0xFFFF0000u);
                 if (r >= L) {
 #pragma unroll
                     for (int x = 0; x < 4; ++x) { qv[x] = 0.f; kv[x] = 0.f; }
@@ -295,45 +307,72 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 st_tf32x4(smem, OFF_XQ + kbi * KB_XQ + sw128_off(64 + r, ch), qt[0], qt[1], qt[2], qt[3]);
                 st_tf32x4(smem, OFF_KB + kbi * KB_KB + sw128_off(r, ch), kb[0], kb[1], kb[2], kb[3]);
             }
-            {   // V slice: token tid/4, value columns 8*(tid%4) .. +7 (exact bf16 -> fp32)
-                const int r = tid >> 2, cp = 2 * (tid & 3);
+            {   // V^T: token tid/4, value columns 8*(tid%4) .. +7 (exact bf16 -> fp32)
+                const int r = tid >> 2, j0 = 8 * (tid & 3);
                 const uint32_t w4[4] = {vreg.x, vreg.y, vreg.z, vreg.w};
-                float f[8];
 #pragma unroll
                 for (int x = 0; x < 4; ++x) {
-                    f[2 * x] = __uint_as_float(w4[x] << 16);
-                    f[2 * x + 1] = __uint_as_float(w4[x] & 0xFFFF0000u);
+                    *K_at(smem, OFF_VT, KB_VT, j0 + 2 * x, r) = __uint_as_float(w4[x] << 16);
+                    *K_at(smem, OFF_VT, KB_VT, j0 + 2 * x + 1, r) = __uint_as_float(w4[x] & 0xFFFF0000u);
                 }
-                *reinterpret_cast<float4*>(smem + OFF_VB + sw128_off(r, cp)) = make_float4(f[0], f[1], f[2], f[3]);
-                *reinterpret_cast<float4*>(smem + OFF_VB + sw128_off(r, cp + 1)) = make_float4(f[4], f[5], f[6], f[7]);
+            }
+            __syncthreads();   // Kb complete and exp(Gamma_C) known
+            {   // Kb^T from Kb: thread = channel c, 4 consecutive tokens per 16-byte store
+                const int cch = tid & 127, tg = tid >> 7;
+#pragma unroll
+                for (int b = 0; b < 8; ++b) {
+                    const int i0 = 32 * tg + 4 * b;
+                    float4 x;
+                    x.x = *K_at(smem, OFF_KB, KB_KB, i0 + 0, cch);
+                    x.y = *K_at(smem, OFF_KB, KB_KB, i0 + 1, cch);
+                    x.z = *K_at(smem, OFF_KB, KB_KB, i0 + 2, cch);
+                    x.w = *K_at(smem, OFF_KB, KB_KB, i0 + 3, cch);
+                    *reinterpret_cast<float4*>(K_at(smem, OFF_KBT, KB_KBT, cch, i0)) = x;
+                }
+            }
+            if (warp < 4) {   // St = Diag(exp(Gamma_C)) S in TMEM (fp32) and as St^T (tf32)
+                float acc[32];
+                tc_fence_after();
+                tmem_ld32(tm_lane(tmem, warp, TM_S), acc);
+                tmem_wait_ld();
+                const int row = 32 * warp + lane;
+                const float dcr = dc_s[row];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) acc[e] *= dcr;
+                tmem_st32(tm_lane(tmem, warp, TM_S), acc);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) *K_at(smem, OFF_ST, KB_ST, e, row) = to_tf32(acc[e]);
+                tmem_wait_st();
             }
         }
         fence_proxy_async_smem();
+        tc_fence_before();
         __syncthreads();
 
-        // ---------------------------------------- next loads, A/P product
+        // ================================ [A ; P] and [Y ; Z] (one commit)
         if (tid == 0) {
-            if (c + 1 < nchunks) issue_load(t0 + kC);
             tc_fence_after();
 #pragma unroll
-            for (int s = 0; s < 16; ++s) {
-                const uint64_t a = sdesc_sw128(sb + OFF_XQ + (s >> 2) * KB_XQ + (s & 3) * 32, 16, 1024);
-                const uint64_t b = sdesc_sw128(sb + OFF_KB + (s >> 2) * KB_KB + (s & 3) * 32, 16, 1024);
-                mma_tf32_ss(tmem + TM_AP, a, b, ID_AP, s > 0);
-            }
+            for (int s = 0; s < 16; ++s)
+                mma_tf32_ss(tmem + TM_AP, kdesc(sb, OFF_XQ, KB_XQ, s), kdesc(sb, OFF_KB, KB_KB, s), ID_N64, s > 0);
+#pragma unroll
+            for (int s = 0; s < 16; ++s)
+                mma_tf32_ss(tmem + TM_X, kdesc(sb, OFF_XQ, KB_XQ, s), kdesc(sb, OFF_ST, KB_ST, s), ID_N32, s > 0);
             mma_commit(bar_mma);
         }
-        load_pending = (c + 1 < nchunks);
-        load_parity = (c + 1) & 1;
         mma_pending = true;
-        if (c + 1 < nchunks) prefetch(t0 + kC, static_cast<int>((eos - t0 - kC < kC ? eos - t0 - kC : (int64_t)kC)));
+        if (c + 1 < nchunks) prefetch(t0 + kC, static_cast<int>(eos - t0 - kC < kC ? eos - t0 - kC : (int64_t)kC));
         ok = !__syncthreads_or(!mbar_wait_bounded(bar_mma, mma_phase));
         if (!ok) break;
         mma_phase ^= 1;
         mma_pending = false;
         tc_fence_after();
+        // Kb (and XQ) are free now: stage the next chunk's q, k
+        if (tid == 0 && c + 1 < nchunks) issue_load(t0 + kC);
+        load_pending = (c + 1 < nchunks);
+        load_parity = (c + 1) & 1;
 
-        // ------------------------------- A -> M (fp32), P -> tf32 operand
+        // ============== A -> M (fp32), P -> tf32 operand, -Y -> (-Y)^T operand
         {
             float acc[32];
             tmem_ld32(tm_lane(tmem, quarter, TM_AP + 32 * half), acc);
@@ -351,20 +390,30 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     x.w = (i0 + 3 < r) ? br * acc[4 * j + 3] : 0.f;
                     *reinterpret_cast<float4*>(M_at(smem, r, i0)) = x;
                 }
+                if (half == 0) {
+                    float y[32];
+                    tmem_ld32(tm_lane(tmem, quarter, TM_X), y);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) *K_at(smem, OFF_YT, KB_VT, e, r) = to_tf32(-y[e]);
+                }
             } else {
                 const int r = 32 * quarter + lane - 64;
 #pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    if (32 * half + e > r) acc[e] = 0.f;
-                st_row32(smem, OFF_TP + half * KB_TP, 64 + r, acc);
+                for (int j = 0; j < 8; ++j) {
+                    const int i0 = 32 * half + 4 * j;
+                    st_tf32x4(smem, OFF_TP + half * KB_TP + sw128_off(64 + r, j),
+                              (i0 + 0 <= r) ? acc[4 * j + 0] : 0.f, (i0 + 1 <= r) ? acc[4 * j + 1] : 0.f,
+                              (i0 + 2 <= r) ? acc[4 * j + 2] : 0.f, (i0 + 3 <= r) ? acc[4 * j + 3] : 0.f);
+                }
             }
         }
         tc_fence_before();
         __syncthreads();
 
-        // ------------------------- T = (I + M)^-1 by 16-blocks, then T' = T diag(beta)
+        // ============== T = (I + M)^-1 by 16-blocks, then T' = T diag(beta)
         {
-            float* tmpY = reinterpret_cast<float*>(smem + OFF_DL);
+            float* tmpY = reinterpret_cast<float*>(smem + OFF_TMP);
             if (tid < 64) {   // diagonal 16 x 16 blocks: column j of block b by substitution
                 const int b = tid >> 4, j = tid & 15;
                 float xv[16];
@@ -379,7 +428,7 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 for (int r = 0; r < 16; ++r) *T_at(smem, 16 * b + r, 16 * b + j) = xv[r];
             } else {          // zero the six blocks above the diagonal
                 for (int e = tid - 64; e < 6 * 256; e += kThreads - 64) {
-                    // block index 0..5 -> (row block, col block) = (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
+                    // block 0..5 -> (row block, col block) = (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
                     const int blk = e >> 8, w = e & 255, rr = w >> 4, jj = w & 15;
                     const int rb = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
                     const int cb = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
@@ -421,13 +470,13 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     y[0] = fmaf(mv, t4.x, y[0]); y[1] = fmaf(mv, t4.y, y[1]);
                     y[2] = fmaf(mv, t4.z, y[2]); y[3] = fmaf(mv, t4.w, y[3]);
                 }
-                *reinterpret_cast<float4*>(tmpY + rr * 32 + j0) = make_float4(y[0], y[1], y[2], y[3]);
+                *reinterpret_cast<float4*>(tmpY + 512 + rr * 32 + j0) = make_float4(y[0], y[1], y[2], y[3]);
                 __syncthreads();
                 float z[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
                 for (int i = 0; i < 32; ++i) {
                     const float tv = *T_at(smem, 32 + rr, 32 + i);
-                    const float4 y4 = *reinterpret_cast<const float4*>(tmpY + i * 32 + j0);
+                    const float4 y4 = *reinterpret_cast<const float4*>(tmpY + 512 + i * 32 + j0);
                     z[0] = fmaf(tv, y4.x, z[0]); z[1] = fmaf(tv, y4.y, z[1]);
                     z[2] = fmaf(tv, y4.z, z[2]); z[3] = fmaf(tv, y4.w, z[3]);
                 }
@@ -450,67 +499,15 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tc_fence_before();
         __syncthreads();
 
-        // ------------------------------------- U = T' V, W' = T' Kt
+        // ============== delta = T' V + T' (-Y)   (lanes 0-63 of TM_U)
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
-            for (int s = 0; s < 8; ++s) {
-                const uint64_t a = sdesc_sw128(sb + OFF_TP + (s >> 2) * KB_TP + (s & 3) * 32, 16, 1024);
-                const uint64_t bv = sdesc_sw128(sb + OFF_VB + s * 1024, 8192, 1024);
-                const uint64_t bk = sdesc_sw128(sb + OFF_XQ + s * 1024, KB_XQ, 1024);
-                mma_tf32_ss(tmem + TM_U, a, bv, ID_U, s > 0);
-                mma_tf32_ss(tmem + TM_W, a, bk, ID_W, s > 0);
-            }
-            mma_commit(bar_mma);
-        }
-        mma_pending = true;
-        // meanwhile: decay the state to the chunk end, St = Diag(exp(Gamma_C)) S,
-        // in TMEM (fp32) and as the tf32 operand
-        if (warp < 4) {
-            float acc[32];
-            tc_fence_after();
-            tmem_ld32(tm_lane(tmem, warp, TM_S), acc);
-            tmem_wait_ld();
-            const int row = 32 * warp + lane;
-            const float dcr = dc_s[row];
+            for (int s = 0; s < 8; ++s)
+                mma_tf32_ss(tmem + TM_U, kdesc(sb, OFF_TP, KB_TP, s), kdesc(sb, OFF_VT, KB_VT, s), ID_N32, s > 0);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) acc[e] *= dcr;
-            tmem_st32(tm_lane(tmem, warp, TM_S), acc);
-            st_row32(smem, OFF_SB, row, acc);
-            tmem_wait_st();
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        ok = !__syncthreads_or(!mbar_wait_bounded(bar_mma, mma_phase));
-        if (!ok) break;
-        mma_phase ^= 1;
-        mma_pending = false;
-        tc_fence_after();
-
-        // ------------------------------------- -W' -> rows 0-63 of the XQ stack
-        if (quarter < 2) {
-            const int r = 32 * quarter + lane;
-#pragma unroll
-            for (int m2 = 0; m2 < 2; ++m2) {
-                float acc[32];
-                tmem_ld32(tm_lane(tmem, quarter, TM_W + 64 * half + 32 * m2), acc);
-                tmem_wait_ld();
-                st_row32(smem, OFF_XQ + (2 * half + m2) * KB_XQ, r, acc, -1.f);
-            }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-
-        // ------------------------------------- [-W' ; Qt] St
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int s = 0; s < 16; ++s) {
-                const uint64_t a = sdesc_sw128(sb + OFF_XQ + (s >> 2) * KB_XQ + (s & 3) * 32, 16, 1024);
-                const uint64_t b = sdesc_sw128(sb + OFF_SB + s * 1024, 8192, 1024);
-                mma_tf32_ss(tmem + TM_X, a, b, ID_X, s > 0);
-            }
+            for (int s = 0; s < 8; ++s)
+                mma_tf32_ss(tmem + TM_U, kdesc(sb, OFF_TP, KB_TP, s), kdesc(sb, OFF_YT, KB_VT, s), ID_N32, 1);
             mma_commit(bar_mma);
         }
         mma_pending = true;
@@ -520,30 +517,26 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         mma_pending = false;
         tc_fence_after();
 
-        // ------------------------------------- delta = U - W' St (token rows 0-63)
+        // ============== delta -> delta^T operand (token rows 0-63)
         if (warp < 2) {
-            float x[32], u[32];
-            tmem_ld32(tm_lane(tmem, warp, TM_X), x);
-            tmem_ld32(tm_lane(tmem, warp, TM_U), u);
+            float d[32];
+            tmem_ld32(tm_lane(tmem, warp, TM_U), d);
             tmem_wait_ld();
+            const int r = 32 * warp + lane;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) x[e] += u[e];
-            st_row32(smem, OFF_DL, 32 * warp + lane, x);
+            for (int e = 0; e < 32; ++e) *K_at(smem, OFF_YT, KB_VT, e, r) = to_tf32(d[e]);
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
 
-        // ------------------------------------- O += P delta, S = St + Kb^T delta
+        // ============== O = Z + P delta,  S_next = St + Kb^T delta
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
             for (int s = 0; s < 8; ++s) {
-                const uint64_t a = sdesc_sw128(sb + OFF_TP + (s >> 2) * KB_TP + (s & 3) * 32, 16, 1024);
-                const uint64_t bd = sdesc_sw128(sb + OFF_DL + s * 1024, 8192, 1024);
-                const uint64_t ak = sdesc_sw128(sb + OFF_KB + s * 1024, KB_KB, 1024);
-                mma_tf32_ss(tmem + TM_X, a, bd, ID_X, 1);
-                mma_tf32_ss(tmem + TM_S, ak, bd, ID_S, 1);
+                mma_tf32_ss(tmem + TM_X, kdesc(sb, OFF_TP, KB_TP, s), kdesc(sb, OFF_YT, KB_VT, s), ID_N32, 1);
+                mma_tf32_ss(tmem + TM_S, kdesc(sb, OFF_KBT, KB_KBT, s), kdesc(sb, OFF_YT, KB_VT, s), ID_N32, 1);
             }
             mma_commit(bar_mma);
         }
@@ -554,7 +547,7 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         mma_pending = false;
         tc_fence_after();
 
-        // ------------------------------------- O (token rows, lanes 64-127) -> global
+        // ============== O (token rows in lanes 64-127) -> global
         if (warp == 2 || warp == 3) {
             float acc[32];
             tmem_ld32(tm_lane(tmem, warp, TM_X), acc);
@@ -617,7 +610,7 @@ EncodeTiledFn get_encode_fn() {
 }
 
 // [total_T, H, 128] bf16 viewed as a 3-D tensor (channel, head, token); one
-// box is 64 tokens x 128 channels of one head, no swizzle.
+// box is 64 tokens x 128 channels of one head, no swizzle, rows of 256 bytes.
 bool make_qk_map(CUtensorMap* map, const void* base, int64_t total_T, int H) {
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) return false;
@@ -634,6 +627,7 @@ bool make_qk_map(CUtensorMap* map, const void* base, int64_t total_T, int H) {
 
 cudaError_t launch_chunk(const PrefillArgs& a, cudaStream_t stream) {
     if (a.N == 0 || a.H == 0) return cudaSuccess;
+    if (a.total_T <= 0) return cudaErrorInvalidValue;   // callers route empty batches elsewhere
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
@@ -642,9 +636,7 @@ cudaError_t launch_chunk(const PrefillArgs& a, cudaStream_t stream) {
     });
     if (attr_err != cudaSuccess) return attr_err;
     CUtensorMap mq, mk;
-    // a zero-token batch still needs valid maps; point them at a 1-token extent
-    const int64_t extent = a.total_T > 0 ? a.total_T : 1;
-    if (!make_qk_map(&mq, a.q, extent, a.H) || !make_qk_map(&mk, a.k, extent, a.H))
+    if (!make_qk_map(&mq, a.q, a.total_T, a.H) || !make_qk_map(&mk, a.k, a.total_T, a.H))
         return cudaErrorInvalidValue;
     const long long blocks = (long long)a.N * a.H * kSplit;
     kda_chunk_kernel<<<static_cast<unsigned>(blocks), kThreads, SMEM_BYTES, stream>>>(

@@ -10,17 +10,17 @@ Gamma_r = g_0 + ... + g_r (per channel) and Gamma_C = Gamma_{L-1}:
 
     E_r = exp(Gamma_r - Gamma_C) >= 1,   F_r = exp(Gamma_C - Gamma_r) <= 1
     Kt = k_r * E_r,  Qt = q_r * E_r,  Kb = k_r * F_r          (rows r)
-    A  = Kt Kb^T  (so A_ri = sum_c k_rc k_ic exp(Gamma_rc - Gamma_ic))
-    M  = strict_lower(diag(beta) A),  T = (I + M)^-1,  T' = T diag(beta)
-    P  = lower_incl(Qt Kb^T)
-    W' = T' Kt,  U = T' V
     St = diag(exp(Gamma_C)) S                     (state decayed to chunk end)
-    delta = U - W' St,   O = Qt St + P delta,   S_next = St + Kb^T delta
+    A  = Kt Kb^T  (so A_ri = sum_c k_rc k_ic exp(Gamma_rc - Gamma_ic))
+    P  = lower_incl(Qt Kb^T)
+    Y  = Kt St,  Z = Qt St
+    M  = strict_lower(diag(beta) A),  T = (I + M)^-1,  T' = T diag(beta)
+    delta = T' (V - Y),   O = Z + P delta,   S_next = St + Kb^T delta
 
 Unrolling the per-token rule inside the chunk gives
-(I + M) delta = diag(beta)(V - K~ S) with K~_r = k_r exp(Gamma_r); K~ S equals
-W'-side Kt St because Kt diag(exp(Gamma_C)) = K~.  The readout and end state
-follow the same way.
+(I + M) delta = diag(beta)(V - K~ S) with K~_r = k_r exp(Gamma_r); K~ S = Kt St
+because Kt diag(exp(Gamma_C)) = K~.  The readout and end state follow the
+same way.
 """
 import numpy as np
 
@@ -35,9 +35,21 @@ def _bf16(x):
     return r.astype(np.uint32).view(np.float32).astype(np.float64)
 
 
+def _tf32(x):
+    """Round an fp64 array to the nearest tf32 value (10-bit mantissa)."""
+    f = np.asarray(x, dtype=np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    r = ((u + 0x1000) >> 13) << 13          # round half away from zero, as cvt.rna
+    return r.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
 def kda_forward_chunked(q, k, v, g, beta, cu_seqlens, initial_state=None, scale=1.0,
-                        l2norm=True, eps=1e-6, round_bf16=False):
-    rd = _bf16 if round_bf16 else (lambda x: x)
+                        l2norm=True, eps=1e-6, round_bf16=False, round_to=None):
+    """``round_to`` in (None, "bf16", "tf32") rounds every MMA operand the way
+    the kernel stores it; ``round_bf16=True`` is the same as ``round_to="bf16"``."""
+    if round_bf16:
+        round_to = "bf16"
+    rd = {None: (lambda x: x), "bf16": _bf16, "tf32": _tf32}[round_to]
     q, k, v, g, beta = (np.asarray(x, dtype=np.float64) for x in (q, k, v, g, beta))
     cu = [int(x) for x in cu_seqlens]
     T, H, d = q.shape
@@ -66,13 +78,12 @@ def kda_forward_chunked(q, k, v, g, beta, cu_seqlens, initial_state=None, scale=
                 Tm = np.linalg.inv(np.eye(L) + Mm)
                 Tp = rd(Tm * b[None, :])
                 P = rd(np.tril(Qt @ Kb.T))
-                W = rd(Tp @ Kt)
-                U = Tp @ rd(v[sl, h])
                 St32 = np.exp(GC)[:, None] * S
                 St = rd(St32)
-                delta = U - W @ St
+                Y, Z = Kt @ St, Qt @ St
+                delta = Tp @ rd(v[sl, h]) + Tp @ rd(-Y)
                 dl = rd(delta)
-                o[sl, h] = Qt @ St + P @ dl
+                o[sl, h] = Z + P @ dl
                 S = St32 + Kb.T @ dl
             sT[n, h] = S
     return o, sT
