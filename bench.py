@@ -83,7 +83,7 @@ class ClockSampler:
             self.out = open(os.devnull, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", self.target, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
 
@@ -195,6 +195,7 @@ def bench_gpu(args, world, rank, local):
     torch.cuda.synchronize(dev)
     barrier(world)
     torch.cuda.synchronize(dev)
+    # SM clocks are sampled from here to the end of the last timed region
     clocks = ClockSampler(dev.index)
     clocks.start()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -204,7 +205,6 @@ def bench_gpu(args, world, rank, local):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier(world)
-    clk = clocks.stop()
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
     prefill_tok_s = world * T / (ms / 1e3)
     bytes_per_launch = T * H * PREFILL_BYTES_PER_TOKEN_HEAD + H * STATE_BYTES
@@ -277,6 +277,7 @@ def bench_gpu(args, world, rank, local):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier(world)
+    clk = clocks.stop()
     dms = max_over_ranks(e0.elapsed_time(e1) / dsteps, world)
     dec_rate = world * N / (dms / 1e3)
     dec_bytes = N * spec.heads * DECODE_BYTES_PER_SEQ_HEAD
@@ -352,7 +353,7 @@ def bench_reference(args, world, rank):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--ref-tokens", type=int, default=1024)

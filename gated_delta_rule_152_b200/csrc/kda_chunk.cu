@@ -77,9 +77,14 @@ constexpr uint32_t KB_TP = 16384;
 constexpr uint32_t KB_ST = 4096;
 constexpr uint32_t KB_VT = 4096;
 
-// Scratch of the triangular solve inside the dead XQ region.
-constexpr uint32_t OFF_M = OFF_XQ;             // M, 64 x 64 fp32 (row-swizzled)
-constexpr uint32_t OFF_TMP = OFF_XQ + 16384;   // block-merge temporaries, 6 KB
+// Scratch of the triangular solve inside the dead XQ region: plain fp32
+// arrays with padded rows (stride kLd floats) so column walks spread over banks.
+constexpr int kLd = 68, kLd1 = 20, kLd2 = 36;
+constexpr uint32_t OFF_M = OFF_XQ;                         // M, 64 x kLd
+constexpr uint32_t OFF_T = OFF_M + 64 * kLd * 4;           // T, 64 x kLd
+constexpr uint32_t OFF_Y1 = OFF_T + 64 * kLd * 4;          // 2 x 16 x kLd1
+constexpr uint32_t OFF_Y2 = OFF_Y1 + 2 * 16 * kLd1 * 4;    // 32 x kLd2
+static_assert(OFF_Y2 + 32 * kLd2 * 4 <= OFF_XQ + 65536, "solve scratch exceeds the XQ region");
 
 // Tensor-memory columns (fp32 accumulators, 128 lanes each).
 constexpr uint32_t TM_AP = 0;     // 64 cols: A | P
@@ -91,15 +96,6 @@ constexpr uint32_t TM_COLS = 256;
 constexpr uint32_t ID_N64 = idesc_tf32(128, 64, false, false);
 constexpr uint32_t ID_N32 = idesc_tf32(128, 32, false, false);
 
-// M (64 x 64 fp32): 16 float4 chunks per row, chunk position XOR-ed with the
-// row so that 32 rows written at the same column hit distinct banks.
-__device__ __forceinline__ float* M_at(uint8_t* smem, int r, int i) {
-    return reinterpret_cast<float*>(smem + OFF_M) + r * 64 + (((i >> 2) ^ (r & 15)) << 2) + (i & 3);
-}
-// T / T' in rows 0-63 of the [T' ; P] operand (tokens along K).
-__device__ __forceinline__ float* T_at(uint8_t* smem, int r, int i) {
-    return reinterpret_cast<float*>(smem + OFF_TP + (i >> 5) * KB_TP + sw128_off(r, (i & 31) >> 2)) + (i & 3);
-}
 // Element (row, k) of a K-major operand tile at `base` with K-block stride `kb`.
 __device__ __forceinline__ float* K_at(uint8_t* smem, uint32_t base, uint32_t kb, int row, int k) {
     return reinterpret_cast<float*>(smem + base + (k >> 5) * kb + sw128_off(row, (k & 31) >> 2)) + (k & 3);
@@ -270,37 +266,42 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
             if (tid < kC) beta_s[tid] = breg;
 
+            // unpack, mask rows past the sequence end, and L2-normalise all 8 rows
+            float qv[8][4], kv[8][4];
+            float nrm[16];
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                const bool live = 8 * warp + m < L;
+                qv[m][0] = __uint_as_float(qraw[m].x << 16); qv[m][1] = __uint_as_float(qraw[m].x & 0xFFFF0000u);
+                qv[m][2] = __uint_as_float(qraw[m].y << 16); qv[m][3] = __uint_as_float(qraw[m].y & 0xFFFF0000u);
+                kv[m][0] = __uint_as_float(kraw[m].x << 16); kv[m][1] = __uint_as_float(kraw[m].x & 0xFFFF0000u);
+                kv[m][2] = __uint_as_float(kraw[m].y << 16); kv[m][3] = __uint_as_float(kraw[m].y & 0xFFFF0000u);
+                float sq = 0.f, sk = 0.f;
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    if (!live) { qv[m][x] = 0.f; kv[m][x] = 0.f; }
+                    sq = fmaf(qv[m][x], qv[m][x], sq);
+                    sk = fmaf(kv[m][x], kv[m][x], sk);
+                }
+                nrm[m] = sq;
+                nrm[8 + m] = sk;
+            }
+            if (l2norm) warp_allreduce16(nrm);
 #pragma unroll
             for (int m = 0; m < 8; ++m) {
                 const int r = 8 * warp + m;
-                float qv[4], kv[4];
-                qv[0] = __uint_as_float(qraw[m].x << 16); qv[1] = __uint_as_float(qraw[m].x & 0xFFFF0000u);
-                qv[2] = __uint_as_float(qraw[m].y << 16); qv[3] = __uint_as_float(qraw[m].y & 0xFFFF0000u);
-                kv[0] = __uint_as_float(kraw[m].x << 16); kv[1] = __uint_as_float(kraw[m].x & 0xFFFF0000u);
-                kv[2] = __uint_as_float(kraw[m].y << 16); kv[3] = __uint_as_float(kraw[m].y & 0xFFFF0000u);
-                if (r >= L) {
-#pragma unroll
-                    for (int x = 0; x < 4; ++x) { qv[x] = 0.f; kv[x] = 0.f; }
-                }
-                float nq = 1.f, nk = 1.f;
-                if (l2norm) {
-                    float sq = 0.f, sk = 0.f;
-#pragma unroll
-                    for (int x = 0; x < 4; ++x) { sq = fmaf(qv[x], qv[x], sq); sk = fmaf(kv[x], kv[x], sk); }
-                    nq = rsqrtf(warp_sum(sq) + kNormEps);
-                    nk = rsqrtf(warp_sum(sk) + kNormEps);
-                }
-                nq *= scale;
+                const float nq = (l2norm ? rsqrtf(nrm[m] + kNormEps) : 1.f) * scale;
+                const float nk = l2norm ? rsqrtf(nrm[8 + m] + kNormEps) : 1.f;
                 float kt[4], qt[4], kb[4];
 #pragma unroll
                 for (int x = 0; x < 4; ++x) {
                     const float gr = G[m][x] + off[x];
                     const float e = ex2(fminf(gr - GC[x], 126.f));   // exp(Gamma_r - Gamma_C) >= 1
                     const float f = ex2(GC[x] - gr);                 // exp(Gamma_C - Gamma_r) <= 1
-                    const float kn = kv[x] * nk;
+                    const float kn = kv[m][x] * nk;
                     kt[x] = kn * e;
                     kb[x] = kn * f;
-                    qt[x] = qv[x] * nq * e;
+                    qt[x] = qv[m][x] * nq * e;
                 }
                 const int kbi = lane >> 3, ch = lane & 7;
                 st_tf32x4(smem, OFF_XQ + kbi * KB_XQ + sw128_off(r, ch), kt[0], kt[1], kt[2], kt[3]);
@@ -380,6 +381,7 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             if (quarter < 2) {
                 const int r = 32 * quarter + lane;
                 const float br = beta_s[r];
+                float* mrow = reinterpret_cast<float*>(smem + OFF_M) + r * kLd + 32 * half;
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     float4 x;
@@ -388,7 +390,7 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     x.y = (i0 + 1 < r) ? br * acc[4 * j + 1] : 0.f;
                     x.z = (i0 + 2 < r) ? br * acc[4 * j + 2] : 0.f;
                     x.w = (i0 + 3 < r) ? br * acc[4 * j + 3] : 0.f;
-                    *reinterpret_cast<float4*>(M_at(smem, r, i0)) = x;
+                    *reinterpret_cast<float4*>(mrow + 4 * j) = x;
                 }
                 if (half == 0) {
                     float y[32];
@@ -411,87 +413,115 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tc_fence_before();
         __syncthreads();
 
-        // ============== T = (I + M)^-1 by 16-blocks, then T' = T diag(beta)
+        // ============== T = (I + M)^-1 by 16-blocks (plain fp32 arrays, row
+        // stride kLd), then T' = T diag(beta) into the swizzled operand
         {
-            float* tmpY = reinterpret_cast<float*>(smem + OFF_TMP);
+            float* Mf = reinterpret_cast<float*>(smem + OFF_M);
+            float* Tf = reinterpret_cast<float*>(smem + OFF_T);
+            float* Y1 = reinterpret_cast<float*>(smem + OFF_Y1);   // [2][16][kLd1]
+            float* Y2 = reinterpret_cast<float*>(smem + OFF_Y2);   // [32][kLd2]
             if (tid < 64) {   // diagonal 16 x 16 blocks: column j of block b by substitution
                 const int b = tid >> 4, j = tid & 15;
+                const float* Mb = Mf + 16 * b * kLd + 16 * b;
                 float xv[16];
 #pragma unroll
                 for (int r = 0; r < 16; ++r) {
-                    float s = (r == j) ? 1.f : 0.f;
+                    float s0 = (r == j) ? 1.f : 0.f, s1 = 0.f;
 #pragma unroll
-                    for (int i = 0; i < r; ++i) s = fmaf(-*M_at(smem, 16 * b + r, 16 * b + i), xv[i], s);
-                    xv[r] = s;
+                    for (int i = 0; i < r; i += 2) {
+                        s0 = fmaf(-Mb[r * kLd + i], xv[i], s0);
+                        if (i + 1 < r) s1 = fmaf(-Mb[r * kLd + i + 1], xv[i + 1], s1);
+                    }
+                    xv[r] = s0 + s1;
                 }
+                float* Tb = Tf + 16 * b * kLd + 16 * b + j;
 #pragma unroll
-                for (int r = 0; r < 16; ++r) *T_at(smem, 16 * b + r, 16 * b + j) = xv[r];
-            } else {          // zero the six blocks above the diagonal
-                for (int e = tid - 64; e < 6 * 256; e += kThreads - 64) {
-                    // block 0..5 -> (row block, col block) = (0,1) (0,2) (0,3) (1,2) (1,3) (2,3)
-                    const int blk = e >> 8, w = e & 255, rr = w >> 4, jj = w & 15;
-                    const int rb = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
-                    const int cb = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-                    *T_at(smem, 16 * rb + rr, 16 * cb + jj) = 0.f;
-                }
+                for (int r = 0; r < 16; ++r) Tb[r * kLd] = xv[r];
+            } else if (tid < 192) {   // zero blocks (0,1) and (2,3), read by the 32 -> 64 merge
+                const int e = tid - 64, blk = e >> 6, rr = (e & 63) >> 2, c4 = (e & 3) * 4;
+                *reinterpret_cast<float4*>(Tf + (32 * blk + rr) * kLd + 32 * blk + 16 + c4) =
+                    make_float4(0.f, 0.f, 0.f, 0.f);
             }
             __syncthreads();
-            {   // 16 -> 32: T_ab = -T_aa M_ab T_bb for (a, b) = (1, 0), (3, 2)
+            {   // 16 -> 32: T_ab = -T_aa (M_ab T_bb) for (a, b) = (1, 0), (3, 2)
                 const int p = tid >> 7, rr = (tid & 127) >> 3, j0 = (tid & 7) * 2;
                 const int a = 2 * p + 1, b = 2 * p;
+                const float* mrow = Mf + (16 * a + rr) * kLd + 16 * b;
+                const float* tcol = Tf + 16 * b * kLd + 16 * b + j0;
                 float y0 = 0.f, y1 = 0.f;
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float mv = *M_at(smem, 16 * a + rr, 16 * b + i);
-                    y0 = fmaf(mv, *T_at(smem, 16 * b + i, 16 * b + j0), y0);
-                    y1 = fmaf(mv, *T_at(smem, 16 * b + i, 16 * b + j0 + 1), y1);
+                for (int i4 = 0; i4 < 16; i4 += 4) {
+                    const float4 mv = *reinterpret_cast<const float4*>(mrow + i4);
+                    const float mm[4] = {mv.x, mv.y, mv.z, mv.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float2 t2 = *reinterpret_cast<const float2*>(tcol + (i4 + u) * kLd);
+                        y0 = fmaf(mm[u], t2.x, y0);
+                        y1 = fmaf(mm[u], t2.y, y1);
+                    }
                 }
-                tmpY[p * 256 + rr * 16 + j0] = y0;
-                tmpY[p * 256 + rr * 16 + j0 + 1] = y1;
+                *reinterpret_cast<float2*>(Y1 + (p * 16 + rr) * kLd1 + j0) = make_float2(y0, y1);
                 __syncthreads();
+                const float* trow = Tf + (16 * a + rr) * kLd + 16 * a;
+                const float* ycol = Y1 + p * 16 * kLd1 + j0;
                 float z0 = 0.f, z1 = 0.f;
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float tv = *T_at(smem, 16 * a + rr, 16 * a + i);
-                    z0 = fmaf(tv, tmpY[p * 256 + i * 16 + j0], z0);
-                    z1 = fmaf(tv, tmpY[p * 256 + i * 16 + j0 + 1], z1);
+                for (int i4 = 0; i4 < 16; i4 += 4) {
+                    const float4 tv = *reinterpret_cast<const float4*>(trow + i4);
+                    const float tt[4] = {tv.x, tv.y, tv.z, tv.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float2 y2 = *reinterpret_cast<const float2*>(ycol + (i4 + u) * kLd1);
+                        z0 = fmaf(tt[u], y2.x, z0);
+                        z1 = fmaf(tt[u], y2.y, z1);
+                    }
                 }
-                *T_at(smem, 16 * a + rr, 16 * b + j0) = -z0;
-                *T_at(smem, 16 * a + rr, 16 * b + j0 + 1) = -z1;
+                *reinterpret_cast<float2*>(Tf + (16 * a + rr) * kLd + 16 * b + j0) = make_float2(-z0, -z1);
             }
             __syncthreads();
-            {   // 32 -> 64: T_hl = -T_hh M_hl T_ll with 32 x 32 blocks
+            {   // 32 -> 64: T_hl = -T_hh (M_hl T_ll) with 32 x 32 blocks
                 const int rr = tid >> 3, j0 = (tid & 7) * 4;
+                const float* mrow = Mf + (32 + rr) * kLd;
                 float y[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-                for (int i = 0; i < 32; ++i) {
-                    const float mv = *M_at(smem, 32 + rr, i);
-                    const float4 t4 = *reinterpret_cast<const float4*>(T_at(smem, i, j0));
-                    y[0] = fmaf(mv, t4.x, y[0]); y[1] = fmaf(mv, t4.y, y[1]);
-                    y[2] = fmaf(mv, t4.z, y[2]); y[3] = fmaf(mv, t4.w, y[3]);
+#pragma unroll
+                for (int i4 = 0; i4 < 32; i4 += 4) {
+                    const float4 mv = *reinterpret_cast<const float4*>(mrow + i4);
+                    const float mm[4] = {mv.x, mv.y, mv.z, mv.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float4 t4 = *reinterpret_cast<const float4*>(Tf + (i4 + u) * kLd + j0);
+                        y[0] = fmaf(mm[u], t4.x, y[0]); y[1] = fmaf(mm[u], t4.y, y[1]);
+                        y[2] = fmaf(mm[u], t4.z, y[2]); y[3] = fmaf(mm[u], t4.w, y[3]);
+                    }
                 }
-                *reinterpret_cast<float4*>(tmpY + 512 + rr * 32 + j0) = make_float4(y[0], y[1], y[2], y[3]);
+                *reinterpret_cast<float4*>(Y2 + rr * kLd2 + j0) = make_float4(y[0], y[1], y[2], y[3]);
                 __syncthreads();
+                const float* trow = Tf + (32 + rr) * kLd + 32;
                 float z[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-                for (int i = 0; i < 32; ++i) {
-                    const float tv = *T_at(smem, 32 + rr, 32 + i);
-                    const float4 y4 = *reinterpret_cast<const float4*>(tmpY + 512 + i * 32 + j0);
-                    z[0] = fmaf(tv, y4.x, z[0]); z[1] = fmaf(tv, y4.y, z[1]);
-                    z[2] = fmaf(tv, y4.z, z[2]); z[3] = fmaf(tv, y4.w, z[3]);
+#pragma unroll
+                for (int i4 = 0; i4 < 32; i4 += 4) {
+                    const float4 tv = *reinterpret_cast<const float4*>(trow + i4);
+                    const float tt[4] = {tv.x, tv.y, tv.z, tv.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const float4 y4 = *reinterpret_cast<const float4*>(Y2 + (i4 + u) * kLd2 + j0);
+                        z[0] = fmaf(tt[u], y4.x, z[0]); z[1] = fmaf(tt[u], y4.y, z[1]);
+                        z[2] = fmaf(tt[u], y4.z, z[2]); z[3] = fmaf(tt[u], y4.w, z[3]);
+                    }
                 }
-                *reinterpret_cast<float4*>(T_at(smem, 32 + rr, j0)) = make_float4(-z[0], -z[1], -z[2], -z[3]);
+                *reinterpret_cast<float4*>(Tf + (32 + rr) * kLd + j0) = make_float4(-z[0], -z[1], -z[2], -z[3]);
             }
             __syncthreads();
-            {   // T' = T diag(beta), rounded to tf32
+            {   // T' = T diag(beta) on and below the diagonal, zero above; tf32 operand
                 const int r = tid >> 2;
 #pragma unroll
                 for (int qd = 0; qd < 4; ++qd) {
                     const int i0 = 16 * (tid & 3) + 4 * qd;
-                    float4* p4 = reinterpret_cast<float4*>(T_at(smem, r, i0));
-                    const float4 t4 = *p4;
-                    *p4 = make_float4(to_tf32(t4.x * beta_s[i0]), to_tf32(t4.y * beta_s[i0 + 1]),
-                                      to_tf32(t4.z * beta_s[i0 + 2]), to_tf32(t4.w * beta_s[i0 + 3]));
+                    const float4 t4 = *reinterpret_cast<const float4*>(Tf + r * kLd + i0);
+                    const float4 b4 = *reinterpret_cast<const float4*>(beta_s + i0);
+                    st_tf32x4(smem, OFF_TP + (i0 >> 5) * KB_TP + sw128_off(r, (i0 & 31) >> 2),
+                              (i0 + 0 <= r) ? t4.x * b4.x : 0.f, (i0 + 1 <= r) ? t4.y * b4.y : 0.f,
+                              (i0 + 2 <= r) ? t4.z * b4.z : 0.f, (i0 + 3 <= r) ? t4.w * b4.w : 0.f);
                 }
             }
         }
