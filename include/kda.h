@@ -133,6 +133,32 @@ KDA_API int kda_decode_step(const void *q, const void *k, const void *v, const f
                     kda_stream_t stream);
 
 /*
+ * kda_chunk_fwd_noalloc -- kda_chunk_fwd for callers that cannot allocate
+ * device memory at all (code running inside an allocator's own callbacks, an
+ * embedding runtime that owns every device byte, or a service that forbids
+ * allocation after start-up).  The reference pages have no counterpart: this
+ * is a packaging of the same prefill.
+ *
+ * Same arguments and result as kda_chunk_fwd, minus the workspace: its
+ * scratch is a fixed 64 KiB array inside the library (every GPU that loads
+ * libkda holds it until the process exits), enough for N up to
+ * KDA_NOALLOC_MAX_SEQS sequences; larger N returns KDA_ERR_WORKSPACE and
+ * launches nothing.  The first call on each device looks up the array's
+ * device address (with that device current), so make that first call before
+ * any stream capture.  All calls share the array: it keeps the last call's
+ * contents, its error word is cleared at the start of each call and cannot be
+ * read back (use kda_chunk_fwd when you need it), and calls that overlap on
+ * the GPU race on it -- order them on one stream.  Nothing is allocated or
+ * freed.
+ */
+#define KDA_NOALLOC_MAX_SEQS 16320
+KDA_API int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const float *g,
+                          const float *beta, const int32_t *cu_seqlens, int32_t N,
+                          int64_t total_T, int32_t H, int32_t d, kda_dtype dt, float scale,
+                          uint32_t flags, const float *initial_state, float *final_state,
+                          float *o, kda_stream_t stream);
+
+/*
  * Copy the device error word of a workspace used by kda_chunk_fwd to *out
  * (synchronises `stream`).  Returns KDA_OK or KDA_ERR_*.
  */
