@@ -48,6 +48,11 @@ STATE_BYTES = 4 * D * D
 PREFILL_FLOPS_PER_TOKEN_HEAD = (5 * 2 * 64 * 64 * D + 3 * 2 * 64 * D * D + 64 ** 3 // 3) // 64
 # Decode: state read + write, plus q, k, v (bf16), g (fp32), beta, o (fp32).
 DECODE_BYTES_PER_SEQ_HEAD = 2 * STATE_BYTES + 3 * 2 * D + 4 * D + 4 + 4 * D
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch,
+# from an ncu capture of the current kernel build on the same workload; set
+# back to None whenever the kernel changes until it is captured again.
+MEASURED_TRAFFIC_PREFILL = None
+MEASURED_TRAFFIC_DECODE = 547.405312e6 + 486.942464e6
 
 
 def load_peaks():
@@ -302,7 +307,7 @@ def bench_gpu(args, world, rank, local):
                    "qkv_dtype": "bf16", "o_dtype": "fp32", "parallelism": f"replicas x{world}",
                    "l2": "inputs 471 MB > 126 MB L2, no flush"},
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved_gbs / hbm, "traffic": None,
+                     "frac": achieved_gbs / hbm, "traffic": MEASURED_TRAFFIC_PREFILL,
                      "peak_source": f"{peak_src} hbm_gbs",
                      "bytes_per_launch": bytes_per_launch,
                      "tensor": {"achieved_tflops": achieved_tflops, "peak_tflops_tf32": tf32_peak,
@@ -311,7 +316,8 @@ def bench_gpu(args, world, rank, local):
         "decode": {"workload": spec.name, "value": dec_rate, "unit": "seq-steps/s/layer",
                    "ms_per_call": dms, "layers_rotated": L,
                    "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": hbm, "unit": "GB/s",
-                                "frac": dec_gbs / hbm, "bytes_per_launch": dec_bytes}},
+                                "frac": dec_gbs / hbm, "traffic": MEASURED_TRAFFIC_DECODE,
+                                "bytes_per_launch": dec_bytes}},
         "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps * 2 + dsteps,
