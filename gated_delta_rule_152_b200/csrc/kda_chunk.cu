@@ -109,9 +109,24 @@ __device__ __forceinline__ uint32_t tm_lane(uint32_t tmem, int quarter, uint32_t
     return tmem + (static_cast<uint32_t>(32 * quarter) << 16) + col;
 }
 
-// K-major SW128 descriptor of K step s (8 tf32 = 32 bytes) of a tile.
-__device__ __forceinline__ uint64_t kdesc(uint32_t sb, uint32_t base, uint32_t kb_stride, int s) {
-    return sdesc_sw128(sb + base + (s >> 2) * kb_stride + (s & 3) * 32, 16, 1024);
+__device__ __forceinline__ uint64_t tdesc(uint32_t sb, uint32_t base) { return sdesc_sw128(sb + base, 16, 1024); }
+
+// mma.sync fragments from plain row-major fp32 arrays (leading dimension ld),
+// rounded to tf32 on the way: A tile 16 x 8 at (r0, k0), B tile 8 x 8 at (k0, n0).
+__device__ __forceinline__ void frag_a(uint32_t (&a)[4], const float* X, int ld, int r0, int k0, int g, int t) {
+    a[0] = tf32_bits(X[(r0 + g) * ld + k0 + t]);
+    a[1] = tf32_bits(X[(r0 + g + 8) * ld + k0 + t]);
+    a[2] = tf32_bits(X[(r0 + g) * ld + k0 + t + 4]);
+    a[3] = tf32_bits(X[(r0 + g + 8) * ld + k0 + t + 4]);
+}
+__device__ __forceinline__ void frag_b(uint32_t (&b)[2], const float* Y, int ld, int k0, int n0, int g, int t) {
+    b[0] = tf32_bits(Y[(k0 + t) * ld + n0 + g]);
+    b[1] = tf32_bits(Y[(k0 + t + 4) * ld + n0 + g]);
+}
+__device__ __forceinline__ void frag_store(float* D, int ld, int r0, int n0, const float (&d)[4], float sgn, int g,
+                                           int t) {
+    *reinterpret_cast<float2*>(D + (r0 + g) * ld + n0 + 2 * t) = make_float2(sgn * d[0], sgn * d[1]);
+    *reinterpret_cast<float2*>(D + (r0 + g + 8) * ld + n0 + 2 * t) = make_float2(sgn * d[2], sgn * d[3]);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -331,18 +346,20 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     *reinterpret_cast<float4*>(K_at(smem, OFF_KBT, KB_KBT, cch, i0)) = x;
                 }
             }
-            if (warp < 4) {   // St = Diag(exp(Gamma_C)) S in TMEM (fp32) and as St^T (tf32)
-                float acc[32];
+            {   // St = Diag(exp(Gamma_C)) S in TMEM (fp32) and as St^T (tf32); the two
+                // warps of a TMEM lane quarter take 16 value columns each
+                float acc[16];
+                const int c0 = 16 * half;
                 tc_fence_after();
-                tmem_ld32(tm_lane(tmem, warp, TM_S), acc);
+                tmem_ld16(tm_lane(tmem, quarter, TM_S + c0), acc);
                 tmem_wait_ld();
-                const int row = 32 * warp + lane;
+                const int row = 32 * quarter + lane;
                 const float dcr = dc_s[row];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) acc[e] *= dcr;
-                tmem_st32(tm_lane(tmem, warp, TM_S), acc);
+                for (int e = 0; e < 16; ++e) acc[e] *= dcr;
+                tmem_st16(tm_lane(tmem, quarter, TM_S + c0), acc);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) *K_at(smem, OFF_ST, KB_ST, e, row) = to_tf32(acc[e]);
+                for (int e = 0; e < 16; ++e) *K_at(smem, OFF_ST, KB_ST, c0 + e, row) = to_tf32(acc[e]);
                 tmem_wait_st();
             }
         }
@@ -353,12 +370,13 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // ================================ [A ; P] and [Y ; Z] (one commit)
         if (tid == 0) {
             tc_fence_after();
+            const uint64_t dxq = tdesc(sb, OFF_XQ), dkb = tdesc(sb, OFF_KB), dst = tdesc(sb, OFF_ST);
 #pragma unroll
             for (int s = 0; s < 16; ++s)
-                mma_tf32_ss(tmem + TM_AP, kdesc(sb, OFF_XQ, KB_XQ, s), kdesc(sb, OFF_KB, KB_KB, s), ID_N64, s > 0);
+                mma_tf32_ss(tmem + TM_AP, kstep(dxq, KB_XQ, s), kstep(dkb, KB_KB, s), ID_N64, s > 0);
 #pragma unroll
             for (int s = 0; s < 16; ++s)
-                mma_tf32_ss(tmem + TM_X, kdesc(sb, OFF_XQ, KB_XQ, s), kdesc(sb, OFF_ST, KB_ST, s), ID_N32, s > 0);
+                mma_tf32_ss(tmem + TM_X, kstep(dxq, KB_XQ, s), kstep(dst, KB_ST, s), ID_N32, s > 0);
             mma_commit(bar_mma);
         }
         mma_pending = true;
@@ -391,13 +409,6 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     x.z = (i0 + 2 < r) ? br * acc[4 * j + 2] : 0.f;
                     x.w = (i0 + 3 < r) ? br * acc[4 * j + 3] : 0.f;
                     *reinterpret_cast<float4*>(mrow + 4 * j) = x;
-                }
-                if (half == 0) {
-                    float y[32];
-                    tmem_ld32(tm_lane(tmem, quarter, TM_X), y);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) *K_at(smem, OFF_YT, KB_VT, e, r) = to_tf32(-y[e]);
                 }
             } else {
                 const int r = 32 * quarter + lane - 64;
@@ -437,79 +448,73 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 float* Tb = Tf + 16 * b * kLd + 16 * b + j;
 #pragma unroll
                 for (int r = 0; r < 16; ++r) Tb[r * kLd] = xv[r];
-            } else if (tid < 192) {   // zero blocks (0,1) and (2,3), read by the 32 -> 64 merge
-                const int e = tid - 64, blk = e >> 6, rr = (e & 63) >> 2, c4 = (e & 3) * 4;
-                *reinterpret_cast<float4*>(Tf + (32 * blk + rr) * kLd + 32 * blk + 16 + c4) =
-                    make_float4(0.f, 0.f, 0.f, 0.f);
+            } else if (tid < 128) {   // zero blocks (0,1) and (2,3), read by the 32 -> 64 merge
+                const int e = tid - 64, blk = e >> 5, rr = (e & 31) >> 1, c8 = (e & 1) * 8;
+                float* z = Tf + (32 * blk + rr) * kLd + 32 * blk + 16 + c8;
+                *reinterpret_cast<float4*>(z) = make_float4(0.f, 0.f, 0.f, 0.f);
+                *reinterpret_cast<float4*>(z + 4) = make_float4(0.f, 0.f, 0.f, 0.f);
+            } else if (warp == 4 || warp == 5) {   // -Y (token rows 0-63) -> (-Y)^T operand
+                float y[32];
+                tc_fence_after();
+                tmem_ld32(tm_lane(tmem, quarter, TM_X), y);
+                tmem_wait_ld();
+                const int r = 32 * quarter + lane;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) *K_at(smem, OFF_YT, KB_VT, e, r) = to_tf32(-y[e]);
             }
             __syncthreads();
-            {   // 16 -> 32: T_ab = -T_aa (M_ab T_bb) for (a, b) = (1, 0), (3, 2)
-                const int p = tid >> 7, rr = (tid & 127) >> 3, j0 = (tid & 7) * 2;
-                const int a = 2 * p + 1, b = 2 * p;
-                const float* mrow = Mf + (16 * a + rr) * kLd + 16 * b;
-                const float* tcol = Tf + 16 * b * kLd + 16 * b + j0;
-                float y0 = 0.f, y1 = 0.f;
+            {   // 16 -> 32 on tensor cores: T_ab = -T_aa (M_ab T_bb) for (a, b) = (1, 0), (3, 2);
+                // warp w < 4 owns pair p = w / 2, output columns 8 (w % 2) .. +7
+                const int g = lane >> 2, t = lane & 3;
+                const int p = warp >> 1, nt = warp & 1, a = 2 * p + 1, b = 2 * p;
+                if (warp < 4) {
+                    float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int i4 = 0; i4 < 16; i4 += 4) {
-                    const float4 mv = *reinterpret_cast<const float4*>(mrow + i4);
-                    const float mm[4] = {mv.x, mv.y, mv.z, mv.w};
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const float2 t2 = *reinterpret_cast<const float2*>(tcol + (i4 + u) * kLd);
-                        y0 = fmaf(mm[u], t2.x, y0);
-                        y1 = fmaf(mm[u], t2.y, y1);
+                    for (int ks = 0; ks < 2; ++ks) {
+                        uint32_t fa[4], fb[2];
+                        frag_a(fa, Mf, kLd, 16 * a, 16 * b + 8 * ks, g, t);
+                        frag_b(fb, Tf, kLd, 16 * b + 8 * ks, 16 * b + 8 * nt, g, t);
+                        mma_m16n8k8_tf32(d, fa, fb);
                     }
+                    frag_store(Y1 + p * 16 * kLd1, kLd1, 0, 8 * nt, d, 1.f, g, t);
                 }
-                *reinterpret_cast<float2*>(Y1 + (p * 16 + rr) * kLd1 + j0) = make_float2(y0, y1);
                 __syncthreads();
-                const float* trow = Tf + (16 * a + rr) * kLd + 16 * a;
-                const float* ycol = Y1 + p * 16 * kLd1 + j0;
-                float z0 = 0.f, z1 = 0.f;
+                if (warp < 4) {
+                    float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int i4 = 0; i4 < 16; i4 += 4) {
-                    const float4 tv = *reinterpret_cast<const float4*>(trow + i4);
-                    const float tt[4] = {tv.x, tv.y, tv.z, tv.w};
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const float2 y2 = *reinterpret_cast<const float2*>(ycol + (i4 + u) * kLd1);
-                        z0 = fmaf(tt[u], y2.x, z0);
-                        z1 = fmaf(tt[u], y2.y, z1);
+                    for (int ks = 0; ks < 2; ++ks) {
+                        uint32_t fa[4], fb[2];
+                        frag_a(fa, Tf, kLd, 16 * a, 16 * a + 8 * ks, g, t);
+                        frag_b(fb, Y1 + p * 16 * kLd1, kLd1, 8 * ks, 8 * nt, g, t);
+                        mma_m16n8k8_tf32(d, fa, fb);
                     }
+                    frag_store(Tf, kLd, 16 * a, 16 * b + 8 * nt, d, -1.f, g, t);
                 }
-                *reinterpret_cast<float2*>(Tf + (16 * a + rr) * kLd + 16 * b + j0) = make_float2(-z0, -z1);
             }
             __syncthreads();
-            {   // 32 -> 64: T_hl = -T_hh (M_hl T_ll) with 32 x 32 blocks
-                const int rr = tid >> 3, j0 = (tid & 7) * 4;
-                const float* mrow = Mf + (32 + rr) * kLd;
-                float y[4] = {0.f, 0.f, 0.f, 0.f};
+            {   // 32 -> 64 on tensor cores: T_hl = -T_hh (M_hl T_ll); warp w owns the
+                // 16 x 8 output tile (rows 16 (w / 4), columns 8 (w % 4))
+                const int g = lane >> 2, t = lane & 3;
+                const int mt = warp >> 2, nt = warp & 3;
+                float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int i4 = 0; i4 < 32; i4 += 4) {
-                    const float4 mv = *reinterpret_cast<const float4*>(mrow + i4);
-                    const float mm[4] = {mv.x, mv.y, mv.z, mv.w};
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const float4 t4 = *reinterpret_cast<const float4*>(Tf + (i4 + u) * kLd + j0);
-                        y[0] = fmaf(mm[u], t4.x, y[0]); y[1] = fmaf(mm[u], t4.y, y[1]);
-                        y[2] = fmaf(mm[u], t4.z, y[2]); y[3] = fmaf(mm[u], t4.w, y[3]);
-                    }
+                for (int ks = 0; ks < 4; ++ks) {
+                    uint32_t fa[4], fb[2];
+                    frag_a(fa, Mf, kLd, 32 + 16 * mt, 8 * ks, g, t);
+                    frag_b(fb, Tf, kLd, 8 * ks, 8 * nt, g, t);
+                    mma_m16n8k8_tf32(d, fa, fb);
                 }
-                *reinterpret_cast<float4*>(Y2 + rr * kLd2 + j0) = make_float4(y[0], y[1], y[2], y[3]);
+                frag_store(Y2, kLd2, 16 * mt, 8 * nt, d, 1.f, g, t);
                 __syncthreads();
-                const float* trow = Tf + (32 + rr) * kLd + 32;
-                float z[4] = {0.f, 0.f, 0.f, 0.f};
+                float e[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int i4 = 0; i4 < 32; i4 += 4) {
-                    const float4 tv = *reinterpret_cast<const float4*>(trow + i4);
-                    const float tt[4] = {tv.x, tv.y, tv.z, tv.w};
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const float4 y4 = *reinterpret_cast<const float4*>(Y2 + (i4 + u) * kLd2 + j0);
-                        z[0] = fmaf(tt[u], y4.x, z[0]); z[1] = fmaf(tt[u], y4.y, z[1]);
-                        z[2] = fmaf(tt[u], y4.z, z[2]); z[3] = fmaf(tt[u], y4.w, z[3]);
-                    }
+                for (int ks = 0; ks < 4; ++ks) {
+                    uint32_t fa[4], fb[2];
+                    frag_a(fa, Tf, kLd, 32 + 16 * mt, 32 + 8 * ks, g, t);
+                    frag_b(fb, Y2, kLd2, 8 * ks, 8 * nt, g, t);
+                    mma_m16n8k8_tf32(e, fa, fb);
                 }
-                *reinterpret_cast<float4*>(Tf + (32 + rr) * kLd + j0) = make_float4(-z[0], -z[1], -z[2], -z[3]);
+                frag_store(Tf, kLd, 32 + 16 * mt, 8 * nt, e, -1.f, g, t);
             }
             __syncthreads();
             {   // T' = T diag(beta) on and below the diagonal, zero above; tf32 operand
@@ -532,12 +537,13 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // ============== delta = T' V + T' (-Y)   (lanes 0-63 of TM_U)
         if (tid == 0) {
             tc_fence_after();
+            const uint64_t dtp = tdesc(sb, OFF_TP), dvt = tdesc(sb, OFF_VT), dyt = tdesc(sb, OFF_YT);
 #pragma unroll
             for (int s = 0; s < 8; ++s)
-                mma_tf32_ss(tmem + TM_U, kdesc(sb, OFF_TP, KB_TP, s), kdesc(sb, OFF_VT, KB_VT, s), ID_N32, s > 0);
+                mma_tf32_ss(tmem + TM_U, kstep(dtp, KB_TP, s), kstep(dvt, KB_VT, s), ID_N32, s > 0);
 #pragma unroll
             for (int s = 0; s < 8; ++s)
-                mma_tf32_ss(tmem + TM_U, kdesc(sb, OFF_TP, KB_TP, s), kdesc(sb, OFF_YT, KB_VT, s), ID_N32, 1);
+                mma_tf32_ss(tmem + TM_U, kstep(dtp, KB_TP, s), kstep(dyt, KB_VT, s), ID_N32, 1);
             mma_commit(bar_mma);
         }
         mma_pending = true;
@@ -548,13 +554,14 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tc_fence_after();
 
         // ============== delta -> delta^T operand (token rows 0-63)
-        if (warp < 2) {
-            float d[32];
-            tmem_ld32(tm_lane(tmem, warp, TM_U), d);
+        if (quarter < 2) {   // two warps per lane quarter, 16 value columns each
+            float d[16];
+            const int c0 = 16 * half;
+            tmem_ld16(tm_lane(tmem, quarter, TM_U + c0), d);
             tmem_wait_ld();
-            const int r = 32 * warp + lane;
+            const int r = 32 * quarter + lane;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) *K_at(smem, OFF_YT, KB_VT, e, r) = to_tf32(d[e]);
+            for (int e = 0; e < 16; ++e) *K_at(smem, OFF_YT, KB_VT, c0 + e, r) = to_tf32(d[e]);
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -563,10 +570,11 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // ============== O = Z + P delta,  S_next = St + Kb^T delta
         if (tid == 0) {
             tc_fence_after();
+            const uint64_t dtp = tdesc(sb, OFF_TP), dkbt = tdesc(sb, OFF_KBT), dyt = tdesc(sb, OFF_YT);
 #pragma unroll
             for (int s = 0; s < 8; ++s) {
-                mma_tf32_ss(tmem + TM_X, kdesc(sb, OFF_TP, KB_TP, s), kdesc(sb, OFF_YT, KB_VT, s), ID_N32, 1);
-                mma_tf32_ss(tmem + TM_S, kdesc(sb, OFF_KBT, KB_KBT, s), kdesc(sb, OFF_YT, KB_VT, s), ID_N32, 1);
+                mma_tf32_ss(tmem + TM_X, kstep(dtp, KB_TP, s), kstep(dyt, KB_VT, s), ID_N32, 1);
+                mma_tf32_ss(tmem + TM_S, kstep(dkbt, KB_KBT, s), kstep(dyt, KB_VT, s), ID_N32, 1);
             }
             mma_commit(bar_mma);
         }

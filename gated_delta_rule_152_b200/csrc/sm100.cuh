@@ -13,10 +13,10 @@
 //     rows ("K-block").  Descriptor: SBO = 1024 (next 8-row group); LBO unused.
 //     One tf32 MMA consumes K = 8 (32 bytes), so the start address advances
 //     by 32 bytes per K step inside a K-block.
-//   * MN-major operand (contiguous along M or N): row = K index, a row holds
-//     32 consecutive M/N elements.  Descriptor: SBO = 1024 (next 8 K rows),
-//     LBO = byte distance between consecutive 32-element M/N blocks.  One
-//     tf32 K step is 8 rows = 1024 bytes.
+// Every operand of the KDA kernels is K-major: for kind::tf32, operands that
+// are contiguous along M or N need a different swizzle (32-byte granules over
+// 4-row atoms), so tiles that would be used both ways are instead stored (or
+// copied) in the K-major orientation each product needs.
 #pragma once
 #include <cstdint>
 #include <cuda.h>
@@ -129,6 +129,9 @@ __host__ __device__ constexpr uint32_t idesc_tf32(uint32_t M, uint32_t N, bool a
 }
 
 // Shared-memory matrix descriptor, 128-byte swizzle, sm_100 version bits.
+// The start-address field holds address / 16 in 14 bits; since shared-memory
+// addresses stay below 256 KB, later K steps of the same tile are obtained by
+// adding their byte offset / 16 to the descriptor (kstep below).
 __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t smem_addr, uint32_t lbo_bytes,
                                                 uint32_t sbo_bytes) {
     uint64_t d = 0;
@@ -138,6 +141,12 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t smem_addr, uint32_t lbo
     d |= static_cast<uint64_t>(1u) << 46;   // descriptor version for sm_100
     d |= static_cast<uint64_t>(2u) << 61;   // SWIZZLE_128B
     return d;
+}
+
+// Descriptor of K step s (8 tf32 = 32 bytes) of a K-major tile whose K-blocks
+// of 32 elements are kb_stride bytes apart.
+__device__ __forceinline__ uint64_t kstep(uint64_t base, uint32_t kb_stride, int s) {
+    return base + ((static_cast<uint32_t>(s >> 2) * kb_stride + static_cast<uint32_t>(s & 3) * 32u) >> 4);
 }
 
 // 32 lanes x 32 columns of 32-bit TMEM -> 32 registers per thread.  The warp
@@ -170,6 +179,28 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&r)[32]) 
         : "memory");
 }
 
+// 32 lanes x 16 columns variants.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&r)[16]) {
+    uint32_t* u = reinterpret_cast<uint32_t*>(r);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]),
+          "=r"(u[7]), "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]),
+          "=r"(u[14]), "=r"(u[15])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&r)[16]) {
+    const uint32_t* u = reinterpret_cast<const uint32_t*>(r);
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+        ::"r"(taddr), "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]),
+          "r"(u[7]), "r"(u[8]), "r"(u[9]), "r"(u[10]), "r"(u[11]), "r"(u[12]), "r"(u[13]),
+          "r"(u[14]), "r"(u[15])
+        : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -178,12 +209,28 @@ __device__ __forceinline__ void tmem_wait_st() {
 }
 
 // ---------------------------------------------------------------- misc
-// Round an fp32 value to the nearest tf32 value (kept in a 32-bit container),
-// so the tensor core sees a rounded rather than truncated operand.
+// Round an fp32 value to the nearest tf32 value (10 explicit mantissa bits,
+// halfway cases away from zero), kept in a 32-bit container, so the tensor
+// core sees a rounded rather than truncated operand.  Done on the integer ALU
+// (add half an ulp of tf32 to the magnitude bits, clear the 13 dropped bits):
+// a carry out of the mantissa bumps the exponent, which is the correct
+// rounding; infinities and NaNs keep their class.
 __device__ __forceinline__ float to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return __uint_as_float(r);
+    return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
+}
+__device__ __forceinline__ uint32_t tf32_bits(float x) {
+    return (__float_as_uint(x) + 0x1000u) & 0xFFFFE000u;
+}
+
+// Warp-level D += A * B with A 16x8 (row-major), B 8x8 (column-major), tf32
+// inputs and fp32 accumulation.  Fragment ownership (g = lane / 4, t = lane % 4):
+// a = {A[g][t], A[g+8][t], A[g][t+4], A[g+8][t+4]}, b = {B[t][g], B[t+4][g]},
+// d = {D[g][2t], D[g][2t+1], D[g+8][2t], D[g+8][2t+1]}.
+__device__ __forceinline__ void mma_m16n8k8_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
 __device__ __forceinline__ float ex2(float x) {
