@@ -32,10 +32,8 @@
 // recomputes the head-level chunk quantities (A, P, T').  Every MMA is
 // M = 128 (two 64-row operands stacked) with both operands K-major in shared
 // memory:
-//     [Kt ; Qt] x Kb^T     -> A (lanes 0-63), P (lanes 64-127)
-//     [Kt ; Qt] x St       -> Y (lanes 0-63), Z (lanes 64-127)
-//     [T' ; P]  x V        -> T'V (lanes 0-63; lanes 64-127 unused)
-//     [T' ; P]  x (-Y)     -> accumulated: lanes 0-63 = delta
+//     [Kt ; Qt] x [Kb^T | St] -> A | Y (lanes 0-63), P | Z (lanes 64-127), N = 96
+//     [T' ; P]  x (V - Y)   -> delta (lanes 0-63; lanes 64-127 unused)
 //     [T' ; P]  x delta    -> accumulated onto [Y ; Z]: lanes 64-127 = O
 //     Kb^T      x delta    -> accumulated onto St in TMEM: S_next
 // Block: 256 threads (8 warps); thread 0 issues TMA and MMA.  A warp may only
@@ -60,21 +58,21 @@ constexpr int kThreads = 256;
 constexpr uint32_t OFF_XQ = 0;         // 64 KB: [Kt ; Qt], 128 rows (token, token) x 128 channels
                                        //   = 4 K-blocks x 16 KB.  After the first MMA pair it is
                                        //   dead and holds the triangular solve's scratch.
-constexpr uint32_t OFF_KB = 65536;     // 32 KB: Kb, 64 rows (token) x 128 channels = 4 K-blocks x 8 KB.
+constexpr uint32_t OFF_KS = 65536;     // 48 KB: [Kb ; St^T], 96 rows x 128 channels = 4 K-blocks x 12 KB:
+                                       //   rows 0-63 Kb (token), rows 64-95 St^T (value column).
                                        //   Also the TMA destination of the next chunk's raw q, k.
-constexpr uint32_t OFF_KBT = 98304;    // 32 KB: Kb^T, 128 rows (channel) x 64 tokens = 2 K-blocks x 16 KB
-constexpr uint32_t OFF_TP = 131072;    // 32 KB: [T' ; P], 128 rows x 64 tokens = 2 K-blocks x 16 KB
-constexpr uint32_t OFF_ST = 163840;    // 16 KB: St^T, 32 rows (value col) x 128 channels = 4 x 4 KB
-constexpr uint32_t OFF_VT = 180224;    // 8 KB: V^T, 32 rows x 64 tokens = 2 x 4 KB
-constexpr uint32_t OFF_YT = 188416;    // 8 KB: (-Y)^T, later delta^T; during prep the Gamma exchange
-constexpr uint32_t OFF_MISC = 196608;  // beta[64], exp(Gamma_C)[128], barriers, TMEM address
-constexpr uint32_t SMEM_BYTES = OFF_MISC + 1024 + 1024;   // + alignment slack
+constexpr uint32_t OFF_KBT = 114688;   // 32 KB: Kb^T, 128 rows (channel) x 64 tokens = 2 K-blocks x 16 KB
+constexpr uint32_t OFF_TP = 147456;    // 32 KB: [T' ; P], 128 rows x 64 tokens = 2 K-blocks x 16 KB
+constexpr uint32_t OFF_VT = 180224;    // 8 KB: V^T, then (V - Y)^T: 32 rows x 64 tokens = 2 x 4 KB
+constexpr uint32_t OFF_YT = 188416;    // 8 KB: delta^T
+constexpr uint32_t OFF_MISC = 196608;  // beta[64], exp(Gamma_C)[128], Gamma exchange [8][128],
+                                       //   barriers, TMEM address
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 6144 + 1024;   // + alignment slack
 
 constexpr uint32_t KB_XQ = 16384;      // K-block strides
-constexpr uint32_t KB_KB = 8192;
+constexpr uint32_t KB_KS = 12288;
 constexpr uint32_t KB_KBT = 16384;
 constexpr uint32_t KB_TP = 16384;
-constexpr uint32_t KB_ST = 4096;
 constexpr uint32_t KB_VT = 4096;
 
 // Scratch of the triangular solve inside the dead XQ region: plain fp32
@@ -93,7 +91,7 @@ constexpr uint32_t TM_U = 96;     // 32 cols: T'V, then delta in lanes 0-63
 constexpr uint32_t TM_S = 128;    // 32 cols: state slice (key rows x 32 value cols)
 constexpr uint32_t TM_COLS = 256;
 
-constexpr uint32_t ID_N64 = idesc_tf32(128, 64, false, false);
+constexpr uint32_t ID_N96 = idesc_tf32(128, 96, false, false);
 constexpr uint32_t ID_N32 = idesc_tf32(128, 32, false, false);
 
 // Element (row, k) of a K-major operand tile at `base` with K-block stride `kb`.
@@ -138,9 +136,10 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(smem);
-    float* beta_s = reinterpret_cast<float*>(smem + OFF_MISC);     // 64
-    float* dc_s = beta_s + 64;                                      // 128: exp(Gamma_C)
-    uint64_t* bar_load = reinterpret_cast<uint64_t*>(smem + OFF_MISC + 768);
+    float* beta_s = reinterpret_cast<float*>(smem + OFF_MISC);            // 64
+    float* dc_s = beta_s + 64;                                             // 128: exp(Gamma_C)
+    float* xch = reinterpret_cast<float*>(smem + OFF_MISC + 1024);         // [8 warps][128]
+    uint64_t* bar_load = reinterpret_cast<uint64_t*>(smem + OFF_MISC + 5120);
     uint64_t* bar_mma = bar_load + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_mma + 1);
 
@@ -195,8 +194,8 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tmem_wait_st();
     }
 
-    // register-staged inputs of the next chunk: g (8 rows x 4 channels),
-    // the thread's 8 values of the V slice, and beta
+    // Register-staged inputs of the next chunk: g (8 rows x 4 channels), the
+    // thread's 8 values of the V slice, and beta.
     float greg[8][4];
     uint4 vreg;
     float breg;
@@ -215,183 +214,205 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         breg = 0.f;
         if (tid < L) breg = __ldg(beta + (size_t)(t0 + tid) * H + h);
     };
-    // raw q and k tiles (64 tokens x 128 channels, bf16) into the Kb region
+    // raw q and k tiles (64 tokens x 128 channels, bf16) into the [Kb ; St^T] region
     auto issue_load = [&](int64_t t0) {
         mbar_arrive_expect_tx(bar_load, 2u * kC * kD * 2u);
-        tma_load_3d(smem + OFF_KB, &tm_q, bar_load, 0, h, static_cast<int32_t>(t0));
-        tma_load_3d(smem + OFF_KB + kC * kD * 2, &tm_k, bar_load, 0, h, static_cast<int32_t>(t0));
+        tma_load_3d(smem + OFF_KS, &tm_q, bar_load, 0, h, static_cast<int32_t>(t0));
+        tma_load_3d(smem + OFF_KS + kC * kD * 2, &tm_k, bar_load, 0, h, static_cast<int32_t>(t0));
+    };
+
+    // Prep of one chunk (state independent): Gamma, L2 norms, the tf32 tiles
+    // Kt, Qt (XQ), Kb (rows 0-63 of KS) and V^T, plus beta and exp(Gamma_C).
+    // Contains one block barrier; every thread must call it.
+    auto prep = [&](int L) {
+        // raw q, k of the thread's 8 rows x 4 channels into registers first:
+        // the tiles written below overwrite the raw staging area
+        uint2 qraw[8], kraw[8];
+        const uint8_t* rq = smem + OFF_KS;
+        const uint8_t* rk = smem + OFF_KS + kC * kD * 2;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            const int r = 8 * warp + m;
+            qraw[m] = *reinterpret_cast<const uint2*>(rq + r * kD * 2 + lane * 8);
+            kraw[m] = *reinterpret_cast<const uint2*>(rk + r * kD * 2 + lane * 8);
+        }
+        // Gamma in log2 units, as channel pairs: prefix over the thread's 8 rows,
+        // then over warps through shared memory
+        const float2 l2e = make_float2(kLog2e, kLog2e);
+        float2 G[8][2];
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+            float2 run = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                run = __ffma2_rn(make_float2(greg[m][2 * x], greg[m][2 * x + 1]), l2e, run);
+                G[m][x] = run;
+            }
+            *reinterpret_cast<float2*>(xch + warp * 128 + 4 * lane + 2 * x) = run;
+        }
+        __syncthreads();   // also: every thread holds its raw q, k in registers
+        float2 off[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        float2 GC[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+        for (int w = 0; w < 8; ++w) {
+            const float4 t = *reinterpret_cast<const float4*>(xch + w * 128 + 4 * lane);
+            if (w < warp) {
+                off[0] = __fadd2_rn(off[0], make_float2(t.x, t.y));
+                off[1] = __fadd2_rn(off[1], make_float2(t.z, t.w));
+            }
+            GC[0] = __fadd2_rn(GC[0], make_float2(t.x, t.y));
+            GC[1] = __fadd2_rn(GC[1], make_float2(t.z, t.w));
+        }
+        if (warp == 0) {
+            dc_s[4 * lane + 0] = ex2(GC[0].x); dc_s[4 * lane + 1] = ex2(GC[0].y);
+            dc_s[4 * lane + 2] = ex2(GC[1].x); dc_s[4 * lane + 3] = ex2(GC[1].y);
+        }
+        if (tid < kC) beta_s[tid] = breg;
+        // offset to the chunk end: Gamma_r - Gamma_C = G + (off - GC)
+        const float2 rel[2] = {__fadd2_rn(off[0], make_float2(-GC[0].x, -GC[0].y)),
+                               __fadd2_rn(off[1], make_float2(-GC[1].x, -GC[1].y))};
+
+        // unpack, mask rows past the sequence end, and L2-normalise all 8 rows
+        float2 qv[8][2], kv[8][2];
+        float nrm[16];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            const bool live = 8 * warp + m < L;
+            qv[m][0] = make_float2(__uint_as_float(qraw[m].x << 16), __uint_as_float(qraw[m].x & 0xFFFF0000u));
+            qv[m][1] = make_float2(__uint_as_float(qraw[m].y << 16), __uint_as_float(qraw[m].y & 0xFFFF0000u));
+            kv[m][0] = make_float2(__uint_as_float(kraw[m].x << 16), __uint_as_float(kraw[m].x & 0xFFFF0000u));
+            kv[m][1] = make_float2(__uint_as_float(kraw[m].y << 16), __uint_as_float(kraw[m].y & 0xFFFF0000u));
+            if (!live) {
+                qv[m][0] = qv[m][1] = kv[m][0] = kv[m][1] = make_float2(0.f, 0.f);
+            }
+            const float2 sq = __ffma2_rn(qv[m][1], qv[m][1], __fmul2_rn(qv[m][0], qv[m][0]));
+            const float2 sk = __ffma2_rn(kv[m][1], kv[m][1], __fmul2_rn(kv[m][0], kv[m][0]));
+            nrm[m] = sq.x + sq.y;
+            nrm[8 + m] = sk.x + sk.y;
+        }
+        if (l2norm) warp_allreduce16(nrm);
+        const int kbi = lane >> 3, ch = lane & 7;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            const int r = 8 * warp + m;
+            const float nq = (l2norm ? rsqrtf(nrm[m] + kNormEps) : 1.f) * scale;
+            const float nk = l2norm ? rsqrtf(nrm[8 + m] + kNormEps) : 1.f;
+            float4 kt, qt, kb;
+            float* ktp = &kt.x;
+            float* qtp = &qt.x;
+            float* kbp = &kb.x;
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                // a = (Gamma_r - Gamma_C) / ln 2 >= 0 (the decay is cumulative, g <= 0)
+                const float2 a = __fadd2_rn(G[m][x], rel[x]);
+                const float2 e = make_float2(ex2(fminf(a.x, 126.f)), ex2(fminf(a.y, 126.f)));   // E >= 1
+                const float2 f = make_float2(ex2(-a.x), ex2(-a.y));                              // F <= 1
+                const float2 kn = __fmul2_rn(kv[m][x], make_float2(nk, nk));
+                const float2 qn = __fmul2_rn(qv[m][x], make_float2(nq, nq));
+                const float2 t1 = __fmul2_rn(kn, e), t2 = __fmul2_rn(qn, e), t3 = __fmul2_rn(kn, f);
+                ktp[2 * x] = t1.x; ktp[2 * x + 1] = t1.y;
+                qtp[2 * x] = t2.x; qtp[2 * x + 1] = t2.y;
+                kbp[2 * x] = t3.x; kbp[2 * x + 1] = t3.y;
+            }
+            st_tf32x4(smem, OFF_XQ + kbi * KB_XQ + sw128_off(r, ch), kt.x, kt.y, kt.z, kt.w);
+            st_tf32x4(smem, OFF_XQ + kbi * KB_XQ + sw128_off(64 + r, ch), qt.x, qt.y, qt.z, qt.w);
+            st_tf32x4(smem, OFF_KS + kbi * KB_KS + sw128_off(r, ch), kb.x, kb.y, kb.z, kb.w);
+        }
+        {   // V^T: token tid/4, value columns 8*(tid%4) .. +7 (exact bf16 -> fp32)
+            const int r = tid >> 2, j0 = 8 * (tid & 3);
+            const uint32_t w4[4] = {vreg.x, vreg.y, vreg.z, vreg.w};
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                *K_at(smem, OFF_VT, KB_VT, j0 + 2 * x, r) = __uint_as_float(w4[x] << 16);
+                *K_at(smem, OFF_VT, KB_VT, j0 + 2 * x + 1, r) = __uint_as_float(w4[x] & 0xFFFF0000u);
+            }
+        }
     };
 
     bool ok = true;
     uint32_t mma_phase = 0, load_parity = 0;
     bool load_pending = false, mma_pending = false;
-    if (nchunks > 0) {
+    auto wait_mma = [&]() -> bool {
+        const bool good = !__syncthreads_or(!mbar_wait_bounded(bar_mma, mma_phase));
+        if (good) {
+            mma_phase ^= 1;
+            mma_pending = false;
+            tc_fence_after();
+        }
+        return good;
+    };
+
+    if (nchunks > 0) {   // prologue: stage and prep chunk 0
         if (tid == 0) issue_load(bos);
         load_pending = true;
         prefetch(bos, static_cast<int>(len < kC ? len : (int64_t)kC));
+        ok = !__syncthreads_or(!mbar_wait_bounded(bar_load, 0));
+        if (ok) {
+            load_pending = false;
+            prep(static_cast<int>(len < kC ? len : (int64_t)kC));
+        }
     }
-    tc_fence_before();
-    __syncthreads();
 
-    for (int c = 0; c < nchunks; ++c) {
+    for (int c = 0; ok && c < nchunks; ++c) {
         const int64_t t0 = bos + (int64_t)c * kC;
         const int L = static_cast<int>(eos - t0 < kC ? eos - t0 : (int64_t)kC);
+        const bool has_next = c + 1 < nchunks;
+        const int Ln = has_next ? static_cast<int>(eos - t0 - kC < kC ? eos - t0 - kC : (int64_t)kC) : 0;
+        tc_fence_before();
+        __syncthreads();   // prep(c) done; the previous chunk's TMEM reads done
 
-        ok = !__syncthreads_or(!mbar_wait_bounded(bar_load, c & 1));
-        if (!ok) break;
-        load_pending = false;
-
-        // ================================================== prep
-        {
-            // raw q, k of the thread's 8 rows x 4 channels into registers first:
-            // the tiles written below overwrite the raw staging area
-            uint2 qraw[8], kraw[8];
-            const uint8_t* rq = smem + OFF_KB;
-            const uint8_t* rk = smem + OFF_KB + kC * kD * 2;
+        // ============== Kb^T, and the state decayed to the chunk end
+        {   // Kb^T from Kb: thread = channel c, 4 consecutive tokens per 16-byte store
+            const int cch = tid & 127, tg = tid >> 7;
 #pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const int r = 8 * warp + m;
-                qraw[m] = *reinterpret_cast<const uint2*>(rq + r * kD * 2 + lane * 8);
-                kraw[m] = *reinterpret_cast<const uint2*>(rk + r * kD * 2 + lane * 8);
+            for (int b = 0; b < 8; ++b) {
+                const int i0 = 32 * tg + 4 * b;
+                float4 x;
+                x.x = *K_at(smem, OFF_KS, KB_KS, i0 + 0, cch);
+                x.y = *K_at(smem, OFF_KS, KB_KS, i0 + 1, cch);
+                x.z = *K_at(smem, OFF_KS, KB_KS, i0 + 2, cch);
+                x.w = *K_at(smem, OFF_KS, KB_KS, i0 + 3, cch);
+                *reinterpret_cast<float4*>(K_at(smem, OFF_KBT, KB_KBT, cch, i0)) = x;
             }
-            // Gamma (log2 units): prefix over the thread's 8 rows, then over warps
-            float* xch = reinterpret_cast<float*>(smem + OFF_YT);   // [8 warps][128]
-            float G[8][4];
+        }
+        {   // St = Diag(exp(Gamma_C)) S in TMEM (fp32) and as St^T (tf32, rows 64-95 of KS);
+            // the two warps of a TMEM lane quarter take 16 value columns each
+            float acc[16];
+            const int c0 = 16 * half;
+            tc_fence_after();
+            tmem_ld16(tm_lane(tmem, quarter, TM_S + c0), acc);
+            tmem_wait_ld();
+            const int row = 32 * quarter + lane;
+            const float dcr = dc_s[row];
 #pragma unroll
-            for (int x = 0; x < 4; ++x) {
-                float run = 0.f;
+            for (int e = 0; e < 16; ++e) acc[e] *= dcr;
+            tmem_st16(tm_lane(tmem, quarter, TM_S + c0), acc);
 #pragma unroll
-                for (int m = 0; m < 8; ++m) {
-                    run = fmaf(greg[m][x], kLog2e, run);
-                    G[m][x] = run;
-                }
-                xch[warp * 128 + 4 * lane + x] = run;
-            }
-            __syncthreads();   // also: every thread has its raw q, k in registers
-            float off[4] = {0.f, 0.f, 0.f, 0.f}, GC[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int w = 0; w < 8; ++w) {
-                const float4 t = *reinterpret_cast<const float4*>(xch + w * 128 + 4 * lane);
-                if (w < warp) { off[0] += t.x; off[1] += t.y; off[2] += t.z; off[3] += t.w; }
-                GC[0] += t.x; GC[1] += t.y; GC[2] += t.z; GC[3] += t.w;
-            }
-            if (warp == 0) {
-#pragma unroll
-                for (int x = 0; x < 4; ++x) dc_s[4 * lane + x] = ex2(GC[x]);
-            }
-            if (tid < kC) beta_s[tid] = breg;
-
-            // unpack, mask rows past the sequence end, and L2-normalise all 8 rows
-            float qv[8][4], kv[8][4];
-            float nrm[16];
-#pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const bool live = 8 * warp + m < L;
-                qv[m][0] = __uint_as_float(qraw[m].x << 16); qv[m][1] = __uint_as_float(qraw[m].x & 0xFFFF0000u);
-                qv[m][2] = __uint_as_float(qraw[m].y << 16); qv[m][3] = __uint_as_float(qraw[m].y & 0xFFFF0000u);
-                kv[m][0] = __uint_as_float(kraw[m].x << 16); kv[m][1] = __uint_as_float(kraw[m].x & 0xFFFF0000u);
-                kv[m][2] = __uint_as_float(kraw[m].y << 16); kv[m][3] = __uint_as_float(kraw[m].y & 0xFFFF0000u);
-                float sq = 0.f, sk = 0.f;
-#pragma unroll
-                for (int x = 0; x < 4; ++x) {
-                    if (!live) { qv[m][x] = 0.f; kv[m][x] = 0.f; }
-                    sq = fmaf(qv[m][x], qv[m][x], sq);
-                    sk = fmaf(kv[m][x], kv[m][x], sk);
-                }
-                nrm[m] = sq;
-                nrm[8 + m] = sk;
-            }
-            if (l2norm) warp_allreduce16(nrm);
-#pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const int r = 8 * warp + m;
-                const float nq = (l2norm ? rsqrtf(nrm[m] + kNormEps) : 1.f) * scale;
-                const float nk = l2norm ? rsqrtf(nrm[8 + m] + kNormEps) : 1.f;
-                float kt[4], qt[4], kb[4];
-#pragma unroll
-                for (int x = 0; x < 4; ++x) {
-                    const float gr = G[m][x] + off[x];
-                    const float e = ex2(fminf(gr - GC[x], 126.f));   // exp(Gamma_r - Gamma_C) >= 1
-                    const float f = ex2(GC[x] - gr);                 // exp(Gamma_C - Gamma_r) <= 1
-                    const float kn = kv[m][x] * nk;
-                    kt[x] = kn * e;
-                    kb[x] = kn * f;
-                    qt[x] = qv[m][x] * nq * e;
-                }
-                const int kbi = lane >> 3, ch = lane & 7;
-                st_tf32x4(smem, OFF_XQ + kbi * KB_XQ + sw128_off(r, ch), kt[0], kt[1], kt[2], kt[3]);
-                st_tf32x4(smem, OFF_XQ + kbi * KB_XQ + sw128_off(64 + r, ch), qt[0], qt[1], qt[2], qt[3]);
-                st_tf32x4(smem, OFF_KB + kbi * KB_KB + sw128_off(r, ch), kb[0], kb[1], kb[2], kb[3]);
-            }
-            {   // V^T: token tid/4, value columns 8*(tid%4) .. +7 (exact bf16 -> fp32)
-                const int r = tid >> 2, j0 = 8 * (tid & 3);
-                const uint32_t w4[4] = {vreg.x, vreg.y, vreg.z, vreg.w};
-#pragma unroll
-                for (int x = 0; x < 4; ++x) {
-                    *K_at(smem, OFF_VT, KB_VT, j0 + 2 * x, r) = __uint_as_float(w4[x] << 16);
-                    *K_at(smem, OFF_VT, KB_VT, j0 + 2 * x + 1, r) = __uint_as_float(w4[x] & 0xFFFF0000u);
-                }
-            }
-            __syncthreads();   // Kb complete and exp(Gamma_C) known
-            {   // Kb^T from Kb: thread = channel c, 4 consecutive tokens per 16-byte store
-                const int cch = tid & 127, tg = tid >> 7;
-#pragma unroll
-                for (int b = 0; b < 8; ++b) {
-                    const int i0 = 32 * tg + 4 * b;
-                    float4 x;
-                    x.x = *K_at(smem, OFF_KB, KB_KB, i0 + 0, cch);
-                    x.y = *K_at(smem, OFF_KB, KB_KB, i0 + 1, cch);
-                    x.z = *K_at(smem, OFF_KB, KB_KB, i0 + 2, cch);
-                    x.w = *K_at(smem, OFF_KB, KB_KB, i0 + 3, cch);
-                    *reinterpret_cast<float4*>(K_at(smem, OFF_KBT, KB_KBT, cch, i0)) = x;
-                }
-            }
-            {   // St = Diag(exp(Gamma_C)) S in TMEM (fp32) and as St^T (tf32); the two
-                // warps of a TMEM lane quarter take 16 value columns each
-                float acc[16];
-                const int c0 = 16 * half;
-                tc_fence_after();
-                tmem_ld16(tm_lane(tmem, quarter, TM_S + c0), acc);
-                tmem_wait_ld();
-                const int row = 32 * quarter + lane;
-                const float dcr = dc_s[row];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) acc[e] *= dcr;
-                tmem_st16(tm_lane(tmem, quarter, TM_S + c0), acc);
-#pragma unroll
-                for (int e = 0; e < 16; ++e) *K_at(smem, OFF_ST, KB_ST, c0 + e, row) = to_tf32(acc[e]);
-                tmem_wait_st();
-            }
+            for (int e = 0; e < 16; ++e) *K_at(smem, OFF_KS, KB_KS, 64 + c0 + e, row) = to_tf32(acc[e]);
+            tmem_wait_st();
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
 
-        // ================================ [A ; P] and [Y ; Z] (one commit)
+        // ============== [Kt ; Qt] x [Kb ; St^T]^T -> [A | Y] (lanes 0-63), [P | Z] (64-127)
         if (tid == 0) {
             tc_fence_after();
-            const uint64_t dxq = tdesc(sb, OFF_XQ), dkb = tdesc(sb, OFF_KB), dst = tdesc(sb, OFF_ST);
+            const uint64_t dxq = tdesc(sb, OFF_XQ), dks = tdesc(sb, OFF_KS);
 #pragma unroll
             for (int s = 0; s < 16; ++s)
-                mma_tf32_ss(tmem + TM_AP, kstep(dxq, KB_XQ, s), kstep(dkb, KB_KB, s), ID_N64, s > 0);
-#pragma unroll
-            for (int s = 0; s < 16; ++s)
-                mma_tf32_ss(tmem + TM_X, kstep(dxq, KB_XQ, s), kstep(dst, KB_ST, s), ID_N32, s > 0);
+                mma_tf32_ss(tmem + TM_AP, kstep(dxq, KB_XQ, s), kstep(dks, KB_KS, s), ID_N96, s > 0);
             mma_commit(bar_mma);
         }
         mma_pending = true;
-        if (c + 1 < nchunks) prefetch(t0 + kC, static_cast<int>(eos - t0 - kC < kC ? eos - t0 - kC : (int64_t)kC));
-        ok = !__syncthreads_or(!mbar_wait_bounded(bar_mma, mma_phase));
-        if (!ok) break;
-        mma_phase ^= 1;
-        mma_pending = false;
-        tc_fence_after();
-        // Kb (and XQ) are free now: stage the next chunk's q, k
-        if (tid == 0 && c + 1 < nchunks) issue_load(t0 + kC);
-        load_pending = (c + 1 < nchunks);
+        if (has_next) prefetch(t0 + kC, Ln);
+        if (!(ok = wait_mma())) break;
+        // XQ and KS are free now: stage the next chunk's q, k
+        if (tid == 0 && has_next) issue_load(t0 + kC);
+        load_pending = has_next;
         load_parity = (c + 1) & 1;
 
-        // ============== A -> M (fp32), P -> tf32 operand, -Y -> (-Y)^T operand
+        // ============== A -> M (fp32), P -> tf32 operand
         {
             float acc[32];
             tmem_ld32(tm_lane(tmem, quarter, TM_AP + 32 * half), acc);
@@ -424,8 +445,8 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tc_fence_before();
         __syncthreads();
 
-        // ============== T = (I + M)^-1 by 16-blocks (plain fp32 arrays, row
-        // stride kLd), then T' = T diag(beta) into the swizzled operand
+        // ============== T = (I + M)^-1 by 16-blocks, then T' = T diag(beta);
+        // meanwhile V^T -> (V - Y)^T
         {
             float* Mf = reinterpret_cast<float*>(smem + OFF_M);
             float* Tf = reinterpret_cast<float*>(smem + OFF_T);
@@ -437,13 +458,13 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 float xv[16];
 #pragma unroll
                 for (int r = 0; r < 16; ++r) {
-                    float s0 = (r == j) ? 1.f : 0.f, s1 = 0.f;
+                    float s0v = (r == j) ? 1.f : 0.f, s1v = 0.f;
 #pragma unroll
                     for (int i = 0; i < r; i += 2) {
-                        s0 = fmaf(-Mb[r * kLd + i], xv[i], s0);
-                        if (i + 1 < r) s1 = fmaf(-Mb[r * kLd + i + 1], xv[i + 1], s1);
+                        s0v = fmaf(-Mb[r * kLd + i], xv[i], s0v);
+                        if (i + 1 < r) s1v = fmaf(-Mb[r * kLd + i + 1], xv[i + 1], s1v);
                     }
-                    xv[r] = s0 + s1;
+                    xv[r] = s0v + s1v;
                 }
                 float* Tb = Tf + 16 * b * kLd + 16 * b + j;
 #pragma unroll
@@ -453,30 +474,33 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 float* z = Tf + (32 * blk + rr) * kLd + 32 * blk + 16 + c8;
                 *reinterpret_cast<float4*>(z) = make_float4(0.f, 0.f, 0.f, 0.f);
                 *reinterpret_cast<float4*>(z + 4) = make_float4(0.f, 0.f, 0.f, 0.f);
-            } else if (warp == 4 || warp == 5) {   // -Y (token rows 0-63) -> (-Y)^T operand
+            } else if (warp == 4 || warp == 5) {   // V^T -> (V - Y)^T for token rows 0-63
                 float y[32];
                 tc_fence_after();
                 tmem_ld32(tm_lane(tmem, quarter, TM_X), y);
                 tmem_wait_ld();
                 const int r = 32 * quarter + lane;
 #pragma unroll
-                for (int e = 0; e < 32; ++e) *K_at(smem, OFF_YT, KB_VT, e, r) = to_tf32(-y[e]);
+                for (int e = 0; e < 32; ++e) {
+                    float* pv = K_at(smem, OFF_VT, KB_VT, e, r);
+                    *pv = to_tf32(*pv - y[e]);
+                }
             }
             __syncthreads();
             {   // 16 -> 32 on tensor cores: T_ab = -T_aa (M_ab T_bb) for (a, b) = (1, 0), (3, 2);
                 // warp w < 4 owns pair p = w / 2, output columns 8 (w % 2) .. +7
-                const int g = lane >> 2, t = lane & 3;
+                const int gq = lane >> 2, tq = lane & 3;
                 const int p = warp >> 1, nt = warp & 1, a = 2 * p + 1, b = 2 * p;
                 if (warp < 4) {
                     float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int ks = 0; ks < 2; ++ks) {
                         uint32_t fa[4], fb[2];
-                        frag_a(fa, Mf, kLd, 16 * a, 16 * b + 8 * ks, g, t);
-                        frag_b(fb, Tf, kLd, 16 * b + 8 * ks, 16 * b + 8 * nt, g, t);
+                        frag_a(fa, Mf, kLd, 16 * a, 16 * b + 8 * ks, gq, tq);
+                        frag_b(fb, Tf, kLd, 16 * b + 8 * ks, 16 * b + 8 * nt, gq, tq);
                         mma_m16n8k8_tf32(d, fa, fb);
                     }
-                    frag_store(Y1 + p * 16 * kLd1, kLd1, 0, 8 * nt, d, 1.f, g, t);
+                    frag_store(Y1 + p * 16 * kLd1, kLd1, 0, 8 * nt, d, 1.f, gq, tq);
                 }
                 __syncthreads();
                 if (warp < 4) {
@@ -484,37 +508,37 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
                     for (int ks = 0; ks < 2; ++ks) {
                         uint32_t fa[4], fb[2];
-                        frag_a(fa, Tf, kLd, 16 * a, 16 * a + 8 * ks, g, t);
-                        frag_b(fb, Y1 + p * 16 * kLd1, kLd1, 8 * ks, 8 * nt, g, t);
+                        frag_a(fa, Tf, kLd, 16 * a, 16 * a + 8 * ks, gq, tq);
+                        frag_b(fb, Y1 + p * 16 * kLd1, kLd1, 8 * ks, 8 * nt, gq, tq);
                         mma_m16n8k8_tf32(d, fa, fb);
                     }
-                    frag_store(Tf, kLd, 16 * a, 16 * b + 8 * nt, d, -1.f, g, t);
+                    frag_store(Tf, kLd, 16 * a, 16 * b + 8 * nt, d, -1.f, gq, tq);
                 }
             }
             __syncthreads();
             {   // 32 -> 64 on tensor cores: T_hl = -T_hh (M_hl T_ll); warp w owns the
                 // 16 x 8 output tile (rows 16 (w / 4), columns 8 (w % 4))
-                const int g = lane >> 2, t = lane & 3;
+                const int gq = lane >> 2, tq = lane & 3;
                 const int mt = warp >> 2, nt = warp & 3;
                 float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
                     uint32_t fa[4], fb[2];
-                    frag_a(fa, Mf, kLd, 32 + 16 * mt, 8 * ks, g, t);
-                    frag_b(fb, Tf, kLd, 8 * ks, 8 * nt, g, t);
+                    frag_a(fa, Mf, kLd, 32 + 16 * mt, 8 * ks, gq, tq);
+                    frag_b(fb, Tf, kLd, 8 * ks, 8 * nt, gq, tq);
                     mma_m16n8k8_tf32(d, fa, fb);
                 }
-                frag_store(Y2, kLd2, 16 * mt, 8 * nt, d, 1.f, g, t);
+                frag_store(Y2, kLd2, 16 * mt, 8 * nt, d, 1.f, gq, tq);
                 __syncthreads();
-                float e[4] = {0.f, 0.f, 0.f, 0.f};
+                float e4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
                     uint32_t fa[4], fb[2];
-                    frag_a(fa, Tf, kLd, 32 + 16 * mt, 32 + 8 * ks, g, t);
-                    frag_b(fb, Y2, kLd2, 8 * ks, 8 * nt, g, t);
-                    mma_m16n8k8_tf32(e, fa, fb);
+                    frag_a(fa, Tf, kLd, 32 + 16 * mt, 32 + 8 * ks, gq, tq);
+                    frag_b(fb, Y2, kLd2, 8 * ks, 8 * nt, gq, tq);
+                    mma_m16n8k8_tf32(e4, fa, fb);
                 }
-                frag_store(Tf, kLd, 32 + 16 * mt, 8 * nt, e, -1.f, g, t);
+                frag_store(Tf, kLd, 32 + 16 * mt, 8 * nt, e4, -1.f, gq, tq);
             }
             __syncthreads();
             {   // T' = T diag(beta) on and below the diagonal, zero above; tf32 operand
@@ -534,24 +558,17 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tc_fence_before();
         __syncthreads();
 
-        // ============== delta = T' V + T' (-Y)   (lanes 0-63 of TM_U)
+        // ============== delta = T' (V - Y)   (lanes 0-63 of TM_U)
         if (tid == 0) {
             tc_fence_after();
-            const uint64_t dtp = tdesc(sb, OFF_TP), dvt = tdesc(sb, OFF_VT), dyt = tdesc(sb, OFF_YT);
+            const uint64_t dtp = tdesc(sb, OFF_TP), dvt = tdesc(sb, OFF_VT);
 #pragma unroll
             for (int s = 0; s < 8; ++s)
                 mma_tf32_ss(tmem + TM_U, kstep(dtp, KB_TP, s), kstep(dvt, KB_VT, s), ID_N32, s > 0);
-#pragma unroll
-            for (int s = 0; s < 8; ++s)
-                mma_tf32_ss(tmem + TM_U, kstep(dtp, KB_TP, s), kstep(dyt, KB_VT, s), ID_N32, 1);
             mma_commit(bar_mma);
         }
         mma_pending = true;
-        ok = !__syncthreads_or(!mbar_wait_bounded(bar_mma, mma_phase));
-        if (!ok) break;
-        mma_phase ^= 1;
-        mma_pending = false;
-        tc_fence_after();
+        if (!(ok = wait_mma())) break;
 
         // ============== delta -> delta^T operand (token rows 0-63)
         if (quarter < 2) {   // two warps per lane quarter, 16 value columns each
@@ -579,11 +596,15 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             mma_commit(bar_mma);
         }
         mma_pending = true;
-        ok = !__syncthreads_or(!mbar_wait_bounded(bar_mma, mma_phase));
-        if (!ok) break;
-        mma_phase ^= 1;
-        mma_pending = false;
-        tc_fence_after();
+
+        // ============== while those run: prep of the next chunk (touches neither
+        // TP, Kb^T, delta^T nor tensor memory)
+        if (has_next) {
+            if (!(ok = !__syncthreads_or(!mbar_wait_bounded(bar_load, (c + 1) & 1)))) break;
+            load_pending = false;
+            prep(Ln);
+        }
+        if (!(ok = wait_mma())) break;
 
         // ============== O (token rows in lanes 64-127) -> global
         if (warp == 2 || warp == 3) {
@@ -598,10 +619,10 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     dst[j] = make_float4(acc[4 * j], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]);
             }
         }
-        tc_fence_before();
-        __syncthreads();
     }
 
+    tc_fence_before();
+    __syncthreads();
     if (ok) {
         if (sT && warp < 4) {
             float acc[32];
