@@ -43,7 +43,8 @@ int kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g, c
     if (N < 0 || H <= 0 || total_T < 0 || total_T >= (int64_t(1) << 31)) return KDA_ERR_INVALID_ARG;
     if (d != 128) return KDA_ERR_UNSUPPORTED;
     if (dt != KDA_DTYPE_BF16 && dt != KDA_DTYPE_FP32) return KDA_ERR_UNSUPPORTED;
-    if (flags & ~uint32_t(KDA_FLAG_L2NORM_QK | KDA_FLAG_RECURRENT)) return KDA_ERR_UNSUPPORTED;
+    if (flags & ~uint32_t(KDA_FLAG_L2NORM_QK | KDA_FLAG_RECURRENT | KDA_FLAG_SCALAR_DECAY))
+        return KDA_ERR_UNSUPPORTED;
     if (cu_seqlens == nullptr) return KDA_ERR_INVALID_ARG;
     if (total_T > 0 && (!q || !k || !v || !g || !beta || !o)) return KDA_ERR_INVALID_ARG;
     const void* ptrs[] = {q, k, v, g, beta, initial_state, final_state, o, workspace};
@@ -60,7 +61,8 @@ int kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g, c
     if (N == 0) return KDA_OK;
 
     kda::PrefillArgs a{q, k, v, g, beta, cu_seqlens, N, total_T, H, dt == KDA_DTYPE_BF16, scale,
-                       (flags & KDA_FLAG_L2NORM_QK) != 0, initial_state, final_state, o, err};
+                       (flags & KDA_FLAG_L2NORM_QK) != 0, (flags & KDA_FLAG_SCALAR_DECAY) != 0,
+                       initial_state, final_state, o, err};
     const bool recurrent = (dt == KDA_DTYPE_FP32) || (flags & KDA_FLAG_RECURRENT) || total_T == 0;
     const cudaError_t e = recurrent ? kda::launch_recurrent(a, s) : kda::launch_chunk(a, s);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
@@ -72,7 +74,7 @@ int kda_decode_step(const void* q, const void* k, const void* v, const float* g,
     if (N < 0 || H <= 0 || static_cast<int64_t>(N) * H >= (int64_t(1) << 31)) return KDA_ERR_INVALID_ARG;
     if (d != 128) return KDA_ERR_UNSUPPORTED;
     if (dt != KDA_DTYPE_BF16 && dt != KDA_DTYPE_FP32) return KDA_ERR_UNSUPPORTED;
-    if (flags & ~uint32_t(KDA_FLAG_L2NORM_QK)) return KDA_ERR_UNSUPPORTED;
+    if (flags & ~uint32_t(KDA_FLAG_L2NORM_QK | KDA_FLAG_SCALAR_DECAY)) return KDA_ERR_UNSUPPORTED;
     if (N == 0) return KDA_OK;
     if (!q || !k || !v || !g || !beta || !state || !o) return KDA_ERR_INVALID_ARG;
     const void* ptrs[] = {q, k, v, g, beta, state, o};
@@ -81,7 +83,7 @@ int kda_decode_step(const void* q, const void* k, const void* v, const float* g,
     int status = KDA_OK;
     if (!device_is_sm100(&status)) return status;
     kda::DecodeArgs a{q, k, v, g, beta, state, o, N, H, dt == KDA_DTYPE_BF16, scale,
-                      (flags & KDA_FLAG_L2NORM_QK) != 0};
+                      (flags & KDA_FLAG_L2NORM_QK) != 0, (flags & KDA_FLAG_SCALAR_DECAY) != 0};
     return kda::launch_decode(a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? KDA_OK
                                                                                          : KDA_ERR_CUDA;
 }

@@ -131,8 +131,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __nv_bfloat16* __restrict__ v, const float* __restrict__ g,
                  const float* __restrict__ beta, const int32_t* __restrict__ cu_seqlens,
-                 int64_t total_T, int H, float scale, int l2norm, const float* s0, float* sT,
-                 float* __restrict__ o, uint32_t* err) {
+                 int64_t total_T, int H, float scale, int l2norm, int scalar_g, const float* s0,
+                 float* sT, float* __restrict__ o, uint32_t* err) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(smem);
@@ -204,7 +204,14 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         for (int m = 0; m < 8; ++m) {
             const int r = 8 * warp + m;
             float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (r < L) x = __ldg(reinterpret_cast<const float4*>(g + ((size_t)(t0 + r) * H + h) * kD + 4 * lane));
+            if (r < L) {
+                if (scalar_g) {   // one decay per (token, head), shared by all channels
+                    const float gs = __ldg(g + (size_t)(t0 + r) * H + h);
+                    x = make_float4(gs, gs, gs, gs);
+                } else {
+                    x = __ldg(reinterpret_cast<const float4*>(g + ((size_t)(t0 + r) * H + h) * kD + 4 * lane));
+                }
+            }
             greg[m][0] = x.x; greg[m][1] = x.y; greg[m][2] = x.z; greg[m][3] = x.w;
         }
         const int vr = tid >> 2;
@@ -700,7 +707,7 @@ cudaError_t launch_chunk(const PrefillArgs& a, cudaStream_t stream) {
     const long long blocks = (long long)a.N * a.H * kSplit;
     kda_chunk_kernel<<<static_cast<unsigned>(blocks), kThreads, SMEM_BYTES, stream>>>(
         mq, mk, static_cast<const __nv_bfloat16*>(a.v), a.g, a.beta, a.cu_seqlens, a.total_T, a.H, a.scale,
-        a.l2norm ? 1 : 0, a.initial_state, a.final_state, a.o, a.err);
+        a.l2norm ? 1 : 0, a.scalar_decay ? 1 : 0, a.initial_state, a.final_state, a.o, a.err);
     return cudaGetLastError();
 }
 

@@ -28,7 +28,7 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads, 2)
 kda_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                   const float* __restrict__ g, const float* __restrict__ beta,
-                  float* __restrict__ state, float* __restrict__ o, float scale, int l2norm) {
+                  float* __restrict__ state, float* __restrict__ o, float scale, int l2norm, int scalar_g) {
     __shared__ float ak[kD], aq[kD], al[kD], kh[kD];
     __shared__ float4 red[8][2][32];
     __shared__ float qk_dot;
@@ -47,7 +47,11 @@ kda_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
         float qv[4], kv[4], gv[4];
         load4(q + (size_t)p * kD + lane * 4, qv);
         load4(k + (size_t)p * kD + lane * 4, kv);
-        load4(g + (size_t)p * kD + lane * 4, gv);
+        if (scalar_g) {   // one decay per (sequence, head), shared by all channels
+            gv[0] = gv[1] = gv[2] = gv[3] = g[p];
+        } else {
+            load4(g + (size_t)p * kD + lane * 4, gv);
+        }
         float rq = 1.f, rk = 1.f;
         if (l2norm) {
             float sq = 0.f, sk = 0.f;
@@ -129,11 +133,12 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
         kda_decode_kernel<__nv_bfloat16><<<(unsigned)pairs, kThreads, 0, stream>>>(
             static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
             static_cast<const __nv_bfloat16*>(a.v), a.g, a.beta, a.state, a.o, a.scale,
-            a.l2norm ? 1 : 0);
+            a.l2norm ? 1 : 0, a.scalar_decay ? 1 : 0);
     else
         kda_decode_kernel<float><<<(unsigned)pairs, kThreads, 0, stream>>>(
             static_cast<const float*>(a.q), static_cast<const float*>(a.k),
-            static_cast<const float*>(a.v), a.g, a.beta, a.state, a.o, a.scale, a.l2norm ? 1 : 0);
+            static_cast<const float*>(a.v), a.g, a.beta, a.state, a.o, a.scale, a.l2norm ? 1 : 0,
+            a.scalar_decay ? 1 : 0);
     return cudaGetLastError();
 }
 

@@ -18,6 +18,7 @@ struct PrefillArgs {
     bool bf16;
     float scale;
     bool l2norm;
+    bool scalar_decay;   // g holds one log-decay per (token, head): [tokens, H]
     const float* initial_state;
     float* final_state;
     float* o;
@@ -43,6 +44,7 @@ struct DecodeArgs {
     bool bf16;
     float scale;
     bool l2norm;
+    bool scalar_decay;   // g is [N, H]
 };
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);

@@ -30,7 +30,7 @@ __global__ void __launch_bounds__(kThreads)
 kda_recurrent_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                      const float* __restrict__ g, const float* __restrict__ beta,
                      const int32_t* __restrict__ cu_seqlens, int64_t total_T, int H, float scale,
-                     int l2norm, const float* s0, float* sT,
+                     int l2norm, int scalar_g, const float* s0, float* sT,
                      float* __restrict__ o, uint32_t* err) {
     __shared__ float Ks[kTB][kD];
     __shared__ float Qs[kTB][kD];
@@ -68,7 +68,12 @@ kda_recurrent_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
                 const size_t off = ((size_t)(t0 + tt) * H + h) * kD + c4;
                 load4(q + off, qv);
                 load4(k + off, kv);
-                load4(g + off, gv);
+                if (scalar_g) {
+                    const float gs = g[(size_t)(t0 + tt) * H + h];
+                    gv[0] = gv[1] = gv[2] = gv[3] = gs;
+                } else {
+                    load4(g + off, gv);
+                }
             }
 #pragma unroll
             for (int x = 0; x < 4; ++x) {
@@ -144,12 +149,12 @@ cudaError_t launch_recurrent(const PrefillArgs& a, cudaStream_t stream) {
         kda_recurrent_kernel<__nv_bfloat16><<<grid, kThreads, 0, stream>>>(
             static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
             static_cast<const __nv_bfloat16*>(a.v), a.g, a.beta, a.cu_seqlens, a.total_T, a.H,
-            a.scale, a.l2norm ? 1 : 0, a.initial_state, a.final_state, a.o, a.err);
+            a.scale, a.l2norm ? 1 : 0, a.scalar_decay ? 1 : 0, a.initial_state, a.final_state, a.o, a.err);
     else
         kda_recurrent_kernel<float><<<grid, kThreads, 0, stream>>>(
             static_cast<const float*>(a.q), static_cast<const float*>(a.k),
             static_cast<const float*>(a.v), a.g, a.beta, a.cu_seqlens, a.total_T, a.H, a.scale,
-            a.l2norm ? 1 : 0, a.initial_state, a.final_state, a.o, a.err);
+            a.l2norm ? 1 : 0, a.scalar_decay ? 1 : 0, a.initial_state, a.final_state, a.o, a.err);
     return cudaGetLastError();
 }
 

@@ -29,6 +29,7 @@ KDA_DTYPE_BF16 = 0
 KDA_DTYPE_FP32 = 1
 KDA_FLAG_L2NORM_QK = 1
 KDA_FLAG_RECURRENT = 2
+KDA_FLAG_SCALAR_DECAY = 4
 KDA_DEVERR_CU_SEQLENS = 1
 KDA_DEVERR_TIMEOUT = 2
 
@@ -116,11 +117,13 @@ def kda_chunk_fwd_workspace_size(N: int, total_T: int, H: int, d: int = 128,
 def kda_chunk_fwd(q, k, v, g, beta, cu_seqlens, *, scale: float = 1.0, l2norm: bool = True,
                   initial_state: Optional[torch.Tensor] = None, final_state=True,
                   o: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-                  recurrent: bool = False, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+                  recurrent: bool = False, scalar_decay: bool = False,
+                  stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Prefill over packed sequences.
 
     q, k, v: [total_T, H, 128] bf16 or fp32 (same dtype); g: [total_T, H, 128]
-    fp32 log-decay; beta: [total_T, H] fp32; cu_seqlens: [N + 1] int32 on the
+    fp32 log-decay ([total_T, H] with ``scalar_decay``, the Gated-DeltaNet
+    form); beta: [total_T, H] fp32; cu_seqlens: [N + 1] int32 on the
     device.  ``final_state`` may be True (allocate), False/None (skip) or a
     [N, H, 128, 128] fp32 tensor (may be ``initial_state`` for an in-place
     continuation).  Returns ``(o, final_state)`` with o fp32 [total_T, H, 128].
@@ -133,7 +136,7 @@ def kda_chunk_fwd(q, k, v, g, beta, cu_seqlens, *, scale: float = 1.0, l2norm: b
     dt = _dtype_code(q)
     for name, t in (("q", q), ("k", k), ("v", v)):
         _check(t, name, (T, H, d), q.dtype, dev)
-    _check(g, "g", (T, H, d), torch.float32, dev)
+    _check(g, "g", (T, H) if scalar_decay else (T, H, d), torch.float32, dev)
     _check(beta, "beta", (T, H), torch.float32, dev)
     if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or cu_seqlens.device != dev:
         raise ValueError("cu_seqlens must be a 1-D int32 tensor on the same device")
@@ -152,7 +155,8 @@ def kda_chunk_fwd(q, k, v, g, beta, cu_seqlens, *, scale: float = 1.0, l2norm: b
     ws_bytes = int(lib.kda_chunk_fwd_workspace_size(N, T, H, d, dt))
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
-    flags = (KDA_FLAG_L2NORM_QK if l2norm else 0) | (KDA_FLAG_RECURRENT if recurrent else 0)
+    flags = ((KDA_FLAG_L2NORM_QK if l2norm else 0) | (KDA_FLAG_RECURRENT if recurrent else 0) |
+             (KDA_FLAG_SCALAR_DECAY if scalar_decay else 0))
     st = lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), N, T, H,
                            d, dt, float(scale), flags, _ptr(initial_state), _ptr(final_state), _ptr(o),
                            _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
@@ -162,9 +166,11 @@ def kda_chunk_fwd(q, k, v, g, beta, cu_seqlens, *, scale: float = 1.0, l2norm: b
 
 
 def kda_decode_step(q, k, v, g, beta, state, *, scale: float = 1.0, l2norm: bool = True,
-                    o: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+                    o: Optional[torch.Tensor] = None, scalar_decay: bool = False,
+                    stream=None) -> torch.Tensor:
     """One decode token per sequence; ``state`` [N, H, 128, 128] fp32 is
-    updated in place.  Returns o [N, H, 128] fp32."""
+    updated in place.  g is [N, H, 128] ([N, H] with ``scalar_decay``).
+    Returns o [N, H, 128] fp32."""
     lib = load_library()
     dev = q.device
     if dev.type != "cuda":
@@ -173,13 +179,13 @@ def kda_decode_step(q, k, v, g, beta, state, *, scale: float = 1.0, l2norm: bool
     dt = _dtype_code(q)
     for name, t in (("q", q), ("k", k), ("v", v)):
         _check(t, name, (N, H, d), q.dtype, dev)
-    _check(g, "g", (N, H, d), torch.float32, dev)
+    _check(g, "g", (N, H) if scalar_decay else (N, H, d), torch.float32, dev)
     _check(beta, "beta", (N, H), torch.float32, dev)
     _check(state, "state", (N, H, d, d), torch.float32, dev)
     if o is None:
         o = torch.empty((N, H, d), dtype=torch.float32, device=dev)
     _check(o, "o", (N, H, d), torch.float32, dev)
-    flags = KDA_FLAG_L2NORM_QK if l2norm else 0
+    flags = (KDA_FLAG_L2NORM_QK if l2norm else 0) | (KDA_FLAG_SCALAR_DECAY if scalar_decay else 0)
     st = lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state), _ptr(o), N,
                              H, d, dt, float(scale), flags, _stream(stream))
     if st != KDA_OK:

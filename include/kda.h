@@ -68,7 +68,13 @@ enum {
     KDA_FLAG_L2NORM_QK = 1u,
     /* Force the token-by-token fp32 kernel for prefill (default for FP32
      * inputs; for BF16 inputs the chunked tensor-core kernel is the default). */
-    KDA_FLAG_RECURRENT = 2u
+    KDA_FLAG_RECURRENT = 2u,
+    /* Gated-DeltaNet form: one decay per (token, head) shared by all d
+     * channels, Diag(alpha_t) = alpha_t I.  g is then [tokens, H] instead of
+     * [tokens, H, d] (decode: [N, H]).  The page names this scalar-gated
+     * delta rule (GDN) as the baseline KDA refines; it is KDA with equal
+     * per-channel decays, and every kernel accepts it. */
+    KDA_FLAG_SCALAR_DECAY = 4u
 };
 
 /* Device-side error bits, OR-ed into the first 32-bit word of the workspace by
@@ -94,6 +100,7 @@ KDA_API size_t kda_chunk_fwd_workspace_size(int32_t N, int64_t total_T, int32_t 
  *
  *   q, k, v       [total_T, H, d]  dtype dt
  *   g             [total_T, H, d]  fp32, log(alpha), finite, <= 0
+ *                 ([total_T, H] with KDA_FLAG_SCALAR_DECAY)
  *   beta          [total_T, H]     fp32
  *   cu_seqlens    [N + 1] int32 DEVICE array: cu[0] = 0, non-decreasing,
  *                 cu[N] = total_T; sequence n is tokens cu[n] .. cu[n+1]-1.
@@ -123,7 +130,8 @@ KDA_API int kda_chunk_fwd(const void *q, const void *k, const void *v, const flo
  * exactly one token, in place, and o receives that token's output
  * (o = scale * S_new^T q).  Same rule as above with T = 1.
  *
- *   q, k, v  [N, H, d] dtype dt      g [N, H, d] fp32      beta [N, H] fp32
+ *   q, k, v  [N, H, d] dtype dt      g [N, H, d] fp32 ([N, H] with
+ *            KDA_FLAG_SCALAR_DECAY)    beta [N, H] fp32
  *   state    [N, H, d, d] fp32, read and overwritten
  *   o        [N, H, d] fp32
  */

@@ -65,6 +65,8 @@ def test_chunk_fwd_host_validation(lib):
     assert _chunk(lib, d=64) == kda.KDA_ERR_UNSUPPORTED
     assert _chunk(lib, dt=7) == kda.KDA_ERR_UNSUPPORTED
     assert _chunk(lib, flags=0x80) == kda.KDA_ERR_UNSUPPORTED
+    # every documented flag passes validation (then fails later only for lack of a GPU)
+    assert _chunk(lib, flags=1 | 2 | 4) == _chunk(lib, flags=1)
     assert _chunk(lib, N=-1) == kda.KDA_ERR_INVALID_ARG
     assert _chunk(lib, H=0) == kda.KDA_ERR_INVALID_ARG
     assert _chunk(lib, T=1 << 31) == kda.KDA_ERR_INVALID_ARG

@@ -234,3 +234,57 @@ def test_decode_workload_full_layer_two_steps():
         o_ref, ref_state = oracle.kda_decode(tok.q, tok.k, tok.v, tok.g, tok.beta, ref_state)
         assert_close(o, o_ref, TOL_BF16, f"o step {step}")
         assert_close(sd, ref_state, TOL_BF16, f"state step {step}")
+
+
+# ---------------------------------------------------------------- scalar decay
+# Gated-DeltaNet form: one decay per (token, head).  The oracle is the same
+# per-channel rule with g broadcast over the channels.
+
+def _scalar_decay_case(seed, lengths, heads=3):
+    x = kin.make_custom_prefill(seed, lengths, heads=heads, init_state_std=0.02)
+    gs = x.g[..., 0].contiguous()                      # [T, H]
+    return x, gs, gs[..., None].expand_as(x.g).contiguous()
+
+
+@pytest.mark.parametrize("recurrent", [False, True])
+def test_scalar_decay_prefill(recurrent):
+    x, gs, gfull = _scalar_decay_case(41, [0, 70, 257, 64, 1])
+    dev = torch.device("cuda")
+    xd = x.to(dev)
+    o, s = kda.kda_chunk_fwd(xd.q, xd.k, xd.v, gs.to(dev), xd.beta, xd.cu_seqlens,
+                             initial_state=xd.initial_state, recurrent=recurrent, scalar_decay=True)
+    torch.cuda.synchronize()
+    o_ref, s_ref = oracle.kda_forward(x.q, x.k, x.v, gfull, x.beta, x.cu_seqlens, x.initial_state)
+    tol = TOL_FP32 if recurrent else TOL_BF16
+    assert_close(o, o_ref, tol, "o")
+    assert_close(s, s_ref, tol, "final state")
+
+
+def test_scalar_decay_prefill_8k_shape():
+    x = kin.make_prefill(kin.PREFILL_8K)
+    gs = x.g[..., 0].contiguous()
+    dev = torch.device("cuda")
+    xd = x.to(dev)
+    o, s = kda.kda_chunk_fwd(xd.q, xd.k, xd.v, gs.to(dev), xd.beta, xd.cu_seqlens, scalar_decay=True)
+    torch.cuda.synchronize()
+    heads = [0, 17]
+    gfull = gs[:, heads, None].expand(-1, -1, 128).contiguous()
+    o_ref, s_ref = oracle.kda_forward(x.q[:, heads].contiguous(), x.k[:, heads].contiguous(),
+                                      x.v[:, heads].contiguous(), gfull, x.beta[:, heads].contiguous(),
+                                      x.cu_seqlens)
+    assert_close(o[:, heads], o_ref, TOL_BF16, "o")
+    assert_close(s[:, heads], s_ref, TOL_BF16, "final state")
+
+
+def test_scalar_decay_decode():
+    spec = kin.DecodeSpec("scalar", 78, 6, 1, 4, torch.bfloat16)
+    tok = kin.make_decode_tokens(spec, 0)
+    st = kin.make_decode_state(spec, 0)
+    gs = tok.g[..., 0].contiguous()
+    dev = torch.device("cuda")
+    td, sd = tok.to(dev), st.to(dev)
+    o = kda.kda_decode_step(td.q, td.k, td.v, gs.to(dev), td.beta, sd, scalar_decay=True)
+    torch.cuda.synchronize()
+    o_ref, s_ref = oracle.kda_decode(tok.q, tok.k, tok.v, gs[..., None].expand_as(tok.g), tok.beta, st)
+    assert_close(o, o_ref, TOL_FP32, "o")
+    assert_close(sd, s_ref, TOL_FP32, "state")
