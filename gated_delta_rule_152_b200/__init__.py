@@ -8,9 +8,12 @@ seeded synthetic workloads.
 from .kda import (  # noqa: F401
     KdaError,
     kda_chunk_fwd,
+    kda_chunk_fwd_slots,
     kda_chunk_fwd_workspace_size,
     kda_decode_step,
+    kda_decode_step_slots,
     kda_status_string,
+    kda_verify_fwd,
     kda_workspace_error,
     load_library,
 )

@@ -35,11 +35,17 @@ size_t kda_chunk_fwd_workspace_size(int32_t N, int64_t total_T, int32_t H, int32
     return kWorkspaceHeader + 4u * static_cast<size_t>(N);   // error word, then a sequence schedule
 }
 
-int kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
-                  const int32_t* cu_seqlens, int32_t N, int64_t total_T, int32_t H, int32_t d,
-                  kda_dtype dt, float scale, uint32_t flags, const float* initial_state,
-                  float* final_state, float* o, void* workspace, size_t workspace_bytes,
-                  kda_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Shared body of kda_chunk_fwd and kda_chunk_fwd_slots.
+int chunk_fwd_impl(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                   const int32_t* cu_seqlens, int32_t N, int64_t total_T, int32_t H, int32_t d,
+                   kda_dtype dt, float scale, uint32_t flags, const float* initial_state,
+                   float* final_state, float* o, void* workspace, size_t workspace_bytes,
+                   kda_stream_t stream, const int32_t* slots, int32_t num_slots,
+                   float* snapshots = nullptr) {
     if (N < 0 || H <= 0 || total_T < 0 || total_T >= (int64_t(1) << 31)) return KDA_ERR_INVALID_ARG;
     if (d != 128) return KDA_ERR_UNSUPPORTED;
     if (dt != KDA_DTYPE_BF16 && dt != KDA_DTYPE_FP32) return KDA_ERR_UNSUPPORTED;
@@ -47,7 +53,7 @@ int kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g, c
         return KDA_ERR_UNSUPPORTED;
     if (cu_seqlens == nullptr) return KDA_ERR_INVALID_ARG;
     if (total_T > 0 && (!q || !k || !v || !g || !beta || !o)) return KDA_ERR_INVALID_ARG;
-    const void* ptrs[] = {q, k, v, g, beta, initial_state, final_state, o, workspace};
+    const void* ptrs[] = {q, k, v, g, beta, initial_state, final_state, o, workspace, snapshots};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
     if (workspace == nullptr || workspace_bytes < kda_chunk_fwd_workspace_size(N, total_T, H, d, dt))
@@ -62,15 +68,16 @@ int kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g, c
 
     kda::PrefillArgs a{q, k, v, g, beta, cu_seqlens, N, total_T, H, dt == KDA_DTYPE_BF16, scale,
                        (flags & KDA_FLAG_L2NORM_QK) != 0, (flags & KDA_FLAG_SCALAR_DECAY) != 0,
-                       initial_state, final_state, o, err};
-    const bool recurrent = (dt == KDA_DTYPE_FP32) || (flags & KDA_FLAG_RECURRENT) || total_T == 0;
+                       initial_state, final_state, o, err, slots, num_slots, snapshots};
+    const bool recurrent = (dt == KDA_DTYPE_FP32) || (flags & KDA_FLAG_RECURRENT) || total_T == 0 ||
+                           snapshots != nullptr;
     const cudaError_t e = recurrent ? kda::launch_recurrent(a, s) : kda::launch_chunk(a, s);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
-int kda_decode_step(const void* q, const void* k, const void* v, const float* g, const float* beta,
-                    float* state, float* o, int32_t N, int32_t H, int32_t d, kda_dtype dt,
-                    float scale, uint32_t flags, kda_stream_t stream) {
+int decode_impl(const void* q, const void* k, const void* v, const float* g, const float* beta, float* state,
+                float* o, int32_t N, int32_t H, int32_t d, kda_dtype dt, float scale, uint32_t flags,
+                kda_stream_t stream, const int32_t* slots, int32_t num_slots) {
     if (N < 0 || H <= 0 || static_cast<int64_t>(N) * H >= (int64_t(1) << 31)) return KDA_ERR_INVALID_ARG;
     if (d != 128) return KDA_ERR_UNSUPPORTED;
     if (dt != KDA_DTYPE_BF16 && dt != KDA_DTYPE_FP32) return KDA_ERR_UNSUPPORTED;
@@ -83,9 +90,59 @@ int kda_decode_step(const void* q, const void* k, const void* v, const float* g,
     int status = KDA_OK;
     if (!device_is_sm100(&status)) return status;
     kda::DecodeArgs a{q, k, v, g, beta, state, o, N, H, dt == KDA_DTYPE_BF16, scale,
-                      (flags & KDA_FLAG_L2NORM_QK) != 0, (flags & KDA_FLAG_SCALAR_DECAY) != 0};
+                      (flags & KDA_FLAG_L2NORM_QK) != 0, (flags & KDA_FLAG_SCALAR_DECAY) != 0, slots,
+                      num_slots};
     return kda::launch_decode(a, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? KDA_OK
                                                                                          : KDA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int kda_chunk_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                  const int32_t* cu_seqlens, int32_t N, int64_t total_T, int32_t H, int32_t d,
+                  kda_dtype dt, float scale, uint32_t flags, const float* initial_state,
+                  float* final_state, float* o, void* workspace, size_t workspace_bytes,
+                  kda_stream_t stream) {
+    return chunk_fwd_impl(q, k, v, g, beta, cu_seqlens, N, total_T, H, d, dt, scale, flags, initial_state,
+                          final_state, o, workspace, workspace_bytes, stream, nullptr, 0);
+}
+
+int kda_chunk_fwd_slots(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                        const int32_t* cu_seqlens, int32_t N, int64_t total_T, int32_t H, int32_t d,
+                        kda_dtype dt, float scale, uint32_t flags, float* state_pool, const int32_t* slots,
+                        int32_t num_slots, float* o, void* workspace, size_t workspace_bytes,
+                        kda_stream_t stream) {
+    if (!state_pool || !slots || num_slots <= 0) return KDA_ERR_INVALID_ARG;
+    if (!aligned16(state_pool)) return KDA_ERR_MISALIGNED;
+    return chunk_fwd_impl(q, k, v, g, beta, cu_seqlens, N, total_T, H, d, dt, scale, flags, state_pool,
+                          state_pool, o, workspace, workspace_bytes, stream, slots, num_slots);
+}
+
+int kda_verify_fwd(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                   const int32_t* cu_seqlens, int32_t N, int64_t total_T, int32_t H, int32_t d,
+                   kda_dtype dt, float scale, uint32_t flags, const float* initial_state,
+                   float* state_snapshots, float* o, void* workspace, size_t workspace_bytes,
+                   kda_stream_t stream) {
+    if (total_T > 0 && state_snapshots == nullptr) return KDA_ERR_INVALID_ARG;
+    return chunk_fwd_impl(q, k, v, g, beta, cu_seqlens, N, total_T, H, d, dt, scale, flags, initial_state,
+                          nullptr, o, workspace, workspace_bytes, stream, nullptr, 0,
+                          total_T > 0 ? state_snapshots : nullptr);
+}
+
+int kda_decode_step(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                    float* state, float* o, int32_t N, int32_t H, int32_t d, kda_dtype dt,
+                    float scale, uint32_t flags, kda_stream_t stream) {
+    return decode_impl(q, k, v, g, beta, state, o, N, H, d, dt, scale, flags, stream, nullptr, 0);
+}
+
+int kda_decode_step_slots(const void* q, const void* k, const void* v, const float* g, const float* beta,
+                          float* state_pool, const int32_t* slots, int32_t num_slots, float* o, int32_t N,
+                          int32_t H, int32_t d, kda_dtype dt, float scale, uint32_t flags,
+                          kda_stream_t stream) {
+    if (N > 0 && (!slots || num_slots <= 0)) return KDA_ERR_INVALID_ARG;
+    return decode_impl(q, k, v, g, beta, state_pool, o, N, H, d, dt, scale, flags, stream, slots, num_slots);
 }
 
 int kda_workspace_error(const void* workspace, uint32_t* out, kda_stream_t stream) {

@@ -132,7 +132,8 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                  const __nv_bfloat16* __restrict__ v, const float* __restrict__ g,
                  const float* __restrict__ beta, const int32_t* __restrict__ cu_seqlens,
                  int64_t total_T, int H, float scale, int l2norm, int scalar_g, const float* s0,
-                 float* sT, float* __restrict__ o, uint32_t* err) {
+                 float* sT, float* __restrict__ o, uint32_t* err, const int32_t* __restrict__ slots,
+                 int num_slots) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(smem);
@@ -157,6 +158,12 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
     const int64_t len = eos - bos;
     const int nchunks = static_cast<int>((len + kC - 1) / kC);
+    // state index of this sequence: n, or its slot in a state pool
+    const int64_t sidx = slots ? static_cast<int64_t>(slots[n]) : static_cast<int64_t>(n);
+    if (slots && (sidx < 0 || sidx >= num_slots)) {
+        if (tid == 0 && slice == 0 && h == 0) set_error(err, 4u);
+        return;   // slot out of range: this sequence is skipped
+    }
 
     if (warp == 0) {
         tmem_alloc(tmem_slot, TM_COLS);
@@ -173,7 +180,7 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const size_t state_off = ((size_t)n * H + h) * kD * kD;
+    const size_t state_off = ((size_t)sidx * H + h) * kD * kD;
 
     // initial state slice -> TMEM (key row = lane, 32 value columns)
     if (warp < 4) {
@@ -231,11 +238,7 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     // Prep of one chunk (state independent): Gamma, L2 norms, the tf32 tiles
     // Kt, Qt (XQ), Kb (rows 0-63 of KS) and V^T, plus beta and exp(Gamma_C).
     // Contains one block barrier; every thread must call it.
-    // `hook(i)` (i = 0..3) runs on thread 0 at four points spread over the
-    // prep, so MMAs can be fed to the tensor core a few at a time while the
-    // rest of the block works (issuing many at once stalls the issuing thread).
-    auto prep = [&](int L, auto&& hook) {
-        if (tid == 0) hook(0);
+    auto prep = [&](int L) {
         // raw q, k of the thread's 8 rows x 4 channels into registers first:
         // the tiles written below overwrite the raw staging area
         uint2 qraw[8], kraw[8];
@@ -261,7 +264,6 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
             *reinterpret_cast<float2*>(xch + warp * 128 + 4 * lane + 2 * x) = run;
         }
-        if (tid == 0) hook(1);
         __syncthreads();   // also: every thread holds its raw q, k in registers
         float2 off[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         float2 GC[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
@@ -302,7 +304,6 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             nrm[m] = sq.x + sq.y;
             nrm[8 + m] = sk.x + sk.y;
         }
-        if (tid == 0) hook(2);
         if (l2norm) warp_allreduce16(nrm);
         const int kbi = lane >> 3, ch = lane & 7;
 #pragma unroll
@@ -331,7 +332,6 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             st_tf32x4(smem, OFF_XQ + kbi * KB_XQ + sw128_off(64 + r, ch), qt.x, qt.y, qt.z, qt.w);
             st_tf32x4(smem, OFF_KS + kbi * KB_KS + sw128_off(r, ch), kb.x, kb.y, kb.z, kb.w);
         }
-        if (tid == 0) hook(3);
         {   // V^T: token tid/4, value columns 8*(tid%4) .. +7 (exact bf16 -> fp32)
             const int r = tid >> 2, j0 = 8 * (tid & 3);
             const uint32_t w4[4] = {vreg.x, vreg.y, vreg.z, vreg.w};
@@ -363,7 +363,7 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         ok = !__syncthreads_or(!mbar_wait_bounded(bar_load, 0));
         if (ok) {
             load_pending = false;
-            prep(static_cast<int>(len < kC ? len : (int64_t)kC), [](int) {});
+            prep(static_cast<int>(len < kC ? len : (int64_t)kC));
         }
     }
 
@@ -375,7 +375,20 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tc_fence_before();
         __syncthreads();   // prep(c) done; the previous chunk's TMEM reads done
 
-        // ============== the state decayed to the chunk end
+        // ============== Kb^T, and the state decayed to the chunk end
+        {   // Kb^T from Kb: thread = channel c, 4 consecutive tokens per 16-byte store
+            const int cch = tid & 127, tg = tid >> 7;
+#pragma unroll
+            for (int b = 0; b < 8; ++b) {
+                const int i0 = 32 * tg + 4 * b;
+                float4 x;
+                x.x = *K_at(smem, OFF_KS, KB_KS, i0 + 0, cch);
+                x.y = *K_at(smem, OFF_KS, KB_KS, i0 + 1, cch);
+                x.z = *K_at(smem, OFF_KS, KB_KS, i0 + 2, cch);
+                x.w = *K_at(smem, OFF_KS, KB_KS, i0 + 3, cch);
+                *reinterpret_cast<float4*>(K_at(smem, OFF_KBT, KB_KBT, cch, i0)) = x;
+            }
+        }
         {   // St = Diag(exp(Gamma_C)) S in TMEM (fp32) and as St^T (tf32, rows 64-95 of KS);
             // the two warps of a TMEM lane quarter take 16 value columns each
             float acc[16];
@@ -407,22 +420,8 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         mma_pending = true;
         if (has_next) prefetch(t0 + kC, Ln);
-        if (warp >= 4) {   // Kb^T from Kb while the tensor core runs: thread = channel
-            const int cch = tid - 128;
-#pragma unroll 4
-            for (int b = 0; b < 16; ++b) {
-                const int i0 = 4 * b;
-                float4 x;
-                x.x = *K_at(smem, OFF_KS, KB_KS, i0 + 0, cch);
-                x.y = *K_at(smem, OFF_KS, KB_KS, i0 + 1, cch);
-                x.z = *K_at(smem, OFF_KS, KB_KS, i0 + 2, cch);
-                x.w = *K_at(smem, OFF_KS, KB_KS, i0 + 3, cch);
-                *reinterpret_cast<float4*>(K_at(smem, OFF_KBT, KB_KBT, cch, i0)) = x;
-            }
-        }
         if (!(ok = wait_mma())) break;
-        // XQ and KS are free now (the block barrier inside wait_mma also
-        // orders the Kb^T copy before it): stage the next chunk's q, k
+        // XQ and KS are free now: stage the next chunk's q, k
         if (tid == 0 && has_next) issue_load(t0 + kC);
         load_pending = has_next;
         load_parity = (c + 1) & 1;
@@ -599,27 +598,25 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tc_fence_before();
         __syncthreads();
 
-        // ============== O = Z + P delta,  S_next = St + Kb^T delta, issued by
-        // thread 0 in four batches of two K steps while the block preps the
-        // next chunk (which touches neither TP, Kb^T, delta^T nor tensor memory)
-        auto os_batch = [&](int i) {
-            if (i == 0) tc_fence_after();
+        // ============== O = Z + P delta,  S_next = St + Kb^T delta
+        if (tid == 0) {
+            tc_fence_after();
             const uint64_t dtp = tdesc(sb, OFF_TP), dkbt = tdesc(sb, OFF_KBT), dyt = tdesc(sb, OFF_YT);
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int s = 2 * i + u;
+            for (int s = 0; s < 8; ++s) {
                 mma_tf32_ss(tmem + TM_X, kstep(dtp, KB_TP, s), kstep(dyt, KB_VT, s), ID_N32, 1);
                 mma_tf32_ss(tmem + TM_S, kstep(dkbt, KB_KBT, s), kstep(dyt, KB_VT, s), ID_N32, 1);
             }
-            if (i == 3) mma_commit(bar_mma);
-        };
+            mma_commit(bar_mma);
+        }
         mma_pending = true;
+
+        // ============== while those run: prep of the next chunk (touches neither
+        // TP, Kb^T, delta^T nor tensor memory)
         if (has_next) {
             if (!(ok = !__syncthreads_or(!mbar_wait_bounded(bar_load, (c + 1) & 1)))) break;
             load_pending = false;
-            prep(Ln, os_batch);
-        } else if (tid == 0) {
-            for (int i = 0; i < 4; ++i) os_batch(i);
+            prep(Ln);
         }
         if (!(ok = wait_mma())) break;
 
@@ -717,7 +714,8 @@ cudaError_t launch_chunk(const PrefillArgs& a, cudaStream_t stream) {
     const long long blocks = (long long)a.N * a.H * kSplit;
     kda_chunk_kernel<<<static_cast<unsigned>(blocks), kThreads, SMEM_BYTES, stream>>>(
         mq, mk, static_cast<const __nv_bfloat16*>(a.v), a.g, a.beta, a.cu_seqlens, a.total_T, a.H, a.scale,
-        a.l2norm ? 1 : 0, a.scalar_decay ? 1 : 0, a.initial_state, a.final_state, a.o, a.err);
+        a.l2norm ? 1 : 0, a.scalar_decay ? 1 : 0, a.initial_state, a.final_state, a.o, a.err, a.slots,
+        a.num_slots);
     return cudaGetLastError();
 }
 

@@ -28,14 +28,22 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads, 2)
 kda_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                   const float* __restrict__ g, const float* __restrict__ beta,
-                  float* __restrict__ state, float* __restrict__ o, float scale, int l2norm, int scalar_g) {
+                  float* __restrict__ state, float* __restrict__ o, float scale, int l2norm, int scalar_g,
+                  int H, const int32_t* __restrict__ slots, int num_slots) {
     __shared__ float ak[kD], aq[kD], al[kD], kh[kD];
     __shared__ float4 red[8][2][32];
     __shared__ float qk_dot;
 
     const int p = blockIdx.x;          // (sequence, head) pair, row-major [N, H]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    float4* S = reinterpret_cast<float4*>(state + (size_t)p * kD * kD);
+    // the state of sequence n sits at index n, or at slots[n] of a state pool
+    size_t sp = static_cast<size_t>(p);
+    if (slots) {
+        const int n = p / H, h = p - n * H, slot = slots[n];
+        if (slot < 0 || slot >= num_slots) return;   // out-of-range slot: sequence skipped
+        sp = static_cast<size_t>(slot) * H + h;
+    }
+    float4* S = reinterpret_cast<float4*>(state + sp * kD * kD);
 
     // 1. put the whole 64 KiB state slab in flight first (streaming loads)
     float4 s[kRows];
@@ -133,12 +141,12 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
         kda_decode_kernel<__nv_bfloat16><<<(unsigned)pairs, kThreads, 0, stream>>>(
             static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
             static_cast<const __nv_bfloat16*>(a.v), a.g, a.beta, a.state, a.o, a.scale,
-            a.l2norm ? 1 : 0, a.scalar_decay ? 1 : 0);
+            a.l2norm ? 1 : 0, a.scalar_decay ? 1 : 0, a.H, a.slots, a.num_slots);
     else
         kda_decode_kernel<float><<<(unsigned)pairs, kThreads, 0, stream>>>(
             static_cast<const float*>(a.q), static_cast<const float*>(a.k),
             static_cast<const float*>(a.v), a.g, a.beta, a.state, a.o, a.scale, a.l2norm ? 1 : 0,
-            a.scalar_decay ? 1 : 0);
+            a.scalar_decay ? 1 : 0, a.H, a.slots, a.num_slots);
     return cudaGetLastError();
 }
 

@@ -23,6 +23,9 @@ struct PrefillArgs {
     float* final_state;
     float* o;
     uint32_t* err;   // device error word
+    const int32_t* slots = nullptr;   // optional: sequence n's state lives at index slots[n]
+    int32_t num_slots = 0;            // of the state arrays (valid slots: 0 .. num_slots-1)
+    float* snapshots = nullptr;       // optional [total_T, H, d, d]: the state after every token
 };
 
 // Token-by-token fp32 recurrence (CUDA cores), any dtype.
@@ -45,6 +48,8 @@ struct DecodeArgs {
     float scale;
     bool l2norm;
     bool scalar_decay;   // g is [N, H]
+    const int32_t* slots = nullptr;   // optional: sequence n's state is state[slots[n]]
+    int32_t num_slots = 0;
 };
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);

@@ -7,7 +7,9 @@
 // one token after the other, in the expanded form
 //     S' = Diag(alpha) S,  u = S'^T k,  S = S' + beta k (v - u)^T,  o = S^T q.
 // It is exact fp32 arithmetic (no tensor cores), so it serves fp32 inputs at
-// the tight tolerance and any input when KDA_FLAG_RECURRENT is set.
+// the tight tolerance and any input when KDA_FLAG_RECURRENT is set.  It also
+// serves multi-token verification: with a snapshot array it stores the state
+// after every token, so a caller can roll back to any accepted prefix.
 //
 // Grid: one block per (sequence, head, 32-column value slice), flattened.
 // Block: 128 threads = 4 warps.
@@ -31,7 +33,8 @@ kda_recurrent_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
                      const float* __restrict__ g, const float* __restrict__ beta,
                      const int32_t* __restrict__ cu_seqlens, int64_t total_T, int H, float scale,
                      int l2norm, int scalar_g, const float* s0, float* sT,
-                     float* __restrict__ o, uint32_t* err) {
+                     float* __restrict__ o, uint32_t* err, const int32_t* __restrict__ slots,
+                     int num_slots, float* __restrict__ snap) {
     __shared__ float Ks[kTB][kD];
     __shared__ float Qs[kTB][kD];
     __shared__ float As[kTB][kD];
@@ -51,7 +54,12 @@ kda_recurrent_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
         return;   // inconsistent cu_seqlens: sequence skipped
     }
 
-    const size_t state_off = ((size_t)n * H + h) * kD * kD;
+    const int64_t sidx = slots ? static_cast<int64_t>(slots[n]) : static_cast<int64_t>(n);
+    if (slots && (sidx < 0 || sidx >= num_slots)) {
+        if (threadIdx.x == 0 && slice == 0 && h == 0) set_error(err, 4u);
+        return;   // slot out of range: this sequence is skipped
+    }
+    const size_t state_off = ((size_t)sidx * H + h) * kD * kD;
     float s[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i)
@@ -133,6 +141,11 @@ kda_recurrent_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
                                  red_o[buf][3][lane];
                 o[((size_t)(t0 + tt) * H + h) * kD + col] = scale * ov;
             }
+            if (snap) {   // state after this token (one coalesced 128-byte row segment per store)
+                float* dst = snap + ((size_t)(t0 + tt) * H + h) * kD * kD + (size_t)(warp * 32) * kD + col;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) dst[(size_t)i * kD] = s[i];
+            }
         }
     }
     if (sT) {
@@ -149,12 +162,14 @@ cudaError_t launch_recurrent(const PrefillArgs& a, cudaStream_t stream) {
         kda_recurrent_kernel<__nv_bfloat16><<<grid, kThreads, 0, stream>>>(
             static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
             static_cast<const __nv_bfloat16*>(a.v), a.g, a.beta, a.cu_seqlens, a.total_T, a.H,
-            a.scale, a.l2norm ? 1 : 0, a.scalar_decay ? 1 : 0, a.initial_state, a.final_state, a.o, a.err);
+            a.scale, a.l2norm ? 1 : 0, a.scalar_decay ? 1 : 0, a.initial_state, a.final_state, a.o, a.err,
+            a.slots, a.num_slots, a.snapshots);
     else
         kda_recurrent_kernel<float><<<grid, kThreads, 0, stream>>>(
             static_cast<const float*>(a.q), static_cast<const float*>(a.k),
             static_cast<const float*>(a.v), a.g, a.beta, a.cu_seqlens, a.total_T, a.H, a.scale,
-            a.l2norm ? 1 : 0, a.scalar_decay ? 1 : 0, a.initial_state, a.final_state, a.o, a.err);
+            a.l2norm ? 1 : 0, a.scalar_decay ? 1 : 0, a.initial_state, a.final_state, a.o, a.err, a.slots,
+            a.num_slots, a.snapshots);
     return cudaGetLastError();
 }
 

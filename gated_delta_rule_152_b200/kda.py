@@ -32,9 +32,11 @@ KDA_FLAG_RECURRENT = 2
 KDA_FLAG_SCALAR_DECAY = 4
 KDA_DEVERR_CU_SEQLENS = 1
 KDA_DEVERR_TIMEOUT = 2
+KDA_DEVERR_SLOT = 4
 
 EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_decode_step",
-            "kda_workspace_error", "kda_status_string")
+            "kda_chunk_fwd_slots", "kda_decode_step_slots", "kda_verify_fwd", "kda_workspace_error",
+            "kda_status_string")
 
 _lock = threading.Lock()
 _lib = None
@@ -65,6 +67,15 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.kda_chunk_fwd.restype = ctypes.c_int
         lib.kda_decode_step.argtypes = [P, P, P, P, P, P, P, I32, I32, I32, ctypes.c_int, F32, U32, P]
         lib.kda_decode_step.restype = ctypes.c_int
+        lib.kda_chunk_fwd_slots.argtypes = [P, P, P, P, P, P, I32, I64, I32, I32, ctypes.c_int, F32, U32,
+                                            P, P, I32, P, P, SZ, P]
+        lib.kda_chunk_fwd_slots.restype = ctypes.c_int
+        lib.kda_decode_step_slots.argtypes = [P, P, P, P, P, P, P, I32, P, I32, I32, I32, ctypes.c_int, F32,
+                                              U32, P]
+        lib.kda_decode_step_slots.restype = ctypes.c_int
+        lib.kda_verify_fwd.argtypes = [P, P, P, P, P, P, I32, I64, I32, I32, ctypes.c_int, F32, U32,
+                                       P, P, P, P, SZ, P]
+        lib.kda_verify_fwd.restype = ctypes.c_int
         lib.kda_workspace_error.argtypes = [P, ctypes.POINTER(U32), P]
         lib.kda_workspace_error.restype = ctypes.c_int
         lib.kda_status_string.argtypes = [ctypes.c_int]
@@ -191,6 +202,119 @@ def kda_decode_step(q, k, v, g, beta, state, *, scale: float = 1.0, l2norm: bool
     if st != KDA_OK:
         raise KdaError(st, "kda_decode_step")
     return o
+
+
+def kda_chunk_fwd_slots(q, k, v, g, beta, cu_seqlens, state_pool, slots, *, scale: float = 1.0,
+                        l2norm: bool = True, o: Optional[torch.Tensor] = None,
+                        workspace: Optional[torch.Tensor] = None, recurrent: bool = False,
+                        scalar_decay: bool = False, stream=None) -> torch.Tensor:
+    """Prefill whose sequences keep their states in a pool: sequence n starts
+    from ``state_pool[slots[n]]`` ([num_slots, H, 128, 128] fp32) and its final
+    state is written back there.  ``slots``: [N] int32 on the device, distinct.
+    Returns o [total_T, H, 128] fp32."""
+    lib = load_library()
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("kda_chunk_fwd_slots needs CUDA tensors")
+    T, H, d = q.shape
+    dt = _dtype_code(q)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check(t, name, (T, H, d), q.dtype, dev)
+    _check(g, "g", (T, H) if scalar_decay else (T, H, d), torch.float32, dev)
+    _check(beta, "beta", (T, H), torch.float32, dev)
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or cu_seqlens.device != dev:
+        raise ValueError("cu_seqlens must be a 1-D int32 tensor on the same device")
+    N = cu_seqlens.numel() - 1
+    _check(slots, "slots", (N,), torch.int32, dev)
+    if state_pool.dim() != 4 or tuple(state_pool.shape[1:]) != (H, d, d):
+        raise ValueError("state_pool must be [num_slots, H, 128, 128]")
+    _check(state_pool, "state_pool", tuple(state_pool.shape), torch.float32, dev)
+    if o is None:
+        o = torch.empty((T, H, d), dtype=torch.float32, device=dev)
+    _check(o, "o", (T, H, d), torch.float32, dev)
+    ws_bytes = int(lib.kda_chunk_fwd_workspace_size(N, T, H, d, dt))
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    flags = ((KDA_FLAG_L2NORM_QK if l2norm else 0) | (KDA_FLAG_RECURRENT if recurrent else 0) |
+             (KDA_FLAG_SCALAR_DECAY if scalar_decay else 0))
+    st = lib.kda_chunk_fwd_slots(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), N, T, H,
+                                 d, dt, float(scale), flags, _ptr(state_pool), _ptr(slots),
+                                 int(state_pool.shape[0]), _ptr(o), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_chunk_fwd_slots")
+    return o
+
+
+def kda_decode_step_slots(q, k, v, g, beta, state_pool, slots, *, scale: float = 1.0,
+                          l2norm: bool = True, o: Optional[torch.Tensor] = None,
+                          scalar_decay: bool = False, stream=None) -> torch.Tensor:
+    """Decode step whose states live in a pool: sequence n updates
+    ``state_pool[slots[n]]`` in place.  Returns o [N, H, 128] fp32."""
+    lib = load_library()
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("kda_decode_step_slots needs CUDA tensors")
+    N, H, d = q.shape
+    dt = _dtype_code(q)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check(t, name, (N, H, d), q.dtype, dev)
+    _check(g, "g", (N, H) if scalar_decay else (N, H, d), torch.float32, dev)
+    _check(beta, "beta", (N, H), torch.float32, dev)
+    _check(slots, "slots", (N,), torch.int32, dev)
+    if state_pool.dim() != 4 or tuple(state_pool.shape[1:]) != (H, d, d):
+        raise ValueError("state_pool must be [num_slots, H, 128, 128]")
+    _check(state_pool, "state_pool", tuple(state_pool.shape), torch.float32, dev)
+    if o is None:
+        o = torch.empty((N, H, d), dtype=torch.float32, device=dev)
+    _check(o, "o", (N, H, d), torch.float32, dev)
+    flags = (KDA_FLAG_L2NORM_QK if l2norm else 0) | (KDA_FLAG_SCALAR_DECAY if scalar_decay else 0)
+    st = lib.kda_decode_step_slots(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_pool),
+                                   _ptr(slots), int(state_pool.shape[0]), _ptr(o), N, H, d, dt,
+                                   float(scale), flags, _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_decode_step_slots")
+    return o
+
+
+def kda_verify_fwd(q, k, v, g, beta, cu_seqlens, *, initial_state: Optional[torch.Tensor] = None,
+                   snapshots: Optional[torch.Tensor] = None, scale: float = 1.0, l2norm: bool = True,
+                   o: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                   scalar_decay: bool = False, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Multi-token (speculative-verify) step: like kda_chunk_fwd, but returns
+    the state after every token, ``snapshots`` [total_T, H, 128, 128] fp32,
+    for rolling back to an accepted prefix.  Returns ``(o, snapshots)``."""
+    lib = load_library()
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("kda_verify_fwd needs CUDA tensors")
+    T, H, d = q.shape
+    dt = _dtype_code(q)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check(t, name, (T, H, d), q.dtype, dev)
+    _check(g, "g", (T, H) if scalar_decay else (T, H, d), torch.float32, dev)
+    _check(beta, "beta", (T, H), torch.float32, dev)
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or cu_seqlens.device != dev:
+        raise ValueError("cu_seqlens must be a 1-D int32 tensor on the same device")
+    N = cu_seqlens.numel() - 1
+    if initial_state is not None:
+        _check(initial_state, "initial_state", (N, H, d, d), torch.float32, dev)
+    if snapshots is None:
+        snapshots = torch.empty((T, H, d, d), dtype=torch.float32, device=dev)
+    _check(snapshots, "snapshots", (T, H, d, d), torch.float32, dev)
+    if o is None:
+        o = torch.empty((T, H, d), dtype=torch.float32, device=dev)
+    _check(o, "o", (T, H, d), torch.float32, dev)
+    ws_bytes = int(lib.kda_chunk_fwd_workspace_size(N, T, H, d, dt))
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    flags = (KDA_FLAG_L2NORM_QK if l2norm else 0) | (KDA_FLAG_SCALAR_DECAY if scalar_decay else 0)
+    st = lib.kda_verify_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), N, T, H, d,
+                            dt, float(scale), flags, _ptr(initial_state), _ptr(snapshots), _ptr(o),
+                            _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_verify_fwd")
+    return o, snapshots
 
 
 def kda_workspace_error(workspace: torch.Tensor, stream=None) -> int:

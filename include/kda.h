@@ -82,8 +82,10 @@ enum {
 enum {
     KDA_DEVERR_CU_SEQLENS = 1u, /* cu_seqlens not non-decreasing in [0, total_T]; the
                                    offending sequences were treated as empty */
-    KDA_DEVERR_TIMEOUT = 2u     /* a bounded wait inside a kernel gave up; outputs of the
+    KDA_DEVERR_TIMEOUT = 2u,    /* a bounded wait inside a kernel gave up; outputs of the
                                    affected (sequence, head) are undefined */
+    KDA_DEVERR_SLOT = 4u        /* kda_chunk_fwd_slots: a slot index outside [0, num_slots);
+                                   that sequence was skipped */
 };
 
 /*
@@ -165,6 +167,57 @@ KDA_API int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, c
                           int64_t total_T, int32_t H, int32_t d, kda_dtype dt, float scale,
                           uint32_t flags, const float *initial_state, float *final_state,
                           float *o, kda_stream_t stream);
+
+/*
+ * State-pool ("slot") forms for continuous batching: instead of a dense
+ * [N, H, d, d] state array, the states live in a pool
+ *   state_pool [num_slots, H, d, d] fp32
+ * and sequence n uses the entry slots[n] (slots: [N] int32 DEVICE array,
+ * distinct values in [0, num_slots); two sequences sharing a slot race).
+ * The pages have no interface at all; the pool only changes where states are
+ * read and written, not the arithmetic.
+ *
+ * kda_chunk_fwd_slots: as kda_chunk_fwd with initial_state = final_state =
+ * state_pool[slots[n]] (the state is read and updated in place; clear a slot
+ * before starting a new sequence in it).  A slot outside [0, num_slots) sets
+ * KDA_DEVERR_SLOT in the workspace and that sequence is skipped.
+ */
+KDA_API int kda_chunk_fwd_slots(const void *q, const void *k, const void *v, const float *g,
+                        const float *beta, const int32_t *cu_seqlens, int32_t N,
+                        int64_t total_T, int32_t H, int32_t d, kda_dtype dt, float scale,
+                        uint32_t flags, float *state_pool, const int32_t *slots,
+                        int32_t num_slots, float *o, void *workspace, size_t workspace_bytes,
+                        kda_stream_t stream);
+
+/*
+ * kda_decode_step_slots: as kda_decode_step with state = state_pool[slots[n]],
+ * updated in place.  A sequence whose slot is outside [0, num_slots) is
+ * skipped (its state and o rows are left untouched).
+ */
+KDA_API int kda_decode_step_slots(const void *q, const void *k, const void *v, const float *g,
+                          const float *beta, float *state_pool, const int32_t *slots,
+                          int32_t num_slots, float *o, int32_t N, int32_t H, int32_t d,
+                          kda_dtype dt, float scale, uint32_t flags, kda_stream_t stream);
+
+/*
+ * kda_verify_fwd -- multi-token step for speculative decoding: each sequence
+ * advances by its (few) draft tokens and the state after EVERY token is kept,
+ * so the caller can roll back to the longest accepted prefix (the state after
+ * token cu[n] + a - 1, or the initial state when a = 0).  Page "18B Active
+ * for Just $0.045: How GLM-5.3-Flash Beat Claude with Hybrid Attention"
+ * (kongchang.com), section "The Architecture Stack", names one MTP draft layer
+ * for speculative decoding and the text after it describes draft, parallel
+ * verify and rollback; the arithmetic is the same update rule.
+ *
+ * Arguments as kda_chunk_fwd (no final_state), plus
+ *   state_snapshots [total_T, H, d, d] fp32: the state after each token.
+ * Runs the token-by-token fp32 kernel (64 KiB written per token and head).
+ */
+KDA_API int kda_verify_fwd(const void *q, const void *k, const void *v, const float *g,
+                   const float *beta, const int32_t *cu_seqlens, int32_t N, int64_t total_T,
+                   int32_t H, int32_t d, kda_dtype dt, float scale, uint32_t flags,
+                   const float *initial_state, float *state_snapshots, float *o,
+                   void *workspace, size_t workspace_bytes, kda_stream_t stream);
 
 /*
  * Copy the device error word of a workspace used by kda_chunk_fwd to *out

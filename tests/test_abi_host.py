@@ -93,6 +93,18 @@ def test_decode_host_validation(lib):
     assert dec(N=0) == kda.KDA_OK                    # nothing to do, nothing launched
 
 
+def test_slot_forms_reject_missing_pool_or_slots(lib):
+    P = ctypes.c_void_p
+    lib.kda_chunk_fwd_slots.argtypes = [P, P, P, P, P, P, ctypes.c_int32, ctypes.c_int64, ctypes.c_int32,
+                                        ctypes.c_int32, ctypes.c_int, ctypes.c_float, ctypes.c_uint32, P, P,
+                                        ctypes.c_int32, P, P, ctypes.c_size_t, P]
+    args = [A, A, A, A, A, A, 2, 100, 4, 128, 0, 1.0, 1]
+    assert lib.kda_chunk_fwd_slots(*args, None, A, 8, A, A, 4096, None) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_chunk_fwd_slots(*args, A, None, 8, A, A, 4096, None) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_chunk_fwd_slots(*args, A, A, 0, A, A, 4096, None) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_chunk_fwd_slots(*args, MIS, A, 8, A, A, 4096, None) == kda.KDA_ERR_MISALIGNED
+
+
 def test_valid_call_without_gpu_reports_cuda_error(lib):
     import torch
     if torch.cuda.is_available():

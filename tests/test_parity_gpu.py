@@ -288,3 +288,87 @@ def test_scalar_decay_decode():
     o_ref, s_ref = oracle.kda_decode(tok.q, tok.k, tok.v, gs[..., None].expand_as(tok.g), tok.beta, st)
     assert_close(o, o_ref, TOL_FP32, "o")
     assert_close(sd, s_ref, TOL_FP32, "state")
+
+
+# ---------------------------------------------------------------- state pools
+# Continuous batching: states live in a pool and sequence n uses slots[n].
+
+@pytest.mark.parametrize("recurrent", [False, True])
+def test_prefill_with_state_pool(recurrent):
+    dev = torch.device("cuda")
+    lengths, slots = [100, 0, 70], [4, 0, 5]
+    x = kin.make_custom_prefill(51, lengths, heads=2, init_state_std=0.02)
+    pool = torch.randn(6, 2, 128, 128) * 0.02
+    pool[slots] = x.initial_state
+    pool_d = pool.to(dev)
+    xd = x.to(dev)
+    o = kda.kda_chunk_fwd_slots(xd.q, xd.k, xd.v, xd.g, xd.beta, xd.cu_seqlens, pool_d,
+                                torch.tensor(slots, dtype=torch.int32, device=dev), recurrent=recurrent)
+    torch.cuda.synchronize()
+    o_ref, s_ref = oracle.kda_forward(x.q, x.k, x.v, x.g, x.beta, x.cu_seqlens, x.initial_state)
+    tol = TOL_FP32 if recurrent else TOL_BF16
+    assert_close(o, o_ref, tol, "o")
+    assert_close(pool_d[slots], s_ref, tol, "pooled final states")
+    untouched = [i for i in range(6) if i not in slots]
+    assert torch.equal(pool_d[untouched].cpu(), pool[untouched])
+
+
+def test_prefill_state_pool_rejects_bad_slot():
+    dev = torch.device("cuda")
+    x = kin.make_custom_prefill(52, [40, 30], heads=2).to(dev)
+    pool = torch.zeros(3, 2, 128, 128, device=dev)
+    ws = torch.zeros(1024, dtype=torch.uint8, device=dev)
+    kda.kda_chunk_fwd_slots(x.q, x.k, x.v, x.g, x.beta, x.cu_seqlens, pool,
+                            torch.tensor([1, 3], dtype=torch.int32, device=dev), workspace=ws)
+    assert kda.kda_workspace_error(ws) & kda.KDA_DEVERR_SLOT
+    assert torch.count_nonzero(pool[1]) > 0 and torch.count_nonzero(pool[[0, 2]]) == 0
+
+
+def test_decode_with_state_pool():
+    dev = torch.device("cuda")
+    spec = kin.DecodeSpec("pool", 53, 4, 1, 3, torch.bfloat16)
+    tok = kin.make_decode_tokens(spec, 0)
+    pool = torch.randn(10, 3, 128, 128) * 0.02
+    slots = [7, 2, 9, 0]
+    pool_d = pool.to(dev)
+    td = tok.to(dev)
+    o = kda.kda_decode_step_slots(td.q, td.k, td.v, td.g, td.beta, pool_d,
+                                  torch.tensor(slots, dtype=torch.int32, device=dev))
+    torch.cuda.synchronize()
+    o_ref, s_ref = oracle.kda_decode(tok.q, tok.k, tok.v, tok.g, tok.beta, pool[slots])
+    assert_close(o, o_ref, TOL_FP32, "o")
+    assert_close(pool_d[slots], s_ref, TOL_FP32, "pooled states")
+    untouched = [i for i in range(10) if i not in slots]
+    assert torch.equal(pool_d[untouched].cpu(), pool[untouched])
+    # an out-of-range slot skips that sequence and touches nothing
+    o2 = torch.full((4, 3, 128), 5.0, device=dev)
+    before = pool_d.clone()
+    kda.kda_decode_step_slots(td.q, td.k, td.v, td.g, td.beta, pool_d,
+                              torch.tensor([7, -1, 9, 10], dtype=torch.int32, device=dev), o=o2)
+    torch.cuda.synchronize()
+    assert torch.all(o2[1] == 5.0) and torch.all(o2[3] == 5.0)
+    assert torch.equal(pool_d[[2, 0]], before[[2, 0]])
+
+
+# ---------------------------------------------------------------- speculative verify
+# Draft tokens are verified in one call; the state after every token is kept
+# so that a rejected suffix can be rolled back.
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_verify_snapshots_match_prefix_states(dtype):
+    dev = torch.device("cuda")
+    lengths = [4, 1, 6, 0]
+    x = kin.make_custom_prefill(61, lengths, heads=2, dtype=dtype, init_state_std=0.02)
+    xd = x.to(dev)
+    o, snaps = kda.kda_verify_fwd(xd.q, xd.k, xd.v, xd.g, xd.beta, xd.cu_seqlens,
+                                  initial_state=xd.initial_state)
+    torch.cuda.synchronize()
+    o_ref, _ = oracle.kda_forward(x.q, x.k, x.v, x.g, x.beta, x.cu_seqlens, x.initial_state)
+    assert_close(o, o_ref, TOL_FP32, "o")
+    cu = x.cu_seqlens.tolist()
+    for n in range(len(lengths)):
+        for t in range(cu[n], cu[n + 1]):   # state after token t = end state of the prefix up to t
+            sl = slice(cu[n], t + 1)
+            _, s_ref = oracle.kda_forward(x.q[sl], x.k[sl], x.v[sl], x.g[sl], x.beta[sl], [0, t + 1 - cu[n]],
+                                          x.initial_state[n:n + 1])
+            assert_close(snaps[t:t + 1], s_ref[:, :], TOL_FP32, f"snapshot of token {t}")
