@@ -376,18 +376,21 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         __syncthreads();   // prep(c) done; the previous chunk's TMEM reads done
 
         // ============== Kb^T, and the state decayed to the chunk end
-        {   // Kb^T from Kb: thread = channel c, 4 consecutive tokens per 16-byte store
+        {   // Kb^T from Kb: thread = channel c, 4 consecutive tokens per 16-byte
+            // store; all 32 loads are issued before the first store
             const int cch = tid & 127, tg = tid >> 7;
+            float4 x[8];
 #pragma unroll
             for (int b = 0; b < 8; ++b) {
                 const int i0 = 32 * tg + 4 * b;
-                float4 x;
-                x.x = *K_at(smem, OFF_KS, KB_KS, i0 + 0, cch);
-                x.y = *K_at(smem, OFF_KS, KB_KS, i0 + 1, cch);
-                x.z = *K_at(smem, OFF_KS, KB_KS, i0 + 2, cch);
-                x.w = *K_at(smem, OFF_KS, KB_KS, i0 + 3, cch);
-                *reinterpret_cast<float4*>(K_at(smem, OFF_KBT, KB_KBT, cch, i0)) = x;
+                x[b].x = *K_at(smem, OFF_KS, KB_KS, i0 + 0, cch);
+                x[b].y = *K_at(smem, OFF_KS, KB_KS, i0 + 1, cch);
+                x[b].z = *K_at(smem, OFF_KS, KB_KS, i0 + 2, cch);
+                x[b].w = *K_at(smem, OFF_KS, KB_KS, i0 + 3, cch);
             }
+#pragma unroll
+            for (int b = 0; b < 8; ++b)
+                *reinterpret_cast<float4*>(K_at(smem, OFF_KBT, KB_KBT, cch, 32 * tg + 4 * b)) = x[b];
         }
         {   // St = Diag(exp(Gamma_C)) S in TMEM (fp32) and as St^T (tf32, rows 64-95 of KS);
             // the two warps of a TMEM lane quarter take 16 value columns each
@@ -494,11 +497,14 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 tmem_ld32(tm_lane(tmem, quarter, TM_X), y);
                 tmem_wait_ld();
                 const int r = 32 * quarter + lane;
+                // all loads before all stores: the compiler cannot prove the
+                // 32 addresses distinct, so an interleaved read-modify-write
+                // would serialise on shared-memory latency
+                float vv[32];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    float* pv = K_at(smem, OFF_VT, KB_VT, e, r);
-                    *pv = to_tf32(*pv - y[e]);
-                }
+                for (int e = 0; e < 32; ++e) vv[e] = *K_at(smem, OFF_VT, KB_VT, e, r);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) *K_at(smem, OFF_VT, KB_VT, e, r) = to_tf32(vv[e] - y[e]);
             }
             __syncthreads();
             {   // 16 -> 32 on tensor cores: T_ab = -T_aa (M_ab T_bb) for (a, b) = (1, 0), (3, 2);
@@ -557,14 +563,19 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             __syncthreads();
             {   // T' = T diag(beta) on and below the diagonal, zero above; tf32 operand
                 const int r = tid >> 2;
+                float4 t4[4], b4[4];
 #pragma unroll
                 for (int qd = 0; qd < 4; ++qd) {
                     const int i0 = 16 * (tid & 3) + 4 * qd;
-                    const float4 t4 = *reinterpret_cast<const float4*>(Tf + r * kLd + i0);
-                    const float4 b4 = *reinterpret_cast<const float4*>(beta_s + i0);
+                    t4[qd] = *reinterpret_cast<const float4*>(Tf + r * kLd + i0);
+                    b4[qd] = *reinterpret_cast<const float4*>(beta_s + i0);
+                }
+#pragma unroll
+                for (int qd = 0; qd < 4; ++qd) {
+                    const int i0 = 16 * (tid & 3) + 4 * qd;
                     st_tf32x4(smem, OFF_TP + (i0 >> 5) * KB_TP + sw128_off(r, (i0 & 31) >> 2),
-                              (i0 + 0 <= r) ? t4.x * b4.x : 0.f, (i0 + 1 <= r) ? t4.y * b4.y : 0.f,
-                              (i0 + 2 <= r) ? t4.z * b4.z : 0.f, (i0 + 3 <= r) ? t4.w * b4.w : 0.f);
+                              (i0 + 0 <= r) ? t4[qd].x * b4[qd].x : 0.f, (i0 + 1 <= r) ? t4[qd].y * b4[qd].y : 0.f,
+                              (i0 + 2 <= r) ? t4[qd].z * b4[qd].z : 0.f, (i0 + 3 <= r) ? t4[qd].w * b4[qd].w : 0.f);
                 }
             }
         }
