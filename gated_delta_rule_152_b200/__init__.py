@@ -10,6 +10,7 @@ from .kda import (  # noqa: F401
     kda_chunk_fwd,
     kda_chunk_fwd_slots,
     kda_chunk_fwd_workspace_size,
+    kda_chunk_fwd_workspace_size_min,
     kda_decode_step,
     kda_decode_step_slots,
     kda_status_string,

@@ -29,10 +29,17 @@ bool device_is_sm100(int* status) {
 
 extern "C" {
 
-size_t kda_chunk_fwd_workspace_size(int32_t N, int64_t total_T, int32_t H, int32_t d, kda_dtype dt) {
+size_t kda_chunk_fwd_workspace_size_min(int32_t N, int64_t total_T, int32_t H, int32_t d, kda_dtype dt) {
     (void)dt;
     if (N < 0 || total_T < 0 || H <= 0 || d != 128) return 0;
-    return kWorkspaceHeader + 4u * static_cast<size_t>(N);   // error word, then a sequence schedule
+    return kWorkspaceHeader + 4u * static_cast<size_t>(N);   // error word + reserved
+}
+
+size_t kda_chunk_fwd_workspace_size(int32_t N, int64_t total_T, int32_t H, int32_t d, kda_dtype dt) {
+    const size_t lo = kda_chunk_fwd_workspace_size_min(N, total_T, H, d, dt);
+    if (lo == 0) return 0;
+    const size_t two_pass = kWorkspaceHeader + kda::two_pass_scratch_bytes(N, total_T, H);
+    return two_pass > lo ? two_pass : lo;
 }
 
 }  // extern "C"
@@ -56,7 +63,7 @@ int chunk_fwd_impl(const void* q, const void* k, const void* v, const float* g, 
     const void* ptrs[] = {q, k, v, g, beta, initial_state, final_state, o, workspace, snapshots};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
-    if (workspace == nullptr || workspace_bytes < kda_chunk_fwd_workspace_size(N, total_T, H, d, dt))
+    if (workspace == nullptr || workspace_bytes < kda_chunk_fwd_workspace_size_min(N, total_T, H, d, dt))
         return KDA_ERR_WORKSPACE;
     int status = KDA_OK;
     if (!device_is_sm100(&status)) return status;
@@ -71,7 +78,13 @@ int chunk_fwd_impl(const void* q, const void* k, const void* v, const float* g, 
                        initial_state, final_state, o, err, slots, num_slots, snapshots};
     const bool recurrent = (dt == KDA_DTYPE_FP32) || (flags & KDA_FLAG_RECURRENT) || total_T == 0 ||
                            snapshots != nullptr;
-    const cudaError_t e = recurrent ? kda::launch_recurrent(a, s) : kda::launch_chunk(a, s);
+    // the two-pass tensor-core path when the workspace holds its scratch,
+    // else the fused single kernel (same arithmetic, no scratch)
+    const bool two_pass =
+        !recurrent && workspace_bytes >= kWorkspaceHeader + kda::two_pass_scratch_bytes(N, total_T, H);
+    const cudaError_t e = recurrent  ? kda::launch_recurrent(a, s)
+                          : two_pass ? kda::launch_chunk_two_pass(a, static_cast<uint8_t*>(workspace) + kWorkspaceHeader, s)
+                                     : kda::launch_chunk(a, s);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

@@ -40,6 +40,7 @@
 // touch tensor-memory lanes 32*(warp%4) .. +31.
 #include "kda_common.cuh"
 #include "kda_launch.h"
+#include "kda_tile.cuh"
 #include "sm100.cuh"
 
 #include <mutex>
@@ -75,9 +76,7 @@ constexpr uint32_t KB_KBT = 16384;
 constexpr uint32_t KB_TP = 16384;
 constexpr uint32_t KB_VT = 4096;
 
-// Scratch of the triangular solve inside the dead XQ region: plain fp32
-// arrays with padded rows (stride kLd floats) so column walks spread over banks.
-constexpr int kLd = 68, kLd1 = 20, kLd2 = 36;
+// Scratch of the triangular solve inside the dead XQ region (kda_tile.cuh).
 constexpr uint32_t OFF_M = OFF_XQ;                         // M, 64 x kLd
 constexpr uint32_t OFF_T = OFF_M + 64 * kLd * 4;           // T, 64 x kLd
 constexpr uint32_t OFF_Y1 = OFF_T + 64 * kLd * 4;          // 2 x 16 x kLd1
@@ -93,39 +92,6 @@ constexpr uint32_t TM_COLS = 256;
 
 constexpr uint32_t ID_N96 = idesc_tf32(128, 96, false, false);
 constexpr uint32_t ID_N32 = idesc_tf32(128, 32, false, false);
-
-// Element (row, k) of a K-major operand tile at `base` with K-block stride `kb`.
-__device__ __forceinline__ float* K_at(uint8_t* smem, uint32_t base, uint32_t kb, int row, int k) {
-    return reinterpret_cast<float*>(smem + base + (k >> 5) * kb + sw128_off(row, (k & 31) >> 2)) + (k & 3);
-}
-
-__device__ __forceinline__ void st_tf32x4(uint8_t* smem, uint32_t off, float a, float b, float c, float d) {
-    *reinterpret_cast<float4*>(smem + off) = make_float4(to_tf32(a), to_tf32(b), to_tf32(c), to_tf32(d));
-}
-
-__device__ __forceinline__ uint32_t tm_lane(uint32_t tmem, int quarter, uint32_t col) {
-    return tmem + (static_cast<uint32_t>(32 * quarter) << 16) + col;
-}
-
-__device__ __forceinline__ uint64_t tdesc(uint32_t sb, uint32_t base) { return sdesc_sw128(sb + base, 16, 1024); }
-
-// mma.sync fragments from plain row-major fp32 arrays (leading dimension ld),
-// rounded to tf32 on the way: A tile 16 x 8 at (r0, k0), B tile 8 x 8 at (k0, n0).
-__device__ __forceinline__ void frag_a(uint32_t (&a)[4], const float* X, int ld, int r0, int k0, int g, int t) {
-    a[0] = tf32_bits(X[(r0 + g) * ld + k0 + t]);
-    a[1] = tf32_bits(X[(r0 + g + 8) * ld + k0 + t]);
-    a[2] = tf32_bits(X[(r0 + g) * ld + k0 + t + 4]);
-    a[3] = tf32_bits(X[(r0 + g + 8) * ld + k0 + t + 4]);
-}
-__device__ __forceinline__ void frag_b(uint32_t (&b)[2], const float* Y, int ld, int k0, int n0, int g, int t) {
-    b[0] = tf32_bits(Y[(k0 + t) * ld + n0 + g]);
-    b[1] = tf32_bits(Y[(k0 + t + 4) * ld + n0 + g]);
-}
-__device__ __forceinline__ void frag_store(float* D, int ld, int r0, int n0, const float (&d)[4], float sgn, int g,
-                                           int t) {
-    *reinterpret_cast<float2*>(D + (r0 + g) * ld + n0 + 2 * t) = make_float2(sgn * d[0], sgn * d[1]);
-    *reinterpret_cast<float2*>(D + (r0 + g + 8) * ld + n0 + 2 * t) = make_float2(sgn * d[2], sgn * d[3]);
-}
 
 __global__ void __launch_bounds__(kThreads, 1)
 kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -239,99 +205,18 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     // Kt, Qt (XQ), Kb (rows 0-63 of KS) and V^T, plus beta and exp(Gamma_C).
     // Contains one block barrier; every thread must call it.
     auto prep = [&](int L) {
-        // raw q, k of the thread's 8 rows x 4 channels into registers first:
-        // the tiles written below overwrite the raw staging area
-        uint2 qraw[8], kraw[8];
-        const uint8_t* rq = smem + OFF_KS;
-        const uint8_t* rk = smem + OFF_KS + kC * kD * 2;
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            const int r = 8 * warp + m;
-            qraw[m] = *reinterpret_cast<const uint2*>(rq + r * kD * 2 + lane * 8);
-            kraw[m] = *reinterpret_cast<const uint2*>(rk + r * kD * 2 + lane * 8);
-        }
-        // Gamma in log2 units, as channel pairs: prefix over the thread's 8 rows,
-        // then over warps through shared memory
-        const float2 l2e = make_float2(kLog2e, kLog2e);
-        float2 G[8][2];
-#pragma unroll
-        for (int x = 0; x < 2; ++x) {
-            float2 run = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                run = __ffma2_rn(make_float2(greg[m][2 * x], greg[m][2 * x + 1]), l2e, run);
-                G[m][x] = run;
-            }
-            *reinterpret_cast<float2*>(xch + warp * 128 + 4 * lane + 2 * x) = run;
-        }
-        __syncthreads();   // also: every thread holds its raw q, k in registers
-        float2 off[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        float2 GC[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll
-        for (int w = 0; w < 8; ++w) {
-            const float4 t = *reinterpret_cast<const float4*>(xch + w * 128 + 4 * lane);
-            if (w < warp) {
-                off[0] = __fadd2_rn(off[0], make_float2(t.x, t.y));
-                off[1] = __fadd2_rn(off[1], make_float2(t.z, t.w));
-            }
-            GC[0] = __fadd2_rn(GC[0], make_float2(t.x, t.y));
-            GC[1] = __fadd2_rn(GC[1], make_float2(t.z, t.w));
-        }
+        float2 GC[2];
+        prep_chunk_rows(smem + OFF_KS, smem + OFF_KS + kC * kD * 2, greg, xch, L, scale, l2norm != 0, GC,
+                        [&](int r, int kbi, int ch, float4 kt, float4 qt, float4 kb) {
+                            st_tf32x4(smem, OFF_XQ + kbi * KB_XQ + sw128_off(r, ch), kt.x, kt.y, kt.z, kt.w);
+                            st_tf32x4(smem, OFF_XQ + kbi * KB_XQ + sw128_off(64 + r, ch), qt.x, qt.y, qt.z, qt.w);
+                            st_tf32x4(smem, OFF_KS + kbi * KB_KS + sw128_off(r, ch), kb.x, kb.y, kb.z, kb.w);
+                        });
         if (warp == 0) {
             dc_s[4 * lane + 0] = ex2(GC[0].x); dc_s[4 * lane + 1] = ex2(GC[0].y);
             dc_s[4 * lane + 2] = ex2(GC[1].x); dc_s[4 * lane + 3] = ex2(GC[1].y);
         }
         if (tid < kC) beta_s[tid] = breg;
-        // offset to the chunk end: Gamma_r - Gamma_C = G + (off - GC)
-        const float2 rel[2] = {__fadd2_rn(off[0], make_float2(-GC[0].x, -GC[0].y)),
-                               __fadd2_rn(off[1], make_float2(-GC[1].x, -GC[1].y))};
-
-        // unpack, mask rows past the sequence end, and L2-normalise all 8 rows
-        float2 qv[8][2], kv[8][2];
-        float nrm[16];
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            const bool live = 8 * warp + m < L;
-            qv[m][0] = make_float2(__uint_as_float(qraw[m].x << 16), __uint_as_float(qraw[m].x & 0xFFFF0000u));
-            qv[m][1] = make_float2(__uint_as_float(qraw[m].y << 16), __uint_as_float(qraw[m].y & 0xFFFF0000u));
-            kv[m][0] = make_float2(__uint_as_float(kraw[m].x << 16), __uint_as_float(kraw[m].x & 0xFFFF0000u));
-            kv[m][1] = make_float2(__uint_as_float(kraw[m].y << 16), __uint_as_float(kraw[m].y & 0xFFFF0000u));
-            if (!live) {
-                qv[m][0] = qv[m][1] = kv[m][0] = kv[m][1] = make_float2(0.f, 0.f);
-            }
-            const float2 sq = __ffma2_rn(qv[m][1], qv[m][1], __fmul2_rn(qv[m][0], qv[m][0]));
-            const float2 sk = __ffma2_rn(kv[m][1], kv[m][1], __fmul2_rn(kv[m][0], kv[m][0]));
-            nrm[m] = sq.x + sq.y;
-            nrm[8 + m] = sk.x + sk.y;
-        }
-        if (l2norm) warp_allreduce16(nrm);
-        const int kbi = lane >> 3, ch = lane & 7;
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            const int r = 8 * warp + m;
-            const float nq = (l2norm ? rsqrtf(nrm[m] + kNormEps) : 1.f) * scale;
-            const float nk = l2norm ? rsqrtf(nrm[8 + m] + kNormEps) : 1.f;
-            float4 kt, qt, kb;
-            float* ktp = &kt.x;
-            float* qtp = &qt.x;
-            float* kbp = &kb.x;
-#pragma unroll
-            for (int x = 0; x < 2; ++x) {
-                // a = (Gamma_r - Gamma_C) / ln 2 >= 0 (the decay is cumulative, g <= 0)
-                const float2 a = __fadd2_rn(G[m][x], rel[x]);
-                const float2 e = make_float2(ex2(fminf(a.x, 126.f)), ex2(fminf(a.y, 126.f)));   // E >= 1
-                const float2 f = make_float2(ex2(-a.x), ex2(-a.y));                              // F <= 1
-                const float2 kn = __fmul2_rn(kv[m][x], make_float2(nk, nk));
-                const float2 qn = __fmul2_rn(qv[m][x], make_float2(nq, nq));
-                const float2 t1 = __fmul2_rn(kn, e), t2 = __fmul2_rn(qn, e), t3 = __fmul2_rn(kn, f);
-                ktp[2 * x] = t1.x; ktp[2 * x + 1] = t1.y;
-                qtp[2 * x] = t2.x; qtp[2 * x + 1] = t2.y;
-                kbp[2 * x] = t3.x; kbp[2 * x + 1] = t3.y;
-            }
-            st_tf32x4(smem, OFF_XQ + kbi * KB_XQ + sw128_off(r, ch), kt.x, kt.y, kt.z, kt.w);
-            st_tf32x4(smem, OFF_XQ + kbi * KB_XQ + sw128_off(64 + r, ch), qt.x, qt.y, qt.z, qt.w);
-            st_tf32x4(smem, OFF_KS + kbi * KB_KS + sw128_off(r, ch), kb.x, kb.y, kb.z, kb.w);
-        }
         {   // V^T: token tid/4, value columns 8*(tid%4) .. +7 (exact bf16 -> fp32)
             const int r = tid >> 2, j0 = 8 * (tid & 3);
             const uint32_t w4[4] = {vreg.x, vreg.y, vreg.z, vreg.w};
@@ -469,98 +354,23 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             float* Tf = reinterpret_cast<float*>(smem + OFF_T);
             float* Y1 = reinterpret_cast<float*>(smem + OFF_Y1);   // [2][16][kLd1]
             float* Y2 = reinterpret_cast<float*>(smem + OFF_Y2);   // [32][kLd2]
-            if (tid < 64) {   // diagonal 16 x 16 blocks: column j of block b by substitution
-                const int b = tid >> 4, j = tid & 15;
-                const float* Mb = Mf + 16 * b * kLd + 16 * b;
-                float xv[16];
+            ut_inverse64(Mf, Tf, Y1, Y2, tid, [&] {
+                if (warp == 4 || warp == 5) {   // V^T -> (V - Y)^T for token rows 0-63
+                    float y[32];
+                    tc_fence_after();
+                    tmem_ld32(tm_lane(tmem, quarter, TM_X), y);
+                    tmem_wait_ld();
+                    const int r = 32 * quarter + lane;
+                    // all loads before all stores: the compiler cannot prove the
+                    // 32 addresses distinct, so an interleaved read-modify-write
+                    // would serialise on shared-memory latency
+                    float vv[32];
 #pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    float s0v = (r == j) ? 1.f : 0.f, s1v = 0.f;
+                    for (int e = 0; e < 32; ++e) vv[e] = *K_at(smem, OFF_VT, KB_VT, e, r);
 #pragma unroll
-                    for (int i = 0; i < r; i += 2) {
-                        s0v = fmaf(-Mb[r * kLd + i], xv[i], s0v);
-                        if (i + 1 < r) s1v = fmaf(-Mb[r * kLd + i + 1], xv[i + 1], s1v);
-                    }
-                    xv[r] = s0v + s1v;
+                    for (int e = 0; e < 32; ++e) *K_at(smem, OFF_VT, KB_VT, e, r) = to_tf32(vv[e] - y[e]);
                 }
-                float* Tb = Tf + 16 * b * kLd + 16 * b + j;
-#pragma unroll
-                for (int r = 0; r < 16; ++r) Tb[r * kLd] = xv[r];
-            } else if (tid < 128) {   // zero blocks (0,1) and (2,3), read by the 32 -> 64 merge
-                const int e = tid - 64, blk = e >> 5, rr = (e & 31) >> 1, c8 = (e & 1) * 8;
-                float* z = Tf + (32 * blk + rr) * kLd + 32 * blk + 16 + c8;
-                *reinterpret_cast<float4*>(z) = make_float4(0.f, 0.f, 0.f, 0.f);
-                *reinterpret_cast<float4*>(z + 4) = make_float4(0.f, 0.f, 0.f, 0.f);
-            } else if (warp == 4 || warp == 5) {   // V^T -> (V - Y)^T for token rows 0-63
-                float y[32];
-                tc_fence_after();
-                tmem_ld32(tm_lane(tmem, quarter, TM_X), y);
-                tmem_wait_ld();
-                const int r = 32 * quarter + lane;
-                // all loads before all stores: the compiler cannot prove the
-                // 32 addresses distinct, so an interleaved read-modify-write
-                // would serialise on shared-memory latency
-                float vv[32];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) vv[e] = *K_at(smem, OFF_VT, KB_VT, e, r);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) *K_at(smem, OFF_VT, KB_VT, e, r) = to_tf32(vv[e] - y[e]);
-            }
-            __syncthreads();
-            {   // 16 -> 32 on tensor cores: T_ab = -T_aa (M_ab T_bb) for (a, b) = (1, 0), (3, 2);
-                // warp w < 4 owns pair p = w / 2, output columns 8 (w % 2) .. +7
-                const int gq = lane >> 2, tq = lane & 3;
-                const int p = warp >> 1, nt = warp & 1, a = 2 * p + 1, b = 2 * p;
-                if (warp < 4) {
-                    float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int ks = 0; ks < 2; ++ks) {
-                        uint32_t fa[4], fb[2];
-                        frag_a(fa, Mf, kLd, 16 * a, 16 * b + 8 * ks, gq, tq);
-                        frag_b(fb, Tf, kLd, 16 * b + 8 * ks, 16 * b + 8 * nt, gq, tq);
-                        mma_m16n8k8_tf32(d, fa, fb);
-                    }
-                    frag_store(Y1 + p * 16 * kLd1, kLd1, 0, 8 * nt, d, 1.f, gq, tq);
-                }
-                __syncthreads();
-                if (warp < 4) {
-                    float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                    for (int ks = 0; ks < 2; ++ks) {
-                        uint32_t fa[4], fb[2];
-                        frag_a(fa, Tf, kLd, 16 * a, 16 * a + 8 * ks, gq, tq);
-                        frag_b(fb, Y1 + p * 16 * kLd1, kLd1, 8 * ks, 8 * nt, gq, tq);
-                        mma_m16n8k8_tf32(d, fa, fb);
-                    }
-                    frag_store(Tf, kLd, 16 * a, 16 * b + 8 * nt, d, -1.f, gq, tq);
-                }
-            }
-            __syncthreads();
-            {   // 32 -> 64 on tensor cores: T_hl = -T_hh (M_hl T_ll); warp w owns the
-                // 16 x 8 output tile (rows 16 (w / 4), columns 8 (w % 4))
-                const int gq = lane >> 2, tq = lane & 3;
-                const int mt = warp >> 2, nt = warp & 3;
-                float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    uint32_t fa[4], fb[2];
-                    frag_a(fa, Mf, kLd, 32 + 16 * mt, 8 * ks, gq, tq);
-                    frag_b(fb, Tf, kLd, 8 * ks, 8 * nt, gq, tq);
-                    mma_m16n8k8_tf32(d, fa, fb);
-                }
-                frag_store(Y2, kLd2, 16 * mt, 8 * nt, d, 1.f, gq, tq);
-                __syncthreads();
-                float e4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    uint32_t fa[4], fb[2];
-                    frag_a(fa, Tf, kLd, 32 + 16 * mt, 32 + 8 * ks, gq, tq);
-                    frag_b(fb, Y2, kLd2, 8 * ks, 8 * nt, gq, tq);
-                    mma_m16n8k8_tf32(e4, fa, fb);
-                }
-                frag_store(Tf, kLd, 32 + 16 * mt, 8 * nt, e4, -1.f, gq, tq);
-            }
-            __syncthreads();
+            });
             {   // T' = T diag(beta) on and below the diagonal, zero above; tf32 operand
                 const int r = tid >> 2;
                 float4 t4[4], b4[4];
@@ -675,6 +485,9 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
 }
 
+}  // namespace
+
+namespace {
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
                                    CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
@@ -692,22 +505,21 @@ EncodeTiledFn get_encode_fn() {
     });
     return fn;
 }
+}  // namespace
 
-// [total_T, H, 128] bf16 viewed as a 3-D tensor (channel, head, token); one
-// box is 64 tokens x 128 channels of one head, no swizzle, rows of 256 bytes.
-bool make_qk_map(CUtensorMap* map, const void* base, int64_t total_T, int H) {
+bool make_token_map(CUtensorMap* map, const void* base, int64_t total_T, int H, bool f32) {
     EncodeTiledFn enc = get_encode_fn();
     if (!enc) return false;
+    const cuuint64_t esz = f32 ? 4 : 2;
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(total_T)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(kD) * 2, static_cast<cuuint64_t>(H) * kD * 2};
-    cuuint32_t box[3] = {kD, 1, kC};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(kD) * esz, static_cast<cuuint64_t>(H) * kD * esz};
+    cuuint32_t box[3] = {kD, 1, 64};
     cuuint32_t estr[3] = {1, 1, 1};
-    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+    return enc(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+               const_cast<void*>(base), dims, strides, box, estr,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
-
-}  // namespace
 
 cudaError_t launch_chunk(const PrefillArgs& a, cudaStream_t stream) {
     if (a.N == 0 || a.H == 0) return cudaSuccess;
@@ -720,7 +532,7 @@ cudaError_t launch_chunk(const PrefillArgs& a, cudaStream_t stream) {
     });
     if (attr_err != cudaSuccess) return attr_err;
     CUtensorMap mq, mk;
-    if (!make_qk_map(&mq, a.q, a.total_T, a.H) || !make_qk_map(&mk, a.k, a.total_T, a.H))
+    if (!make_token_map(&mq, a.q, a.total_T, a.H) || !make_token_map(&mk, a.k, a.total_T, a.H))
         return cudaErrorInvalidValue;
     const long long blocks = (long long)a.N * a.H * kSplit;
     kda_chunk_kernel<<<static_cast<unsigned>(blocks), kThreads, SMEM_BYTES, stream>>>(

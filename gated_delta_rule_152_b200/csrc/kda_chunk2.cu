@@ -1,0 +1,783 @@
+// kda_chunk2.cu -- two-pass chunked KDA prefill on Blackwell tensor cores
+// (tcgen05 kind::tf32, accumulators in tensor memory, TMA and bulk copies).
+//
+// The layer's rule (page "GLM-5.3-FLASH", dimsnsums.com, section "How can a
+// layer remember without rereading?"):
+//     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,
+//     o_t = scale * S_t^T q_t.
+// Evaluated 64 tokens at a time with the chunk algebra of kda_chunk.cu
+// (Gamma, E, F, Kt, Qt, Kb, A, P, M, T' as defined there).  With
+//     W = T' Kt   and   U = T' V,
+// the correction of a chunk is delta = T' (V - Kt St) = U - W St, so
+//     O = Qt St + P delta,    S_next = St + Kb^T delta,    St = Diag(e^Gamma_C) S.
+// Everything except the last line is independent of the state.  Pass 1
+// (kda_chunk_prep_kernel) therefore runs over all (chunk, head) pairs in
+// parallel and writes, per pair, ready-made tensor-core operand images of
+// [Qt ; W] and [Kb^T ; P], and U and e^Gamma_C, to scratch.  Pass 2
+// (kda_chunk_state_kernel) walks the chunks of one (sequence, head) in order
+// and only carries the state:
+//     [Z^T | Y^T] = St^T [Qt ; W]^T            (M = 128 value columns, N = 128)
+//     delta^T = U^T - Y^T
+//     [S_next^T | O^T] = [St^T | Z^T] + delta^T [Kb^T ; P]^T    (N = 192)
+// The state is kept transposed in tensor memory (lane = value column, column
+// = key channel), so it is the A operand of the first product and the
+// accumulator of the second, and the readout O^T lands with the value
+// column in the lane, which is the contiguous axis of o in global memory.
+//
+// Precision: as the fused kernel -- tf32 operands (rounded to nearest),
+// fp32 accumulation, fp32 state; U is kept in fp32.
+#include "kda_common.cuh"
+#include "kda_launch.h"
+#include "kda_tile.cuh"
+#include "sm100.cuh"
+
+#include <mutex>
+
+namespace kda {
+namespace {
+
+constexpr int kC = 64;
+constexpr int kThreads = 256;
+
+// ---- per (chunk, head) operand image in scratch (byte offsets); tiles are
+// K-major with the 128-byte swizzle, exactly as they sit in shared memory.
+constexpr uint32_t IMG_B1 = 0;        // [Qt ; W]: rows 0-63 Qt, 64-127 W (token) x 128 channels, 4 K-blocks x 16 KB
+constexpr uint32_t IMG_DC = 65536;    // exp(Gamma_C): 128 fp32 (+ 512 B pad)
+constexpr uint32_t IMG_B2 = 66560;    // [Kb^T ; P]: rows 0-127 Kb^T (channel), 128-191 P (token) x 64 tokens, 2 K-blocks x 24 KB
+constexpr uint32_t IMG_U = 115712;    // U: [token][value column] fp32, 64 x 128
+constexpr uint32_t IMG_BYTES = 148480;
+constexpr uint32_t KB_B1 = 16384, KB_B2 = 24576;
+constexpr uint32_t B1_COPY = IMG_DC + 512;   // [Qt ; W] and exp(Gamma_C) in one copy
+constexpr uint32_t B2_COPY = 49152;
+static_assert(IMG_B2 % 1024 == 0 && IMG_U == IMG_B2 + B2_COPY && IMG_BYTES == IMG_U + 32768, "image layout");
+
+__device__ __forceinline__ bool seq_bounds(const int32_t* cu, int n, int64_t total_T, int64_t& bos, int64_t& eos) {
+    bos = cu[n];
+    eos = cu[n + 1];
+    return !(bos < 0 || eos < bos || eos > total_T);
+}
+
+// ============================================================ chunk index
+// chunk_off[n] = number of 64-token chunks of sequences 0..n-1 (exclusive
+// scan), chunk_off[N] = total.  A sequence with inconsistent cu_seqlens gets
+// no chunks and sets error bit 1.  Sequences that are each in bounds but
+// overlap (cu_seqlens not non-decreasing) can add up to more chunks than the
+// scratch holds (max_total): that also sets error bit 1, and both passes
+// skip every chunk at or past max_total.  One block.
+__global__ void __launch_bounds__(1024) kda_chunk_index_kernel(const int32_t* __restrict__ cu, int N,
+                                                               int64_t total_T, int64_t max_total,
+                                                               int32_t* __restrict__ chunk_off, uint32_t* err) {
+    __shared__ int32_t wsum[32];
+    __shared__ int32_t carry_s;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) carry_s = 0;
+    __syncthreads();
+    for (int base = 0; base < N; base += 1024) {
+        const int n = base + tid;
+        int32_t cnt = 0;
+        if (n < N) {
+            int64_t bos, eos;
+            if (seq_bounds(cu, n, total_T, bos, eos)) cnt = static_cast<int32_t>((eos - bos + kC - 1) / kC);
+            else set_error(err, 1u);
+        }
+        int32_t x = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) wsum[warp] = x;
+        __syncthreads();
+        if (warp == 0) {
+            int32_t w = wsum[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int32_t y = __shfl_up_sync(0xffffffffu, w, o);
+                if (lane >= o) w += y;
+            }
+            wsum[lane] = w;
+        }
+        __syncthreads();
+        const int32_t carry = carry_s;
+        const int32_t incl = x + (warp > 0 ? wsum[warp - 1] : 0);
+        if (n < N) chunk_off[n] = carry + incl - cnt;
+        __syncthreads();
+        if (tid == 1023) carry_s = carry + incl;
+        __syncthreads();
+    }
+    if (tid == 0) {
+        chunk_off[N] = carry_s;
+        if (carry_s > max_total) set_error(err, 1u);
+    }
+}
+
+// ============================================================ pass 1
+// Shared memory (byte offsets from a 1024-aligned base).
+constexpr uint32_t P_X = 0;          // 64 KB [Qt ; Kt]: 128 rows x 128 channels, 4 K-blocks x 16 KB.
+                                     //   After the Gram MMA: triangular-solve scratch, and T' at P_TP.
+constexpr uint32_t P_TP = 49152;     // 16 KB T': 64 rows (token r) x 64 (token i), 2 K-blocks x 8 KB
+constexpr uint32_t P_KB = 65536;     // 32 KB Kb: 64 rows x 128 channels, 4 K-blocks x 8 KB; also the
+                                     //   TMA destination of the next item's raw q (16 KB) and k (16 KB)
+constexpr uint32_t P_KTT = 98304;    // 32 KB Kt^T: 128 channel rows x 64 tokens, 2 K-blocks x 16 KB
+constexpr uint32_t P_VT = 131072;    // 32 KB V^T: 128 value rows x 64 tokens, 2 K-blocks x 16 KB
+constexpr uint32_t P_RV = 163840;    // 16 KB raw v (bf16 [64 tokens][128]); after the prep, the P tile
+                                     //   (64 rows x 64 tokens, 2 K-blocks x 8 KB) on its way to the image
+constexpr uint32_t P_KBTS = 180224;  // 32 KB Kb^T (128 channel rows x 64 tokens) on its way to the image
+constexpr uint32_t P_MISC = 212992;  // beta[64] | xch[8][128] at +1024 | barriers at +5120
+constexpr uint32_t P_SMEM = P_MISC + 6144 + 1024;
+constexpr uint32_t P_KB_KB = 8192, P_KB_TP = 8192, P_KB_T = 16384;
+constexpr int kStoreThread = 128;    // issues the bulk stores and the next item's TMA loads
+static_assert(kUtScratchBytes <= P_TP, "solve scratch overlaps T'");
+
+constexpr uint32_t TP_AP = 0;     // 64 cols: P (lanes 0-63) | A (lanes 64-127)
+constexpr uint32_t TP_W = 64;     // 64 cols: W^T (lane = channel, column = token)
+constexpr uint32_t TP_U = 128;    // 64 cols: U^T (lane = value column, column = token)
+constexpr uint32_t TP_COLS = 256;
+constexpr uint32_t ID_N64 = idesc_tf32(128, 64, false, false);
+
+__global__ void __launch_bounds__(kThreads, 1)
+kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ g,
+                      const float* __restrict__ beta, const int32_t* __restrict__ cu,
+                      const int32_t* __restrict__ chunk_off, int N, int H, int64_t max_total, float scale,
+                      int l2norm, int scalar_g, uint8_t* __restrict__ img, uint32_t* err) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sb = smem_u32(smem);
+    float* beta_s = reinterpret_cast<float*>(smem + P_MISC);
+    float* xch = reinterpret_cast<float*>(smem + P_MISC + 1024);
+    uint64_t* bar_load = reinterpret_cast<uint64_t*>(smem + P_MISC + 5120);
+    uint64_t* bar_mma = bar_load + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_mma + 1);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quarter = warp & 3, half = warp >> 2;
+    const int64_t total = chunk_off[N];
+    const int64_t items = (total < max_total ? total : max_total) * H;
+    if (static_cast<int64_t>(blockIdx.x) >= items) return;
+
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, TP_COLS);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(bar_load, 1);
+        mbar_init(bar_mma, 1);
+        fence_mbar_init();
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    // work item w -> chunk gc = w / H of head h = w % H; sequence n = the last
+    // one whose first chunk is <= gc (sequences without chunks are skipped)
+    struct Item {
+        int64_t t0, gc;
+        int L, h;
+    };
+    auto decode = [&](int64_t w) {
+        Item it;
+        it.gc = w / H;
+        it.h = static_cast<int>(w - it.gc * H);
+        int lo = 0, hi = N;
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (chunk_off[mid] <= it.gc) lo = mid;
+            else hi = mid;
+        }
+        it.t0 = cu[lo] + (it.gc - chunk_off[lo]) * kC;
+        const int64_t rem = cu[lo + 1] - it.t0;
+        it.L = static_cast<int>(rem < kC ? rem : (int64_t)kC);
+        return it;
+    };
+    float greg[8][4];
+    float breg;
+    auto prefetch = [&](const Item& it) {
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            const int r = 8 * warp + m;
+            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (r < it.L) {
+                if (scalar_g) {
+                    const float gs = __ldg(g + (size_t)(it.t0 + r) * H + it.h);
+                    x = make_float4(gs, gs, gs, gs);
+                } else {
+                    x = __ldg(reinterpret_cast<const float4*>(g + ((size_t)(it.t0 + r) * H + it.h) * kD + 4 * lane));
+                }
+            }
+            greg[m][0] = x.x; greg[m][1] = x.y; greg[m][2] = x.z; greg[m][3] = x.w;
+        }
+        breg = 0.f;
+        if (tid < it.L) breg = __ldg(beta + (size_t)(it.t0 + tid) * H + it.h);
+    };
+    auto issue_load = [&](const Item& it) {
+        mbar_arrive_expect_tx(bar_load, 3u * kC * kD * 2u);
+        const int32_t t0 = static_cast<int32_t>(it.t0);
+        tma_load_3d(smem + P_KB, &tm_q, bar_load, 0, it.h, t0);
+        tma_load_3d(smem + P_KB + kC * kD * 2, &tm_k, bar_load, 0, it.h, t0);
+        tma_load_3d(smem + P_RV, &tm_v, bar_load, 0, it.h, t0);
+    };
+
+    bool ok = true;
+    uint32_t load_parity = 0, mma_phase = 0;
+    bool load_pending = false, mma_pending = false;
+    auto wait_mma = [&]() -> bool {
+        const bool good = !__syncthreads_or(!mbar_wait_bounded(bar_mma, mma_phase));
+        if (good) {
+            mma_phase ^= 1;
+            mma_pending = false;
+            tc_fence_after();
+        }
+        return good;
+    };
+
+    int64_t w = blockIdx.x;
+    Item cur = decode(w);
+    if (tid == 0) issue_load(cur);
+    load_pending = true;
+    prefetch(cur);
+
+    for (; ok && w < items; w += gridDim.x) {
+        const int64_t wn = w + gridDim.x;
+        const bool has_next = wn < items;
+        const Item nxt = has_next ? decode(wn) : cur;
+        uint8_t* im = img + (static_cast<size_t>(cur.gc) * H + cur.h) * IMG_BYTES;
+        const int L = cur.L;
+
+        if (!(ok = !__syncthreads_or(!mbar_wait_bounded(bar_load, load_parity)))) break;
+        load_pending = false;
+        load_parity ^= 1;
+
+        // ============== prep: [Qt ; Kt] -> X, Kb -> KB, V^T -> VT, exp(Gamma_C) -> image
+        {
+            float2 GC[2];
+            prep_chunk_rows(smem + P_KB, smem + P_KB + kC * kD * 2, greg, xch, L, scale, l2norm != 0, GC,
+                            [&](int r, int kbi, int ch, float4 kt, float4 qt, float4 kb) {
+                                st_tf32x4(smem, P_X + kbi * KB_B1 + sw128_off(r, ch), qt.x, qt.y, qt.z, qt.w);
+                                st_tf32x4(smem, P_X + kbi * KB_B1 + sw128_off(64 + r, ch), kt.x, kt.y, kt.z, kt.w);
+                                st_tf32x4(smem, P_KB + kbi * P_KB_KB + sw128_off(r, ch), kb.x, kb.y, kb.z, kb.w);
+                            });
+            if (warp == 0)
+                *reinterpret_cast<float4*>(im + IMG_DC + 16 * lane) =
+                    make_float4(ex2(GC[0].x), ex2(GC[0].y), ex2(GC[1].x), ex2(GC[1].y));
+            if (tid < kC) beta_s[tid] = breg;
+            // V^T from the raw v tile: thread = value column e, 32 tokens; rows past L are zero
+            const int e = tid & 127, tg = tid >> 7;
+            const __nv_bfloat16* rv = reinterpret_cast<const __nv_bfloat16*>(smem + P_RV);
+            float vv[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int i = 32 * tg + j;
+                vv[j] = (i < L) ? __bfloat162float(rv[i * kD + e]) : 0.f;
+            }
+#pragma unroll
+            for (int b = 0; b < 8; ++b)
+                *reinterpret_cast<float4*>(K_at(smem, P_VT, P_KB_T, e, 32 * tg + 4 * b)) =
+                    make_float4(vv[4 * b], vv[4 * b + 1], vv[4 * b + 2], vv[4 * b + 3]);
+        }
+        __syncthreads();
+
+        // ============== Kt^T -> KTT (shared), Kb^T -> image; thread = channel, 32 tokens
+        {
+            const int cch = tid & 127, tg = tid >> 7;
+            float4 x[8], y[8];
+#pragma unroll
+            for (int b = 0; b < 8; ++b) {
+                const int i0 = 32 * tg + 4 * b;
+                x[b].x = *K_at(smem, P_X, KB_B1, 64 + i0 + 0, cch);
+                x[b].y = *K_at(smem, P_X, KB_B1, 64 + i0 + 1, cch);
+                x[b].z = *K_at(smem, P_X, KB_B1, 64 + i0 + 2, cch);
+                x[b].w = *K_at(smem, P_X, KB_B1, 64 + i0 + 3, cch);
+                y[b].x = *K_at(smem, P_KB, P_KB_KB, i0 + 0, cch);
+                y[b].y = *K_at(smem, P_KB, P_KB_KB, i0 + 1, cch);
+                y[b].z = *K_at(smem, P_KB, P_KB_KB, i0 + 2, cch);
+                y[b].w = *K_at(smem, P_KB, P_KB_KB, i0 + 3, cch);
+            }
+#pragma unroll
+            for (int b = 0; b < 8; ++b) {
+                const int i0 = 32 * tg + 4 * b;
+                *reinterpret_cast<float4*>(K_at(smem, P_KTT, P_KB_T, cch, i0)) = x[b];
+                *reinterpret_cast<float4*>(K_at(smem, P_KBTS, P_KB_T, cch, i0)) = y[b];
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == kStoreThread) {   // Kb^T -> image rows 0-127 of [Kb^T ; P]; Qt -> rows 0-63 of [Qt ; W]
+#pragma unroll
+            for (int kb = 0; kb < 2; ++kb)
+                bulk_store(im + IMG_B2 + kb * KB_B2, smem + P_KBTS + kb * P_KB_T, P_KB_T);
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb)
+                bulk_store(im + IMG_B1 + kb * KB_B1, smem + P_X + kb * KB_B1, 64 * 128);
+            bulk_commit();
+        }
+
+        // ============== [Qt ; Kt] x Kb^T -> P (lanes 0-63), A (lanes 64-127)
+        if (tid == 0) {
+            tc_fence_after();
+            const uint64_t dx = tdesc(sb, P_X), dkb = tdesc(sb, P_KB);
+#pragma unroll
+            for (int s = 0; s < 16; ++s)
+                mma_tf32_ss(tmem + TP_AP, kstep(dx, KB_B1, s), kstep(dkb, P_KB_KB, s), ID_N64, s > 0);
+            mma_commit(bar_mma);
+        }
+        mma_pending = true;
+        if (tid == kStoreThread) bulk_wait_read();   // X is scratch from here on
+        if (!(ok = wait_mma())) break;
+
+        // ============== P -> staging tile (tf32, lower incl.), A -> M = strict_lower(beta A) (fp32)
+        float* Mf = reinterpret_cast<float*>(smem + P_X);
+        float* Tf = Mf + 64 * kLd;
+        float* Y1 = Tf + 64 * kLd;
+        float* Y2 = Y1 + 2 * 16 * kLd1;
+        {
+            float acc[32];
+            tmem_ld32(tm_lane(tmem, quarter, TP_AP + 32 * half), acc);
+            tmem_wait_ld();
+            if (quarter < 2) {   // P (lower incl.) -> the staging tile in RV (raw v is consumed)
+                const int r = 32 * quarter + lane;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int i0 = 32 * half + 4 * j;
+                    *reinterpret_cast<float4*>(smem + P_RV + half * P_KB_TP + sw128_off(r, j)) =
+                        tf32x4((i0 + 0 <= r) ? acc[4 * j + 0] : 0.f, (i0 + 1 <= r) ? acc[4 * j + 1] : 0.f,
+                               (i0 + 2 <= r) ? acc[4 * j + 2] : 0.f, (i0 + 3 <= r) ? acc[4 * j + 3] : 0.f);
+                }
+            } else {
+                const int r = 32 * quarter + lane - 64;
+                const float br = beta_s[r];
+                float* mrow = Mf + r * kLd + 32 * half;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int i0 = 32 * half + 4 * j;
+                    *reinterpret_cast<float4*>(mrow + 4 * j) =
+                        make_float4((i0 + 0 < r) ? br * acc[4 * j + 0] : 0.f, (i0 + 1 < r) ? br * acc[4 * j + 1] : 0.f,
+                                    (i0 + 2 < r) ? br * acc[4 * j + 2] : 0.f, (i0 + 3 < r) ? br * acc[4 * j + 3] : 0.f);
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // ============== T = (I + M)^-1, T' = T diag(beta) -> TP (tf32 operand, rows r, K = i);
+        // meanwhile the store thread sends P to the image and, once the staging
+        // tiles have been read, stages the next item's raw q, k, v (KB and RV are free)
+        ut_inverse64(Mf, Tf, Y1, Y2, tid, [&] {
+            if (tid == kStoreThread) {
+#pragma unroll
+                for (int kb = 0; kb < 2; ++kb)
+                    bulk_store(im + IMG_B2 + kb * KB_B2 + 128 * 128, smem + P_RV + kb * P_KB_TP, P_KB_TP);
+                bulk_commit();
+                bulk_wait_read();
+                if (has_next) issue_load(nxt);
+            }
+        });
+        load_pending = has_next;
+        {
+            const int r = tid >> 2;
+            float4 t4[4], b4[4];
+#pragma unroll
+            for (int qd = 0; qd < 4; ++qd) {
+                const int i0 = 16 * (tid & 3) + 4 * qd;
+                t4[qd] = *reinterpret_cast<const float4*>(Tf + r * kLd + i0);
+                b4[qd] = *reinterpret_cast<const float4*>(beta_s + i0);
+            }
+#pragma unroll
+            for (int qd = 0; qd < 4; ++qd) {
+                const int i0 = 16 * (tid & 3) + 4 * qd;
+                st_tf32x4(smem, P_TP + (i0 >> 5) * P_KB_TP + sw128_off(r, (i0 & 31) >> 2),
+                          (i0 + 0 <= r) ? t4[qd].x * b4[qd].x : 0.f, (i0 + 1 <= r) ? t4[qd].y * b4[qd].y : 0.f,
+                          (i0 + 2 <= r) ? t4[qd].z * b4[qd].z : 0.f, (i0 + 3 <= r) ? t4[qd].w * b4[qd].w : 0.f);
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // ============== W^T = Kt^T T'^T,  U^T = V^T T'^T
+        if (tid == 0) {
+            tc_fence_after();
+            const uint64_t dkt = tdesc(sb, P_KTT), dvt = tdesc(sb, P_VT), dtp = tdesc(sb, P_TP);
+#pragma unroll
+            for (int s = 0; s < 8; ++s) {
+                mma_tf32_ss(tmem + TP_W, kstep(dkt, P_KB_T, s), kstep(dtp, P_KB_TP, s), ID_N64, s > 0);
+                mma_tf32_ss(tmem + TP_U, kstep(dvt, P_KB_T, s), kstep(dtp, P_KB_TP, s), ID_N64, s > 0);
+            }
+            mma_commit(bar_mma);
+        }
+        mma_pending = true;
+        if (has_next) prefetch(nxt);
+        if (!(ok = wait_mma())) break;
+
+        // ============== W (tf32, a 64-row K-major tile) and U ([token][value],
+        // fp32) staged in X (free now), then bulk-stored to the image
+        {
+            float acc[32];
+            const int c = 32 * quarter + lane;   // channel (W) or value column (U)
+            tmem_ld32(tm_lane(tmem, quarter, TP_W + 32 * half), acc);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) *K_at(smem, P_X, P_KB_KB, 32 * half + j, c) = to_tf32(acc[j]);
+            tmem_ld32(tm_lane(tmem, quarter, TP_U + 32 * half), acc);
+            tmem_wait_ld();
+            float* dst = reinterpret_cast<float*>(smem + P_X + 32768) + (32 * half) * kD + c;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) dst[j * kD] = acc[j];
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == kStoreThread) {
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb)
+                bulk_store(im + IMG_B1 + kb * KB_B1 + 64 * 128, smem + P_X + kb * P_KB_KB, P_KB_KB);
+            bulk_store(im + IMG_U, smem + P_X + 32768, 32768);
+            bulk_commit();
+            bulk_wait_read();   // the next item's prep rewrites X
+        }
+        cur = nxt;
+    }
+
+    if (tid == kStoreThread) bulk_wait_all();
+    tc_fence_before();
+    __syncthreads();
+    if (!ok && tid == 0) {
+        set_error(err, 2u);
+        if (load_pending) mbar_wait_bounded(bar_load, load_parity, 1u << 16);
+        if (mma_pending) mbar_wait_bounded(bar_mma, mma_phase, 1u << 16);
+    }
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TP_COLS);
+    }
+}
+
+// ============================================================ pass 2
+constexpr uint32_t S_B1 = 0;          // 64 KB [Qt ; W] of the current chunk
+constexpr uint32_t S_DC = 65536;      // exp(Gamma_C), copied with [Qt ; W]
+constexpr uint32_t S_B2 = 66560;      // 48 KB [Kb^T ; P]
+constexpr uint32_t S_SA = 115712;     // 64 KB St^T: 128 value rows x 128 channels, 4 K-blocks x 16 KB
+constexpr uint32_t S_DT = 181248;     // 32 KB delta^T: 128 value rows x 64 tokens, 2 K-blocks x 16 KB
+constexpr uint32_t S_MISC = 214016;   // barriers, TMEM slot
+constexpr uint32_t S_SMEM = S_MISC + 1024 + 1024;
+static_assert(S_DC == S_B1 + IMG_DC && S_B2 % 1024 == 0 && S_SA % 1024 == 0 && S_DT % 1024 == 0, "layout");
+
+constexpr uint32_t TS_S = 0;      // 128 cols: S^T (lane = value column, column = key channel)
+constexpr uint32_t TS_Z = 128;    // 64 cols: Z^T, then O^T (column = token)
+constexpr uint32_t TS_Y = 192;    // 64 cols: Y^T
+constexpr uint32_t TS_COLS = 256;
+constexpr uint32_t ID_N128 = idesc_tf32(128, 128, false, false);
+constexpr uint32_t ID_N192 = idesc_tf32(128, 192, false, false);
+constexpr int kOutThread = 32;   // issues the O stores and the L2 prefetches (not the MMA thread)
+
+__global__ void __launch_bounds__(kThreads, 1)
+kda_chunk_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t* __restrict__ img,
+                       const int32_t* __restrict__ chunk_off,
+                       const int32_t* __restrict__ cu, int64_t total_T, int H, int64_t max_total,
+                       const float* s0, float* sT,
+                       float* __restrict__ o, uint32_t* err, const int32_t* __restrict__ slots, int num_slots) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sb = smem_u32(smem);
+    uint64_t* bar_b1 = reinterpret_cast<uint64_t*>(smem + S_MISC);
+    uint64_t* bar_b2 = bar_b1 + 1;
+    uint64_t* bar_mma = bar_b1 + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_b1 + 3);
+    const float* dc_s = reinterpret_cast<const float*>(smem + S_DC);
+
+    const int h = blockIdx.x % H;
+    const int n = blockIdx.x / H;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quarter = warp & 3, half = warp >> 2;
+    const int e = 32 * quarter + lane;   // value column of this thread's TMEM lane
+
+    int64_t bos, eos;
+    if (!seq_bounds(cu, n, total_T, bos, eos)) return;   // flagged by the index kernel
+    const int64_t sidx = slots ? static_cast<int64_t>(slots[n]) : static_cast<int64_t>(n);
+    if (slots && (sidx < 0 || sidx >= num_slots)) {
+        if (tid == 0 && h == 0) set_error(err, 4u);
+        return;
+    }
+    const int nch = static_cast<int>((eos - bos + kC - 1) / kC);
+    const int64_t gc0 = chunk_off[n];
+    if (gc0 + nch > max_total) return;   // overlapping sequences overflowed the scratch: flagged above
+    auto image = [&](int c) { return img + (static_cast<size_t>(gc0 + c) * H + h) * IMG_BYTES; };
+
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, TS_COLS);
+        tmem_relinquish();
+    }
+    if (tid == 0) {
+        mbar_init(bar_b1, 1);
+        mbar_init(bar_b2, 1);
+        mbar_init(bar_mma, 1);
+        fence_mbar_init();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const size_t state_off = ((size_t)sidx * H + h) * kD * kD;
+
+    // initial state, transposed: lane e = value column, columns = key rows 64*half ..
+    {
+        float r[32];
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+            const int c0 = 64 * half + 32 * part;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) r[j] = s0 ? s0[state_off + (size_t)(c0 + j) * kD + e] : 0.f;
+            tmem_st32(tm_lane(tmem, quarter, TS_S + c0), r);
+        }
+        tmem_wait_st();
+    }
+    auto load_b1 = [&](int c) {
+        mbar_arrive_expect_tx(bar_b1, B1_COPY);
+        const uint8_t* src = image(c);
+#pragma unroll
+        for (int p = 0; p < 4; ++p) bulk_load(smem + S_B1 + p * 16384, src + p * 16384, 16384, bar_b1);
+        bulk_load(smem + S_DC, src + IMG_DC, 512, bar_b1);
+    };
+    auto load_b2 = [&](int c) {
+        mbar_arrive_expect_tx(bar_b2, B2_COPY);
+        const uint8_t* src = image(c) + IMG_B2;
+#pragma unroll
+        for (int p = 0; p < 3; ++p) bulk_load(smem + S_B2 + p * 16384, src + p * 16384, 16384, bar_b2);
+    };
+    if (tid == 0 && nch > 0) {
+        load_b1(0);
+        load_b2(0);
+    }
+    // in-flight copies: pending flag and the chunk they belong to (its parity)
+    bool b1_pending = nch > 0, b2_pending = nch > 0, mma_pending = false, ok = true;
+    int b1_chunk = 0, b2_chunk = 0;
+    uint32_t mma_phase = 0;
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+        return !__syncthreads_or(!mbar_wait_bounded(bar, parity));
+    };
+    // O^T of the chunk at t0 (lanes = value column, columns = tokens 32*half ..):
+    // into the DT tile as [token][value] for one TMA store by kOutThread
+    // (staged, full chunks; DT is free between the second product of one
+    // chunk and the delta of the next), else straight to o
+    auto emit_o = [&](int64_t t0, int L, bool staged) {
+        float acc[32];
+        tmem_ld32(tm_lane(tmem, quarter, TS_Z + 32 * half), acc);
+        tmem_wait_ld();
+        if (staged) {
+            float* dst = reinterpret_cast<float*>(smem + S_DT) + (32 * half) * kD + e;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) dst[j * kD] = acc[j];
+        } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int r = 32 * half + j;
+                if (r < L) o[((size_t)(t0 + r) * H + h) * kD + e] = acc[j];
+            }
+        }
+    };
+    if (tid == kOutThread && nch > 1) prefetch_l2(image(1), IMG_BYTES);
+
+    int64_t t_prev = bos;
+    int L_prev = 0;
+    for (int c = 0; c < nch; ++c) {
+        const int64_t t0 = bos + (int64_t)c * kC;
+        const int L = static_cast<int>(eos - t0 < kC ? eos - t0 : (int64_t)kC);
+        const uint8_t* im = image(c);
+
+        // ---- the state of the chunk start is in TMEM: O of the previous chunk out,
+        // the state decayed to this chunk's end as the A operand
+        bool o_tma = false;
+        if (c > 0) {
+            if (!(ok = wait_all(bar_mma, mma_phase))) break;
+            mma_phase ^= 1;
+            mma_pending = false;
+            tc_fence_after();
+            if (tid == 0) load_b2(c);
+            b2_pending = true;
+            b2_chunk = c;
+            o_tma = L_prev == kC;
+            emit_o(t_prev, L_prev, o_tma);
+        }
+        if (tid == kOutThread && c + 2 < nch) prefetch_l2(image(c + 2), IMG_BYTES);
+        float u[32];   // U of this thread's value column, tokens 32*half .. (one 128-byte row per warp load)
+        {
+            const float* src = reinterpret_cast<const float*>(im + IMG_U) + (32 * half) * kD + e;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) u[j] = src[j * kD];
+        }
+        if (!(ok = wait_all(bar_b1, c & 1))) break;
+        b1_pending = false;
+        float st[2][32];   // St^T of this lane, key channels 64*half ..
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+            const int c0 = 64 * half + 32 * part;
+            tmem_ld32(tm_lane(tmem, quarter, TS_S + c0), st[part]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float4 d4 = *reinterpret_cast<const float4*>(dc_s + c0 + 4 * j);
+                st[part][4 * j] *= d4.x; st[part][4 * j + 1] *= d4.y;
+                st[part][4 * j + 2] *= d4.z; st[part][4 * j + 3] *= d4.w;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<float4*>(K_at(smem, S_SA, 16384, e, c0 + 4 * j)) =
+                    tf32x4(st[part][4 * j], st[part][4 * j + 1], st[part][4 * j + 2], st[part][4 * j + 3]);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // ---- [Z^T | Y^T] = St^T [Qt ; W]^T; meanwhile O of the previous chunk
+        // leaves by TMA and St goes back to TMEM (the second product accumulates onto it)
+        if (tid == 0) {
+            tc_fence_after();
+            const uint64_t da = tdesc(sb, S_SA), db = tdesc(sb, S_B1);
+#pragma unroll
+            for (int s = 0; s < 16; ++s)
+                mma_tf32_ss(tmem + TS_Z, kstep(da, 16384, s), kstep(db, KB_B1, s), ID_N128, s > 0);
+            mma_commit(bar_mma);
+        }
+        mma_pending = true;
+        if (tid == kOutThread && o_tma) {
+            tma_store_3d(&tm_o, smem + S_DT, 0, h, static_cast<int32_t>(t_prev));
+            bulk_commit();
+        }
+#pragma unroll
+        for (int part = 0; part < 2; ++part)
+            tmem_st32(tm_lane(tmem, quarter, TS_S + 64 * half + 32 * part), st[part]);
+        tmem_wait_st();
+        if (tid == kOutThread) bulk_wait_read();   // DT is written again below
+        if (!(ok = wait_all(bar_mma, mma_phase))) break;
+        mma_phase ^= 1;
+        mma_pending = false;
+        tc_fence_after();
+        if (tid == 0 && c + 1 < nch) load_b1(c + 1);
+        b1_pending = c + 1 < nch;
+        b1_chunk = c + 1;
+
+        // ---- delta^T = U^T - Y^T (tf32 operand, row = value column, K = token)
+        {
+            float y[32];
+            tmem_ld32(tm_lane(tmem, quarter, TS_Y + 32 * half), y);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<float4*>(K_at(smem, S_DT, 16384, e, 32 * half + 4 * j)) =
+                    tf32x4(u[4 * j] - y[4 * j], u[4 * j + 1] - y[4 * j + 1], u[4 * j + 2] - y[4 * j + 2],
+                           u[4 * j + 3] - y[4 * j + 3]);
+        }
+        if (!(ok = wait_all(bar_b2, c & 1))) break;
+        b2_pending = false;
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // ---- [S^T | O^T] += delta^T [Kb^T ; P]^T
+        if (tid == 0) {
+            tc_fence_after();
+            const uint64_t da = tdesc(sb, S_DT), db = tdesc(sb, S_B2);
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+                mma_tf32_ss(tmem + TS_S, kstep(da, 16384, s), kstep(db, KB_B2, s), ID_N192, 1);
+            mma_commit(bar_mma);
+        }
+        mma_pending = true;
+        t_prev = t0;
+        L_prev = L;
+    }
+    if (ok && nch > 0) {
+        if ((ok = wait_all(bar_mma, mma_phase))) {
+            mma_pending = false;
+            tc_fence_after();
+            emit_o(t_prev, L_prev, false);
+        }
+    }
+    if (ok) {
+        if (sT) {
+            float acc[32];
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                const int c0 = 64 * half + 32 * part;
+                tmem_ld32(tm_lane(tmem, quarter, TS_S + c0), acc);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) sT[state_off + (size_t)(c0 + j) * kD + e] = acc[j];
+            }
+        }
+    } else if (tid == 0) {
+        // a bounded wait gave up: report, give outstanding copies and MMAs a
+        // last bounded chance to land, then release tensor memory
+        set_error(err, 2u);
+        if (b1_pending) mbar_wait_bounded(bar_b1, b1_chunk & 1, 1u << 16);
+        if (b2_pending) mbar_wait_bounded(bar_b2, b2_chunk & 1, 1u << 16);
+        if (mma_pending) mbar_wait_bounded(bar_mma, mma_phase, 1u << 16);
+    }
+    if (tid == kOutThread) bulk_wait_all();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TS_COLS);
+    }
+}
+
+int num_sms() {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms > 0 ? sms : 148;
+}
+
+size_t max_chunks(int32_t N, int64_t total_T) { return static_cast<size_t>((total_T + 63 * (int64_t)N) / kC); }
+size_t index_bytes(int32_t N) { return (static_cast<size_t>(N + 1) * 4 + 1023) & ~size_t(1023); }
+
+}  // namespace
+
+size_t two_pass_scratch_bytes(int32_t N, int64_t total_T, int32_t H) {
+    if (N < 0 || total_T < 0 || H <= 0) return 0;
+    return index_bytes(N) + max_chunks(N, total_T) * static_cast<size_t>(H) * IMG_BYTES;
+}
+
+cudaError_t launch_chunk_two_pass(const PrefillArgs& a, void* scratch, cudaStream_t stream) {
+    if (a.N == 0 || a.H == 0) return cudaSuccess;
+    if (a.total_T <= 0) return cudaErrorInvalidValue;   // callers route empty batches elsewhere
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(kda_chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        static_cast<int>(P_SMEM));
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(kda_chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            static_cast<int>(S_SMEM));
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    CUtensorMap mq, mk, mv, mo;
+    if (!make_token_map(&mq, a.q, a.total_T, a.H) || !make_token_map(&mk, a.k, a.total_T, a.H) ||
+        !make_token_map(&mv, a.v, a.total_T, a.H) || !make_token_map(&mo, a.o, a.total_T, a.H, true))
+        return cudaErrorInvalidValue;
+    int32_t* chunk_off = static_cast<int32_t*>(scratch);
+    uint8_t* img = static_cast<uint8_t*>(scratch) + index_bytes(a.N);
+
+    const int64_t max_total = static_cast<int64_t>(max_chunks(a.N, a.total_T));
+    kda_chunk_index_kernel<<<1, 1024, 0, stream>>>(a.cu_seqlens, a.N, a.total_T, max_total, chunk_off, a.err);
+    const size_t items_ub = max_chunks(a.N, a.total_T) * static_cast<size_t>(a.H);
+    const size_t grid1 = items_ub < static_cast<size_t>(num_sms()) ? items_ub : static_cast<size_t>(num_sms());
+    if (grid1 > 0)
+        kda_chunk_prep_kernel<<<static_cast<unsigned>(grid1), kThreads, P_SMEM, stream>>>(
+            mq, mk, mv, a.g, a.beta, a.cu_seqlens, chunk_off, a.N, a.H, max_total, a.scale, a.l2norm ? 1 : 0,
+            a.scalar_decay ? 1 : 0, img, a.err);
+    const long long blocks = (long long)a.N * a.H;
+    kda_chunk_state_kernel<<<static_cast<unsigned>(blocks), kThreads, S_SMEM, stream>>>(
+        mo, img, chunk_off, a.cu_seqlens, a.total_T, a.H, max_total, a.initial_state, a.final_state, a.o, a.err, a.slots,
+        a.num_slots);
+    return cudaGetLastError();
+}
+
+}  // namespace kda

@@ -1,6 +1,7 @@
 // kda_launch.h -- host-side launchers of the KDA kernels (internal to libkda).
 #pragma once
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace kda {
@@ -31,8 +32,20 @@ struct PrefillArgs {
 // Token-by-token fp32 recurrence (CUDA cores), any dtype.
 cudaError_t launch_recurrent(const PrefillArgs& a, cudaStream_t stream);
 
-// Chunked tensor-core prefill (tcgen05, kind::tf32), bf16 q/k/v.
+// Chunked tensor-core prefill (tcgen05, kind::tf32), bf16 q/k/v, one fused
+// kernel per (sequence, head, 32-column value slice); needs no scratch.
 cudaError_t launch_chunk(const PrefillArgs& a, cudaStream_t stream);
+
+// Two-pass chunked prefill: a parallel pass over (chunk, head) that writes
+// each chunk's state-independent operands to scratch, then a sequential pass
+// per (sequence, head) that carries the state.  `scratch` (16-byte aligned)
+// must hold two_pass_scratch_bytes(N, total_T, H) bytes.
+size_t two_pass_scratch_bytes(int32_t N, int64_t total_T, int32_t H);
+cudaError_t launch_chunk_two_pass(const PrefillArgs& a, void* scratch, cudaStream_t stream);
+
+// [total_T, H, 128] bf16 (or fp32) viewed as a 3-D tensor (channel, head,
+// token) for TMA; one box is 64 tokens x 128 channels of one head, no swizzle.
+bool make_token_map(CUtensorMap* map, const void* base, int64_t total_T, int H, bool f32 = false);
 
 struct DecodeArgs {
     const void* q;

@@ -7,7 +7,10 @@
 // process that must not allocate after start-up).  For them this entry point
 // uses a scratch buffer that lives inside the library itself: a file-scope
 // __device__ array of kNoAllocScratchBytes bytes.  Every GPU that loads the
-// library holds that array until the process exits.
+// library holds that array until the process exits.  The array holds the
+// error word and the per-sequence reserve (kda_chunk_fwd_workspace_size_min),
+// not the per-chunk scratch of the two-pass path, so bf16 prefill through
+// this entry point runs the fused single kernel.
 //
 // The array's host-side name is only a stand-in for the symbol, not a device
 // address, so the device address is looked up with cudaGetSymbolAddress, once
@@ -41,7 +44,7 @@ extern "C" KDA_API int kda_chunk_fwd_noalloc(const void* q, const void* k, const
                                              int64_t total_T, int32_t H, int32_t d, kda_dtype dt,
                                              float scale, uint32_t flags, const float* initial_state,
                                              float* final_state, float* o, kda_stream_t stream) {
-    const size_t need = kda_chunk_fwd_workspace_size(N, total_T, H, d, dt);
+    const size_t need = kda_chunk_fwd_workspace_size_min(N, total_T, H, d, dt);
     if (need == 0) return d != 128 ? KDA_ERR_UNSUPPORTED : KDA_ERR_INVALID_ARG;
     if (need > kNoAllocScratchBytes) return KDA_ERR_WORKSPACE;   // N above KDA_NOALLOC_MAX_SEQS
 

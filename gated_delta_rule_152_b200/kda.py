@@ -34,7 +34,8 @@ KDA_DEVERR_CU_SEQLENS = 1
 KDA_DEVERR_TIMEOUT = 2
 KDA_DEVERR_SLOT = 4
 
-EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_decode_step",
+EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd_workspace_size_min", "kda_chunk_fwd",
+            "kda_decode_step",
             "kda_chunk_fwd_slots", "kda_decode_step_slots", "kda_verify_fwd", "kda_workspace_error",
             "kda_status_string")
 
@@ -62,6 +63,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                      ctypes.c_uint32, ctypes.c_float, ctypes.c_size_t)
         lib.kda_chunk_fwd_workspace_size.argtypes = [I32, I64, I32, I32, ctypes.c_int]
         lib.kda_chunk_fwd_workspace_size.restype = SZ
+        lib.kda_chunk_fwd_workspace_size_min.argtypes = [I32, I64, I32, I32, ctypes.c_int]
+        lib.kda_chunk_fwd_workspace_size_min.restype = SZ
         lib.kda_chunk_fwd.argtypes = [P, P, P, P, P, P, I32, I64, I32, I32, ctypes.c_int, F32, U32,
                                       P, P, P, P, SZ, P]
         lib.kda_chunk_fwd.restype = ctypes.c_int
@@ -125,6 +128,12 @@ def kda_chunk_fwd_workspace_size(N: int, total_T: int, H: int, d: int = 128,
     return int(load_library().kda_chunk_fwd_workspace_size(N, total_T, H, d, code))
 
 
+def kda_chunk_fwd_workspace_size_min(N: int, total_T: int, H: int, d: int = 128,
+                                     dtype: torch.dtype = torch.bfloat16) -> int:
+    code = KDA_DTYPE_BF16 if dtype == torch.bfloat16 else KDA_DTYPE_FP32
+    return int(load_library().kda_chunk_fwd_workspace_size_min(N, total_T, H, d, code))
+
+
 def kda_chunk_fwd(q, k, v, g, beta, cu_seqlens, *, scale: float = 1.0, l2norm: bool = True,
                   initial_state: Optional[torch.Tensor] = None, final_state=True,
                   o: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
@@ -163,9 +172,12 @@ def kda_chunk_fwd(q, k, v, g, beta, cu_seqlens, *, scale: float = 1.0, l2norm: b
     if o is None:
         o = torch.empty((T, H, d), dtype=torch.float32, device=dev)
     _check(o, "o", (T, H, d), torch.float32, dev)
-    ws_bytes = int(lib.kda_chunk_fwd_workspace_size(N, T, H, d, dt))
     if workspace is None:
-        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+        # the fp32 / recurrent path uses only the error word; bf16 gets the
+        # scratch of the two-pass tensor-core path
+        size_fn = (lib.kda_chunk_fwd_workspace_size_min if recurrent or dt == KDA_DTYPE_FP32
+                   else lib.kda_chunk_fwd_workspace_size)
+        workspace = torch.empty(max(int(size_fn(N, T, H, d, dt)), 256), dtype=torch.uint8, device=dev)
     flags = ((KDA_FLAG_L2NORM_QK if l2norm else 0) | (KDA_FLAG_RECURRENT if recurrent else 0) |
              (KDA_FLAG_SCALAR_DECAY if scalar_decay else 0))
     st = lib.kda_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), N, T, H,
@@ -232,9 +244,12 @@ def kda_chunk_fwd_slots(q, k, v, g, beta, cu_seqlens, state_pool, slots, *, scal
     if o is None:
         o = torch.empty((T, H, d), dtype=torch.float32, device=dev)
     _check(o, "o", (T, H, d), torch.float32, dev)
-    ws_bytes = int(lib.kda_chunk_fwd_workspace_size(N, T, H, d, dt))
     if workspace is None:
-        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+        # the fp32 / recurrent path uses only the error word; bf16 gets the
+        # scratch of the two-pass tensor-core path
+        size_fn = (lib.kda_chunk_fwd_workspace_size_min if recurrent or dt == KDA_DTYPE_FP32
+                   else lib.kda_chunk_fwd_workspace_size)
+        workspace = torch.empty(max(int(size_fn(N, T, H, d, dt)), 256), dtype=torch.uint8, device=dev)
     flags = ((KDA_FLAG_L2NORM_QK if l2norm else 0) | (KDA_FLAG_RECURRENT if recurrent else 0) |
              (KDA_FLAG_SCALAR_DECAY if scalar_decay else 0))
     st = lib.kda_chunk_fwd_slots(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), N, T, H,
@@ -305,7 +320,7 @@ def kda_verify_fwd(q, k, v, g, beta, cu_seqlens, *, initial_state: Optional[torc
     if o is None:
         o = torch.empty((T, H, d), dtype=torch.float32, device=dev)
     _check(o, "o", (T, H, d), torch.float32, dev)
-    ws_bytes = int(lib.kda_chunk_fwd_workspace_size(N, T, H, d, dt))
+    ws_bytes = int(lib.kda_chunk_fwd_workspace_size_min(N, T, H, d, dt))
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
     flags = (KDA_FLAG_L2NORM_QK if l2norm else 0) | (KDA_FLAG_SCALAR_DECAY if scalar_decay else 0)

@@ -57,7 +57,7 @@ typedef enum {
     KDA_ERR_INVALID_ARG = -1, /* NULL required pointer, negative size, bad cu_seqlens length */
     KDA_ERR_UNSUPPORTED = -2, /* d != 128, unsupported dtype or flag, device not sm_100 */
     KDA_ERR_MISALIGNED = -3,  /* a pointer is not 16-byte aligned */
-    KDA_ERR_WORKSPACE = -4,   /* workspace NULL or smaller than kda_chunk_fwd_workspace_size() */
+    KDA_ERR_WORKSPACE = -4,   /* workspace NULL or smaller than kda_chunk_fwd_workspace_size_min() */
     KDA_ERR_CUDA = -5         /* a CUDA runtime call or kernel launch failed */
 } kda_status;
 
@@ -89,11 +89,26 @@ enum {
 };
 
 /*
- * Bytes of device workspace kda_chunk_fwd needs for these sizes (the
- * error word plus the sequence schedule).  Returns 0 for invalid sizes.
+ * Bytes of device workspace with which kda_chunk_fwd (and _slots) runs its
+ * fastest path for these sizes: the error word, a chunk index, and the
+ * state-independent tensor-core operands of every (64-token chunk, head)
+ * pair, about 145 KiB per pair (8192 tokens x 32 heads: 608 MB).  Returns 0
+ * for invalid sizes.
  */
 KDA_API size_t kda_chunk_fwd_workspace_size(int32_t N, int64_t total_T, int32_t H, int32_t d,
                                     kda_dtype dt);
+
+/*
+ * The smallest workspace the prefill calls accept: the error word plus 4
+ * bytes per sequence.  With less than kda_chunk_fwd_workspace_size() the
+ * bf16 prefill runs a single fused kernel per (sequence, head, 32-column
+ * value slice) instead of the two-pass path; both evaluate the same chunk
+ * algebra in tf32 with fp32 accumulation.  kda_verify_fwd and the fp32 /
+ * KDA_FLAG_RECURRENT paths never need more than this.  Returns 0 for
+ * invalid sizes.
+ */
+KDA_API size_t kda_chunk_fwd_workspace_size_min(int32_t N, int64_t total_T, int32_t H, int32_t d,
+                                        kda_dtype dt);
 
 /*
  * Prefill over N packed variable-length sequences (the chunked form of the
@@ -117,9 +132,11 @@ KDA_API size_t kda_chunk_fwd_workspace_size(int32_t N, int64_t total_T, int32_t 
  *                 sequence gets final = initial.
  *   o             [total_T, H, d] fp32, written for every token.
  *   workspace     device scratch of at least
- *                 kda_chunk_fwd_workspace_size(...) bytes; its first word is
- *                 cleared by this call and receives KDA_DEVERR_* bits.  Calls
- *                 that share a workspace must be stream-ordered.
+ *                 kda_chunk_fwd_workspace_size_min(...) bytes (with
+ *                 kda_chunk_fwd_workspace_size(...) bytes the two-pass path
+ *                 runs); its first word is cleared by this call and receives
+ *                 KDA_DEVERR_* bits.  Calls that share a workspace must be
+ *                 stream-ordered.
  */
 KDA_API int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g,
                   const float *beta, const int32_t *cu_seqlens, int32_t N, int64_t total_T,

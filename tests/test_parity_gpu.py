@@ -41,11 +41,26 @@ def assert_close(gpu, ref, tol, what):
     return r
 
 
-def run_both(x: kin.PrefillInputs, recurrent=False, scale=1.0, l2norm=True, heads=None):
+# The bf16 prefill has two tensor-core paths: the two-pass one (prep pass over
+# all chunks, then the sequential state pass) runs when the workspace holds
+# its scratch -- the binding's default -- and the fused single kernel runs
+# with the minimum workspace.
+PATHS = ["two_pass", "fused"]
+
+
+def small_workspace(x: kin.PrefillInputs, dev):
+    T, H, _ = x.q.shape
+    N = x.cu_seqlens.numel() - 1
+    return torch.zeros(kda.kda_chunk_fwd_workspace_size_min(N, T, H), dtype=torch.uint8, device=dev)
+
+
+def run_both(x: kin.PrefillInputs, recurrent=False, scale=1.0, l2norm=True, heads=None, path="two_pass"):
     dev = torch.device("cuda")
     xd = x.to(dev)
+    ws = small_workspace(x, dev) if path == "fused" else None
     o, sT = kda.kda_chunk_fwd(xd.q, xd.k, xd.v, xd.g, xd.beta, xd.cu_seqlens, scale=scale,
-                              l2norm=l2norm, initial_state=xd.initial_state, recurrent=recurrent)
+                              l2norm=l2norm, initial_state=xd.initial_state, recurrent=recurrent,
+                              workspace=ws)
     torch.cuda.synchronize()
     sel = slice(None) if heads is None else list(heads)
     s0 = None if x.initial_state is None else x.initial_state[:, sel].contiguous()
@@ -71,17 +86,19 @@ def test_recurrent_kernel_bf16(lengths):
     assert_close(s, s_ref, TOL_FP32, "final state")
 
 
+@pytest.mark.parametrize("path", PATHS)
 @pytest.mark.parametrize("lengths", [[1], [63], [64], [65], [200], [1000]])
-def test_chunk_kernel_single_sequence(lengths):
+def test_chunk_kernel_single_sequence(lengths, path):
     x = kin.make_custom_prefill(21, lengths, heads=2, init_state_std=0.02)
-    o, s, o_ref, s_ref = run_both(x)
+    o, s, o_ref, s_ref = run_both(x, path=path)
     assert_close(o, o_ref, TOL_BF16, "o")
     assert_close(s, s_ref, TOL_BF16, "final state")
 
 
-def test_chunk_kernel_varlen_with_empty_and_ragged():
+@pytest.mark.parametrize("path", PATHS)
+def test_chunk_kernel_varlen_with_empty_and_ragged(path):
     x = kin.make_custom_prefill(22, [0, 5, 64, 130, 1, 257, 0, 128], heads=3, init_state_std=0.05)
-    o, s, o_ref, s_ref = run_both(x, scale=0.5)
+    o, s, o_ref, s_ref = run_both(x, scale=0.5, path=path)
     assert_close(o, o_ref, TOL_BF16, "o")
     assert_close(s, s_ref, TOL_BF16, "final state")
     # empty sequences: final state equals the initial state exactly
@@ -99,11 +116,12 @@ def test_chunk_kernel_without_l2norm():
     assert_close(s, s_ref, TOL_BF16, "final state")
 
 
-def test_chunk_kernel_strong_decay():
+@pytest.mark.parametrize("path", PATHS)
+def test_chunk_kernel_strong_decay(path):
     # per-chunk decay per channel around 40 nats (inside the tensor-core path's range)
     x = kin.make_custom_prefill(24, [300], heads=2, init_state_std=0.02)
     x.g = x.g * 8.0
-    o, s, o_ref, s_ref = run_both(x)
+    o, s, o_ref, s_ref = run_both(x, path=path)
     assert_close(o, o_ref, TOL_BF16, "o")
     assert_close(s, s_ref, TOL_BF16, "final state")
 
@@ -152,14 +170,16 @@ def test_zero_tokens_copies_initial_state():
     assert o.numel() == 0 and torch.equal(s, s0)
 
 
-def test_bad_cu_seqlens_flags_error_and_skips_only_that_sequence():
+@pytest.mark.parametrize("path", PATHS)
+def test_bad_cu_seqlens_flags_error_and_skips_only_that_sequence(path):
     x = kin.make_custom_prefill(27, [40, 30, 50], heads=2)
     dev = torch.device("cuda")
     xd = x.to(dev)
     # sequence 2 runs backwards (120 -> 60): flagged and skipped; sequences 0
     # and 1 (tokens 0-39 and 40-119) are consistent and do not overlap it
     bad = torch.tensor([0, 40, 120, 60], dtype=torch.int32, device=dev)
-    ws = torch.zeros(1024, dtype=torch.uint8, device=dev)
+    ws = torch.zeros(kda.kda_chunk_fwd_workspace_size(3, 120, 2) if path == "two_pass" else 1024,
+                     dtype=torch.uint8, device=dev)
     s0 = torch.randn(3, 2, 128, 128, device=dev)
     sT = torch.full((3, 2, 128, 128), 7.0, device=dev)
     o, s = kda.kda_chunk_fwd(xd.q, xd.k, xd.v, xd.g, xd.beta, bad, initial_state=s0, final_state=sT,
@@ -177,9 +197,33 @@ def test_bad_cu_seqlens_flags_error_and_skips_only_that_sequence():
     assert kda.kda_workspace_error(ws) == 0
 
 
-def test_prefill_8k_workload_full():
+def test_overlapping_sequences_cannot_overrun_the_two_pass_scratch():
+    # cu_seqlens [0, 200, 0, 200, 0, 200]: sequences 0, 2 and 4 are each in
+    # bounds but cover the same 200 tokens, 12 chunks in all, while the
+    # scratch is sized for (200 + 63 * 5) / 64 = 8.  The chunks past the
+    # scratch are not computed (sequence 4 is skipped) and the error bit is set.
+    x = kin.make_custom_prefill(28, [200], heads=2, init_state_std=0.02)
+    dev = torch.device("cuda")
+    xd = x.to(dev)
+    cu = torch.tensor([0, 200, 0, 200, 0, 200], dtype=torch.int32, device=dev)
+    s0 = xd.initial_state.expand(5, -1, -1, -1).contiguous()   # same start, so overlaps agree
+    sT = torch.full((5, 2, 128, 128), 7.0, device=dev)
+    ws = torch.zeros(kda.kda_chunk_fwd_workspace_size(5, 200, 2), dtype=torch.uint8, device=dev)
+    o, s = kda.kda_chunk_fwd(xd.q, xd.k, xd.v, xd.g, xd.beta, cu, initial_state=s0, final_state=sT,
+                             workspace=ws)
+    assert kda.kda_workspace_error(ws) & kda.KDA_DEVERR_CU_SEQLENS
+    o_ref, s_ref = oracle.kda_forward(x.q, x.k, x.v, x.g, x.beta, x.cu_seqlens, x.initial_state)
+    assert_close(o, o_ref, TOL_BF16, "o of the overlapping sequences")
+    for n in (0, 2):
+        assert_close(s[n:n + 1], s_ref, TOL_BF16, f"final state of sequence {n}")
+    for n in (1, 3, 4):
+        assert torch.all(s[n] == 7.0), f"sequence {n} must be skipped"
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_prefill_8k_workload_full(path):
     x = kin.make_prefill(kin.PREFILL_8K)
-    o, s, o_ref, s_ref = run_both(x)
+    o, s, o_ref, s_ref = run_both(x, path=path)
     assert_close(o, o_ref, TOL_BF16, "o")
     assert_close(s, s_ref, TOL_BF16, "final state")
 
@@ -246,13 +290,15 @@ def _scalar_decay_case(seed, lengths, heads=3):
     return x, gs, gs[..., None].expand_as(x.g).contiguous()
 
 
-@pytest.mark.parametrize("recurrent", [False, True])
-def test_scalar_decay_prefill(recurrent):
+@pytest.mark.parametrize("mode", ["recurrent"] + PATHS)
+def test_scalar_decay_prefill(mode):
     x, gs, gfull = _scalar_decay_case(41, [0, 70, 257, 64, 1])
     dev = torch.device("cuda")
     xd = x.to(dev)
+    recurrent = mode == "recurrent"
     o, s = kda.kda_chunk_fwd(xd.q, xd.k, xd.v, gs.to(dev), xd.beta, xd.cu_seqlens,
-                             initial_state=xd.initial_state, recurrent=recurrent, scalar_decay=True)
+                             initial_state=xd.initial_state, recurrent=recurrent, scalar_decay=True,
+                             workspace=small_workspace(x, dev) if mode == "fused" else None)
     torch.cuda.synchronize()
     o_ref, s_ref = oracle.kda_forward(x.q, x.k, x.v, gfull, x.beta, x.cu_seqlens, x.initial_state)
     tol = TOL_FP32 if recurrent else TOL_BF16
@@ -293,8 +339,9 @@ def test_scalar_decay_decode():
 # ---------------------------------------------------------------- state pools
 # Continuous batching: states live in a pool and sequence n uses slots[n].
 
-@pytest.mark.parametrize("recurrent", [False, True])
-def test_prefill_with_state_pool(recurrent):
+@pytest.mark.parametrize("mode", ["recurrent"] + PATHS)
+def test_prefill_with_state_pool(mode):
+    recurrent = mode == "recurrent"
     dev = torch.device("cuda")
     lengths, slots = [100, 0, 70], [4, 0, 5]
     x = kin.make_custom_prefill(51, lengths, heads=2, init_state_std=0.02)
@@ -303,7 +350,8 @@ def test_prefill_with_state_pool(recurrent):
     pool_d = pool.to(dev)
     xd = x.to(dev)
     o = kda.kda_chunk_fwd_slots(xd.q, xd.k, xd.v, xd.g, xd.beta, xd.cu_seqlens, pool_d,
-                                torch.tensor(slots, dtype=torch.int32, device=dev), recurrent=recurrent)
+                                torch.tensor(slots, dtype=torch.int32, device=dev), recurrent=recurrent,
+                                workspace=small_workspace(x, dev) if mode == "fused" else None)
     torch.cuda.synchronize()
     o_ref, s_ref = oracle.kda_forward(x.q, x.k, x.v, x.g, x.beta, x.cu_seqlens, x.initial_state)
     tol = TOL_FP32 if recurrent else TOL_BF16

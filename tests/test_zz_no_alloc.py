@@ -58,8 +58,11 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row():
         x = kin.make_custom_prefill(seed, lengths, heads=3, init_state_std=0.02).to(dev)
         T, H, d = x.q.shape
         N = len(lengths)
+        # the allocation-free entry point has only a small fixed scratch, so it
+        # runs the fused kernel; give kda_chunk_fwd the minimum workspace too
+        ws = torch.zeros(kda.kda_chunk_fwd_workspace_size_min(N, T, H), dtype=torch.uint8, device=dev)
         o_ref, s_ref = kda.kda_chunk_fwd(x.q, x.k, x.v, x.g, x.beta, x.cu_seqlens,
-                                         initial_state=x.initial_state)
+                                         initial_state=x.initial_state, workspace=ws)
         o = torch.full_like(o_ref, float("nan"))
         s = torch.full_like(s_ref, float("nan"))
         st = fn(_p(x.q), _p(x.k), _p(x.v), _p(x.g), _p(x.beta), _p(x.cu_seqlens), N, T, H, d,
