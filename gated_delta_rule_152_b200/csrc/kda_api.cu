@@ -82,9 +82,15 @@ int chunk_fwd_impl(const void* q, const void* k, const void* v, const float* g, 
     // else the fused single kernel (same arithmetic, no scratch)
     const bool two_pass =
         !recurrent && workspace_bytes >= kWorkspaceHeader + kda::two_pass_scratch_bytes(N, total_T, H);
-    const cudaError_t e = recurrent  ? kda::launch_recurrent(a, s)
-                          : two_pass ? kda::launch_chunk_two_pass(a, static_cast<uint8_t*>(workspace) + kWorkspaceHeader, s)
-                                     : kda::launch_chunk(a, s);
+    cudaError_t e;
+    if (recurrent) {
+        e = kda::launch_recurrent(a, s);
+    } else {
+        e = two_pass ? kda::launch_chunk_two_pass(a, static_cast<uint8_t*>(workspace) + kWorkspaceHeader, s)
+                     : cudaErrorNotSupported;
+        // not enough room for the two-pass path on this device: the fused kernel
+        if (e == cudaErrorNotSupported) e = kda::launch_chunk(a, s);
+    }
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

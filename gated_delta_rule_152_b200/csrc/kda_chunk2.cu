@@ -63,13 +63,16 @@ __device__ __forceinline__ bool seq_bounds(const int32_t* cu, int n, int64_t tot
 // no chunks and sets error bit 1.  Sequences that are each in bounds but
 // overlap (cu_seqlens not non-decreasing) can add up to more chunks than the
 // scratch holds (max_total): that also sets error bit 1, and both passes
-// skip every chunk at or past max_total.  One block.
+// skip every chunk at or past max_total.  Also clears the ring flags of the
+// overlapped mode.  One block.
 __global__ void __launch_bounds__(1024) kda_chunk_index_kernel(const int32_t* __restrict__ cu, int N,
                                                                int64_t total_T, int64_t max_total,
-                                                               int32_t* __restrict__ chunk_off, uint32_t* err) {
+                                                               int32_t* __restrict__ chunk_off, uint32_t* err,
+                                                               int32_t* __restrict__ zero, int nzero) {
     __shared__ int32_t wsum[32];
     __shared__ int32_t carry_s;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int i = tid; i < nzero; i += 1024) zero[i] = 0;   // ring flags of the overlapped mode
     if (tid == 0) carry_s = 0;
     __syncthreads();
     for (int base = 0; base < N; base += 1024) {
@@ -135,12 +138,28 @@ constexpr uint32_t TP_U = 128;    // 64 cols: U^T (lane = value column, column =
 constexpr uint32_t TP_COLS = 256;
 constexpr uint32_t ID_N64 = idesc_tf32(128, 64, false, false);
 
-__global__ void __launch_bounds__(kThreads, 1)
-kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ g,
-                      const float* __restrict__ beta, const int32_t* __restrict__ cu,
-                      const int32_t* __restrict__ chunk_off, int N, int H, int64_t max_total, float scale,
-                      int l2norm, int scalar_g, uint8_t* __restrict__ img, uint32_t* err) {
+// Overlapped mode (one sequence): the prep role writes each (chunk, head)
+// image into a ring of kRing slots per head instead of its own place in the
+// scratch, and the two roles hand slots over through flags in global memory:
+//   ready[h * kRing + s] = c + 1 once chunk c's image sits complete in slot s,
+//   done[h]              = number of chunks of head h the state role has read.
+// A slot is rewritten only after its previous chunk was read, so the ring
+// (kRing x H x IMG_BYTES, 37 MB for 32 heads) stays in L2.
+constexpr int kRing = 8;
+struct Ring {
+    int32_t* ready;
+    int32_t* done;
+};
+
+// Pass 1 for the work items first, first + stride, ... (item w = chunk w / H
+// of head w % H, in the global chunk order of chunk_off).
+template <bool RING>
+__device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                                          const float* __restrict__ g, const float* __restrict__ beta,
+                                          const int32_t* __restrict__ cu, const int32_t* __restrict__ chunk_off,
+                                          int N, int H, int64_t max_total, float scale, int l2norm, int scalar_g,
+                                          uint8_t* __restrict__ img, uint32_t* err, int64_t first, int64_t stride,
+                                          Ring ring) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(smem);
@@ -154,7 +173,7 @@ kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     const int quarter = warp & 3, half = warp >> 2;
     const int64_t total = chunk_off[N];
     const int64_t items = (total < max_total ? total : max_total) * H;
-    if (static_cast<int64_t>(blockIdx.x) >= items) return;
+    if (first >= items) return;
 
     if (warp == 0) {
         tmem_alloc(tmem_slot, TP_COLS);
@@ -164,9 +183,9 @@ kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         mbar_init(bar_load, 1);
         mbar_init(bar_mma, 1);
         fence_mbar_init();
-        prefetch_tmap(&tm_q);
-        prefetch_tmap(&tm_k);
-        prefetch_tmap(&tm_v);
+        prefetch_tmap(tm_q);
+        prefetch_tmap(tm_k);
+        prefetch_tmap(tm_v);
     }
     tc_fence_before();
     __syncthreads();
@@ -177,7 +196,7 @@ kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     // one whose first chunk is <= gc (sequences without chunks are skipped)
     struct Item {
         int64_t t0, gc;
-        int L, h;
+        int L, h, c;   // c: chunk index inside its sequence
     };
     auto decode = [&](int64_t w) {
         Item it;
@@ -189,10 +208,30 @@ kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             if (chunk_off[mid] <= it.gc) lo = mid;
             else hi = mid;
         }
-        it.t0 = cu[lo] + (it.gc - chunk_off[lo]) * kC;
+        it.c = static_cast<int>(it.gc - chunk_off[lo]);
+        it.t0 = cu[lo] + static_cast<int64_t>(it.c) * kC;
         const int64_t rem = cu[lo + 1] - it.t0;
         it.L = static_cast<int>(rem < kC ? rem : (int64_t)kC);
         return it;
+    };
+    // the item's image: its own place in the scratch, or its head's ring slot
+    auto image_of = [&](const Item& it) {
+        const size_t slot = RING ? static_cast<size_t>(it.h) * kRing + (it.c & (kRing - 1))
+                                 : static_cast<size_t>(it.gc) * H + it.h;
+        return img + slot * IMG_BYTES;
+    };
+    // ring mode: the image of the previous item is announced once its bulk
+    // stores have completed (checked when the store thread next issues stores)
+    int32_t* pub_flag = nullptr;
+    int32_t pub_val = 0;
+    auto publish = [&]() {
+        if (RING && pub_flag) {
+            bulk_wait_all();
+            fence_proxy_async_global();
+            __threadfence();
+            st_release_gpu(pub_flag, pub_val);
+            pub_flag = nullptr;
+        }
     };
     float greg[8][4];
     float breg;
@@ -217,9 +256,9 @@ kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     auto issue_load = [&](const Item& it) {
         mbar_arrive_expect_tx(bar_load, 3u * kC * kD * 2u);
         const int32_t t0 = static_cast<int32_t>(it.t0);
-        tma_load_3d(smem + P_KB, &tm_q, bar_load, 0, it.h, t0);
-        tma_load_3d(smem + P_KB + kC * kD * 2, &tm_k, bar_load, 0, it.h, t0);
-        tma_load_3d(smem + P_RV, &tm_v, bar_load, 0, it.h, t0);
+        tma_load_3d(smem + P_KB, tm_q, bar_load, 0, it.h, t0);
+        tma_load_3d(smem + P_KB + kC * kD * 2, tm_k, bar_load, 0, it.h, t0);
+        tma_load_3d(smem + P_RV, tm_v, bar_load, 0, it.h, t0);
     };
 
     bool ok = true;
@@ -235,20 +274,29 @@ kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         return good;
     };
 
-    int64_t w = blockIdx.x;
+    int64_t w = first;
     Item cur = decode(w);
     if (tid == 0) issue_load(cur);
     load_pending = true;
     prefetch(cur);
 
-    for (; ok && w < items; w += gridDim.x) {
-        const int64_t wn = w + gridDim.x;
+    for (; ok && w < items; w += stride) {
+        const int64_t wn = w + stride;
         const bool has_next = wn < items;
         const Item nxt = has_next ? decode(wn) : cur;
-        uint8_t* im = img + (static_cast<size_t>(cur.gc) * H + cur.h) * IMG_BYTES;
+        uint8_t* im = image_of(cur);
         const int L = cur.L;
 
-        if (!(ok = !__syncthreads_or(!mbar_wait_bounded(bar_load, load_parity)))) break;
+        // ring mode: the slot must have been read by the state role first.  A
+        // producer never blocks on it while holding an unannounced image (the
+        // state role that it waits for may need exactly that image).
+        bool slot_free = true;
+        if (RING && tid == kStoreThread && cur.c >= kRing &&
+            ld_acquire_gpu(ring.done + cur.h) < cur.c - kRing + 1) {
+            publish();
+            slot_free = wait_flag_ge(ring.done + cur.h, cur.c - kRing + 1);
+        }
+        if (!(ok = !__syncthreads_or(!mbar_wait_bounded(bar_load, load_parity) || !slot_free))) break;
         load_pending = false;
         load_parity ^= 1;
 
@@ -308,6 +356,7 @@ kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         tc_fence_before();
         __syncthreads();
         if (tid == kStoreThread) {   // Kb^T -> image rows 0-127 of [Kb^T ; P]; Qt -> rows 0-63 of [Qt ; W]
+            publish();
 #pragma unroll
             for (int kb = 0; kb < 2; ++kb)
                 bulk_store(im + IMG_B2 + kb * KB_B2, smem + P_KBTS + kb * P_KB_T, P_KB_T);
@@ -440,11 +489,18 @@ kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             bulk_store(im + IMG_U, smem + P_X + 32768, 32768);
             bulk_commit();
             bulk_wait_read();   // the next item's prep rewrites X
+            if (RING) {
+                pub_flag = ring.ready + cur.h * kRing + (cur.c & (kRing - 1));
+                pub_val = cur.c + 1;
+            }
         }
         cur = nxt;
     }
 
-    if (tid == kStoreThread) bulk_wait_all();
+    if (tid == kStoreThread) {
+        if (ok) publish();
+        bulk_wait_all();
+    }
     tc_fence_before();
     __syncthreads();
     if (!ok && tid == 0) {
@@ -462,27 +518,33 @@ kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 // ============================================================ pass 2
 constexpr uint32_t S_B1 = 0;          // 64 KB [Qt ; W] of the current chunk
 constexpr uint32_t S_DC = 65536;      // exp(Gamma_C), copied with [Qt ; W]
-constexpr uint32_t S_B2 = 66560;      // 48 KB [Kb^T ; P]
-constexpr uint32_t S_SA = 115712;     // 64 KB St^T: 128 value rows x 128 channels, 4 K-blocks x 16 KB
-constexpr uint32_t S_DT = 181248;     // 32 KB delta^T: 128 value rows x 64 tokens, 2 K-blocks x 16 KB
-constexpr uint32_t S_MISC = 214016;   // barriers, TMEM slot
+constexpr uint32_t S_B2 = 66560;      // 48 KB [Kb^T ; P], then
+constexpr uint32_t S_U = 115712;      //   32 KB U ([token][value] fp32), copied together
+constexpr uint32_t S_DT = 148480;     // 32 KB delta^T: 128 value rows x 64 tokens, 2 K-blocks x 16 KB
+constexpr uint32_t S_MISC = 181248;   // barriers, TMEM slot
 constexpr uint32_t S_SMEM = S_MISC + 1024 + 1024;
-static_assert(S_DC == S_B1 + IMG_DC && S_B2 % 1024 == 0 && S_SA % 1024 == 0 && S_DT % 1024 == 0, "layout");
+constexpr uint32_t B2U_COPY = B2_COPY + 32768;
+static_assert(S_DC == S_B1 + IMG_DC && S_B2 % 1024 == 0 && S_U == S_B2 + B2_COPY && S_DT % 1024 == 0 &&
+              IMG_U == IMG_B2 + B2_COPY, "layout");
 
-constexpr uint32_t TS_S = 0;      // 128 cols: S^T (lane = value column, column = key channel)
+constexpr uint32_t TS_S = 0;      // 128 cols: S^T fp32 (lane = value column, column = key channel)
 constexpr uint32_t TS_Z = 128;    // 64 cols: Z^T, then O^T (column = token)
 constexpr uint32_t TS_Y = 192;    // 64 cols: Y^T
-constexpr uint32_t TS_COLS = 256;
+constexpr uint32_t TS_A = 256;    // 128 cols: St^T rounded to tf32, the A operand of the first product
+constexpr uint32_t TS_COLS = 512;
 constexpr uint32_t ID_N128 = idesc_tf32(128, 128, false, false);
 constexpr uint32_t ID_N192 = idesc_tf32(128, 192, false, false);
-constexpr int kOutThread = 32;   // issues the O stores and the L2 prefetches (not the MMA thread)
+constexpr int kOutThread = 128;   // issues the O stores, the L2 prefetches and the ring hand-back
+                                  // (first thread of the O warps; not the MMA thread)
+constexpr bool kStageO = true;    // O leaves through shared memory and one TMA store per chunk
 
-__global__ void __launch_bounds__(kThreads, 1)
-kda_chunk_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t* __restrict__ img,
-                       const int32_t* __restrict__ chunk_off,
-                       const int32_t* __restrict__ cu, int64_t total_T, int H, int64_t max_total,
-                       const float* s0, float* sT,
-                       float* __restrict__ o, uint32_t* err, const int32_t* __restrict__ slots, int num_slots) {
+// Pass 2 for sequence n, head h.
+template <bool RING>
+__device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_t* __restrict__ img,
+                                           const int32_t* __restrict__ chunk_off, const int32_t* __restrict__ cu,
+                                           int64_t total_T, int H, int64_t max_total, const float* s0, float* sT,
+                                           float* __restrict__ o, uint32_t* err, const int32_t* __restrict__ slots,
+                                           int num_slots, int n, int h, Ring ring) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(smem);
@@ -492,8 +554,6 @@ kda_chunk_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t* 
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_b1 + 3);
     const float* dc_s = reinterpret_cast<const float*>(smem + S_DC);
 
-    const int h = blockIdx.x % H;
-    const int n = blockIdx.x / H;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quarter = warp & 3, half = warp >> 2;
     const int e = 32 * quarter + lane;   // value column of this thread's TMEM lane
@@ -508,7 +568,19 @@ kda_chunk_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t* 
     const int nch = static_cast<int>((eos - bos + kC - 1) / kC);
     const int64_t gc0 = chunk_off[n];
     if (gc0 + nch > max_total) return;   // overlapping sequences overflowed the scratch: flagged above
-    auto image = [&](int c) { return img + (static_cast<size_t>(gc0 + c) * H + h) * IMG_BYTES; };
+    auto image = [&](int c) {
+        const size_t slot = RING ? static_cast<size_t>(h) * kRing + (c & (kRing - 1))
+                                 : static_cast<size_t>(gc0 + c) * H + h;
+        return img + slot * IMG_BYTES;
+    };
+    // ring mode: chunk c's image must be complete before its first copy is issued
+    auto await_image = [&](int c) -> bool {
+        if (!RING) return true;
+        const bool good = wait_flag_ge(ring.ready + h * kRing + (c & (kRing - 1)), c + 1);
+        fence_proxy_async_global();
+        return good;
+    };
+    bool img_ok = true;   // thread 0: the image wait did not give up (checked at the next barrier)
 
     if (warp == 0) {
         tmem_alloc(tmem_slot, TS_COLS);
@@ -545,44 +617,48 @@ kda_chunk_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t* 
         for (int p = 0; p < 4; ++p) bulk_load(smem + S_B1 + p * 16384, src + p * 16384, 16384, bar_b1);
         bulk_load(smem + S_DC, src + IMG_DC, 512, bar_b1);
     };
-    auto load_b2 = [&](int c) {
-        mbar_arrive_expect_tx(bar_b2, B2_COPY);
+    auto load_b2 = [&](int c) {   // [Kb^T ; P] and U
+        mbar_arrive_expect_tx(bar_b2, B2U_COPY);
         const uint8_t* src = image(c) + IMG_B2;
 #pragma unroll
-        for (int p = 0; p < 3; ++p) bulk_load(smem + S_B2 + p * 16384, src + p * 16384, 16384, bar_b2);
+        for (int p = 0; p < 5; ++p) bulk_load(smem + S_B2 + p * 16384, src + p * 16384, 16384, bar_b2);
     };
-    if (tid == 0 && nch > 0) {
+    if (tid == 0 && nch > 0 && (img_ok = await_image(0))) {
         load_b1(0);
         load_b2(0);
     }
     // in-flight copies: pending flag and the chunk they belong to (its parity)
-    bool b1_pending = nch > 0, b2_pending = nch > 0, mma_pending = false, ok = true;
+    bool ok = !__syncthreads_or(!img_ok);
+    bool b1_pending = ok && nch > 0, b2_pending = ok && nch > 0, mma_pending = false;
     int b1_chunk = 0, b2_chunk = 0;
     uint32_t mma_phase = 0;
     auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
         return !__syncthreads_or(!mbar_wait_bounded(bar, parity));
     };
-    // O^T of the chunk at t0 (lanes = value column, columns = tokens 32*half ..):
-    // into the DT tile as [token][value] for one TMA store by kOutThread
-    // (staged, full chunks; DT is free between the second product of one
-    // chunk and the delta of the next), else straight to o
+    // O^T of the chunk at t0 (lane = value column, columns = its 64 tokens), read
+    // by the warps of one half: into the DT tile as [token][value] (staged; DT
+    // is free between the second product of one chunk and the delta of the
+    // next), else straight to o
     auto emit_o = [&](int64_t t0, int L, bool staged) {
-        float acc[32];
-        tmem_ld32(tm_lane(tmem, quarter, TS_Z + 32 * half), acc);
-        tmem_wait_ld();
-        if (staged) {
-            float* dst = reinterpret_cast<float*>(smem + S_DT) + (32 * half) * kD + e;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) dst[j * kD] = acc[j];
-        } else {
+        for (int part = 0; part < 2; ++part) {
+            float acc[32];
+            tmem_ld32(tm_lane(tmem, quarter, TS_Z + 32 * part), acc);
+            tmem_wait_ld();
+            if (staged) {
+                float* dst = reinterpret_cast<float*>(smem + S_DT) + (32 * part) * kD + e;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int r = 32 * half + j;
-                if (r < L) o[((size_t)(t0 + r) * H + h) * kD + e] = acc[j];
+                for (int j = 0; j < 32; ++j) dst[j * kD] = acc[j];
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int r = 32 * part + j;
+                    if (r < L) o[((size_t)(t0 + r) * H + h) * kD + e] = acc[j];
+                }
             }
         }
     };
-    if (tid == kOutThread && nch > 1) prefetch_l2(image(1), IMG_BYTES);
+    if (!RING && tid == kOutThread && nch > 1) prefetch_l2(image(1), IMG_BYTES);
 
     int64_t t_prev = bos;
     int L_prev = 0;
@@ -591,8 +667,9 @@ kda_chunk_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t* 
         const int L = static_cast<int>(eos - t0 < kC ? eos - t0 : (int64_t)kC);
         const uint8_t* im = image(c);
 
-        // ---- the state of the chunk start is in TMEM: O of the previous chunk out,
-        // the state decayed to this chunk's end as the A operand
+        // ---- the state of the chunk start is in TMEM: warps 4-7 read O of the
+        // previous chunk out while warps 0-3 decay the state to this chunk's end
+        // (back into TMEM, and as the A operand)
         bool o_tma = false;
         if (c > 0) {
             if (!(ok = wait_all(bar_mma, mma_phase))) break;
@@ -603,70 +680,80 @@ kda_chunk_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t* 
             b2_pending = true;
             b2_chunk = c;
             o_tma = L_prev == kC;
-            emit_o(t_prev, L_prev, o_tma);
         }
-        if (tid == kOutThread && c + 2 < nch) prefetch_l2(image(c + 2), IMG_BYTES);
-        float u[32];   // U of this thread's value column, tokens 32*half .. (one 128-byte row per warp load)
-        {
-            const float* src = reinterpret_cast<const float*>(im + IMG_U) + (32 * half) * kD + e;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) u[j] = src[j * kD];
+        if (!RING && tid == kOutThread && c + 2 < nch) prefetch_l2(image(c + 2), IMG_BYTES);
+        // warps 4-7: O of the previous chunk out; a full chunk's tile leaves by
+        // one TMA store as soon as those four warps have written it
+        if (half == 1 && c > 0) {
+            emit_o(t_prev, L_prev, kStageO && o_tma);
+            if (kStageO && o_tma) {
+                fence_proxy_async_smem();
+                named_barrier(1, 128);
+                if (tid == kOutThread) {
+                    tma_store_3d(tm_o, smem + S_DT, 0, h, static_cast<int32_t>(t_prev));
+                    bulk_commit();
+                }
+            }
         }
-        if (!(ok = wait_all(bar_b1, c & 1))) break;
-        b1_pending = false;
-        float st[2][32];   // St^T of this lane, key channels 64*half ..
+        // all warps: the state decayed to this chunk's end (key channels
+        // 64*half ..): fp32 back into TMEM, and rounded to tf32 into the
+        // A-operand columns; it needs exp(Gamma_C), which comes with [Qt ; W]
+        const bool b1_ok = mbar_wait_bounded(bar_b1, c & 1);
+        if (b1_ok) {
+            float st[2][32];
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {
-            const int c0 = 64 * half + 32 * part;
-            tmem_ld32(tm_lane(tmem, quarter, TS_S + c0), st[part]);
+            for (int part = 0; part < 2; ++part) tmem_ld32(tm_lane(tmem, quarter, TS_S + 64 * half + 32 * part), st[part]);
             tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const float4 d4 = *reinterpret_cast<const float4*>(dc_s + c0 + 4 * j);
-                st[part][4 * j] *= d4.x; st[part][4 * j + 1] *= d4.y;
-                st[part][4 * j + 2] *= d4.z; st[part][4 * j + 3] *= d4.w;
-            }
+            for (int part = 0; part < 2; ++part) {
+                const int c0 = 64 * half + 32 * part;
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-                *reinterpret_cast<float4*>(K_at(smem, S_SA, 16384, e, c0 + 4 * j)) =
-                    tf32x4(st[part][4 * j], st[part][4 * j + 1], st[part][4 * j + 2], st[part][4 * j + 3]);
+                for (int j = 0; j < 8; ++j) {
+                    const float4 d4 = *reinterpret_cast<const float4*>(dc_s + c0 + 4 * j);
+                    st[part][4 * j] *= d4.x; st[part][4 * j + 1] *= d4.y;
+                    st[part][4 * j + 2] *= d4.z; st[part][4 * j + 3] *= d4.w;
+                }
+                tmem_st32(tm_lane(tmem, quarter, TS_S + c0), st[part]);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) st[part][j] = to_tf32(st[part][j]);
+                tmem_st32(tm_lane(tmem, quarter, TS_A + c0), st[part]);
+            }
+            tmem_wait_st();
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        __syncthreads();
+        if (!(ok = !__syncthreads_or(!b1_ok))) break;
+        b1_pending = false;
 
-        // ---- [Z^T | Y^T] = St^T [Qt ; W]^T; meanwhile O of the previous chunk
-        // leaves by TMA and St goes back to TMEM (the second product accumulates onto it)
+        // ---- [Z^T | Y^T] = St^T [Qt ; W]^T; meanwhile O of the previous chunk leaves by TMA
         if (tid == 0) {
             tc_fence_after();
-            const uint64_t da = tdesc(sb, S_SA), db = tdesc(sb, S_B1);
+            const uint64_t db = tdesc(sb, S_B1);
 #pragma unroll
             for (int s = 0; s < 16; ++s)
-                mma_tf32_ss(tmem + TS_Z, kstep(da, 16384, s), kstep(db, KB_B1, s), ID_N128, s > 0);
+                mma_tf32_ts(tmem + TS_Z, tmem + TS_A + 8 * s, kstep(db, KB_B1, s), ID_N128, s > 0);
             mma_commit(bar_mma);
         }
         mma_pending = true;
-        if (tid == kOutThread && o_tma) {
-            tma_store_3d(&tm_o, smem + S_DT, 0, h, static_cast<int32_t>(t_prev));
-            bulk_commit();
-        }
-#pragma unroll
-        for (int part = 0; part < 2; ++part)
-            tmem_st32(tm_lane(tmem, quarter, TS_S + 64 * half + 32 * part), st[part]);
-        tmem_wait_st();
-        if (tid == kOutThread) bulk_wait_read();   // DT is written again below
+        if (kStageO && tid == kOutThread) bulk_wait_read();   // DT is written again below
         if (!(ok = wait_all(bar_mma, mma_phase))) break;
         mma_phase ^= 1;
         mma_pending = false;
         tc_fence_after();
-        if (tid == 0 && c + 1 < nch) load_b1(c + 1);
+        if (tid == 0 && c + 1 < nch && (img_ok = await_image(c + 1))) load_b1(c + 1);
         b1_pending = c + 1 < nch;
         b1_chunk = c + 1;
 
-        // ---- delta^T = U^T - Y^T (tf32 operand, row = value column, K = token)
-        {
+        // ---- delta^T = U^T - Y^T (tf32 operand, row = value column, K = token);
+        // U came with [Kb^T ; P]
+        const bool b2_ok = mbar_wait_bounded(bar_b2, c & 1);
+        if (b2_ok) {
             float y[32];
             tmem_ld32(tm_lane(tmem, quarter, TS_Y + 32 * half), y);
+            const float* us = reinterpret_cast<const float*>(smem + S_U) + (32 * half) * kD + e;
+            float u[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) u[j] = us[j * kD];
             tmem_wait_ld();
 #pragma unroll
             for (int j = 0; j < 8; ++j)
@@ -674,11 +761,16 @@ kda_chunk_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t* 
                     tf32x4(u[4 * j] - y[4 * j], u[4 * j + 1] - y[4 * j + 1], u[4 * j + 2] - y[4 * j + 2],
                            u[4 * j + 3] - y[4 * j + 3]);
         }
-        if (!(ok = wait_all(bar_b2, c & 1))) break;
-        b2_pending = false;
         fence_proxy_async_smem();
         tc_fence_before();
-        __syncthreads();
+        if (!(ok = !__syncthreads_or(!b2_ok || !img_ok))) {
+            b1_pending = b1_pending && img_ok;
+            break;
+        }
+        b2_pending = false;
+        // chunk c's slot is read: both copies have landed (their mbarriers
+        // completed), so the slot can be handed back with a plain store
+        if (RING && tid == kOutThread) st_relaxed_gpu(ring.done + h, c + 1);
 
         // ---- [S^T | O^T] += delta^T [Kb^T ; P]^T
         if (tid == 0) {
@@ -697,7 +789,7 @@ kda_chunk_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t* 
         if ((ok = wait_all(bar_mma, mma_phase))) {
             mma_pending = false;
             tc_fence_after();
-            emit_o(t_prev, L_prev, false);
+            if (half == 1) emit_o(t_prev, L_prev, false);
         }
     }
     if (ok) {
@@ -729,6 +821,44 @@ kda_chunk_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t* 
     }
 }
 
+__global__ void __launch_bounds__(kThreads, 1)
+kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ g,
+                      const float* __restrict__ beta, const int32_t* __restrict__ cu,
+                      const int32_t* __restrict__ chunk_off, int N, int H, int64_t max_total, float scale,
+                      int l2norm, int scalar_g, uint8_t* __restrict__ img, uint32_t* err) {
+    prep_role<false>(&tm_q, &tm_k, &tm_v, g, beta, cu, chunk_off, N, H, max_total, scale, l2norm, scalar_g, img,
+                     err, blockIdx.x, gridDim.x, Ring{nullptr, nullptr});
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+kda_chunk_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t* __restrict__ img,
+                       const int32_t* __restrict__ chunk_off, const int32_t* __restrict__ cu, int64_t total_T, int H,
+                       int64_t max_total, const float* s0, float* sT, float* __restrict__ o, uint32_t* err,
+                       const int32_t* __restrict__ slots, int num_slots) {
+    state_role<false>(&tm_o, img, chunk_off, cu, total_T, H, max_total, s0, sT, o, err, slots, num_slots,
+                      blockIdx.x / H, blockIdx.x % H, Ring{nullptr, nullptr});
+}
+
+// One sequence, both passes in one cooperative launch (all CTAs resident):
+// CTAs 0 .. H-1 carry the states of the H heads, the others prepare chunks
+// ahead of them through the ring.
+__global__ void __launch_bounds__(kThreads, 1)
+kda_chunk_overlap_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                         const float* __restrict__ g, const float* __restrict__ beta, const int32_t* __restrict__ cu,
+                         const int32_t* __restrict__ chunk_off, int H, int64_t total_T, int64_t max_total,
+                         float scale, int l2norm, int scalar_g, uint8_t* __restrict__ img, const float* s0,
+                         float* sT, float* __restrict__ o, uint32_t* err, const int32_t* __restrict__ slots,
+                         int num_slots, Ring ring) {
+    if (static_cast<int>(blockIdx.x) < H)
+        state_role<true>(&tm_o, img, chunk_off, cu, total_T, H, max_total, s0, sT, o, err, slots, num_slots, 0,
+                         blockIdx.x, ring);
+    else
+        prep_role<true>(&tm_q, &tm_k, &tm_v, g, beta, cu, chunk_off, 1, H, max_total, scale, l2norm, scalar_g, img,
+                        err, blockIdx.x - H, gridDim.x - H, ring);
+}
+
 int num_sms() {
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -738,24 +868,36 @@ int num_sms() {
 size_t max_chunks(int32_t N, int64_t total_T) { return static_cast<size_t>((total_T + 63 * (int64_t)N) / kC); }
 size_t index_bytes(int32_t N) { return (static_cast<size_t>(N + 1) * 4 + 1023) & ~size_t(1023); }
 
+// Overlapped mode: one sequence, and enough SMs left for the prep role.
+constexpr int kMinPrepCtas = 16;
+constexpr int kMaxRingHeads = 96;
+bool ring_eligible(int32_t N, int32_t H) { return N == 1 && H <= kMaxRingHeads; }
+size_t ring_flag_bytes(int32_t H) { return (static_cast<size_t>(H) * (kRing + 1) * 4 + 1023) & ~size_t(1023); }
+
+template <class K>
+cudaError_t set_smem(K kernel, uint32_t bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+}
+
 }  // namespace
 
 size_t two_pass_scratch_bytes(int32_t N, int64_t total_T, int32_t H) {
     if (N < 0 || total_T < 0 || H <= 0) return 0;
+    if (ring_eligible(N, H))
+        return index_bytes(N) + ring_flag_bytes(H) + static_cast<size_t>(H) * kRing * IMG_BYTES;
     return index_bytes(N) + max_chunks(N, total_T) * static_cast<size_t>(H) * IMG_BYTES;
 }
 
 cudaError_t launch_chunk_two_pass(const PrefillArgs& a, void* scratch, cudaStream_t stream) {
     if (a.N == 0 || a.H == 0) return cudaSuccess;
     if (a.total_T <= 0) return cudaErrorInvalidValue;   // callers route empty batches elsewhere
+    constexpr uint32_t O_SMEM = P_SMEM > S_SMEM ? P_SMEM : S_SMEM;
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(kda_chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        static_cast<int>(P_SMEM));
-        if (attr_err == cudaSuccess)
-            attr_err = cudaFuncSetAttribute(kda_chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            static_cast<int>(S_SMEM));
+        attr_err = set_smem(kda_chunk_prep_kernel, P_SMEM);
+        if (attr_err == cudaSuccess) attr_err = set_smem(kda_chunk_state_kernel, S_SMEM);
+        if (attr_err == cudaSuccess) attr_err = set_smem(kda_chunk_overlap_kernel, O_SMEM);
     });
     if (attr_err != cudaSuccess) return attr_err;
     CUtensorMap mq, mk, mv, mo;
@@ -763,20 +905,54 @@ cudaError_t launch_chunk_two_pass(const PrefillArgs& a, void* scratch, cudaStrea
         !make_token_map(&mv, a.v, a.total_T, a.H) || !make_token_map(&mo, a.o, a.total_T, a.H, true))
         return cudaErrorInvalidValue;
     int32_t* chunk_off = static_cast<int32_t*>(scratch);
-    uint8_t* img = static_cast<uint8_t*>(scratch) + index_bytes(a.N);
-
     const int64_t max_total = static_cast<int64_t>(max_chunks(a.N, a.total_T));
-    kda_chunk_index_kernel<<<1, 1024, 0, stream>>>(a.cu_seqlens, a.N, a.total_T, max_total, chunk_off, a.err);
+    const int sms = num_sms();
+
+    if (ring_eligible(a.N, a.H)) {
+        // both passes in one cooperative launch: H state CTAs + the rest preparing
+        int dev = 0, coop = 0, per_sm = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kda_chunk_overlap_kernel, kThreads, O_SMEM) !=
+                cudaSuccess)
+            return cudaGetLastError();
+        if (!coop || per_sm < 1 || a.H + kMinPrepCtas > sms) return cudaErrorNotSupported;
+        uint8_t* flags = static_cast<uint8_t*>(scratch) + index_bytes(a.N);
+        Ring ring{reinterpret_cast<int32_t*>(flags), reinterpret_cast<int32_t*>(flags) + a.H * kRing};
+        uint8_t* img = flags + ring_flag_bytes(a.H);
+        kda_chunk_index_kernel<<<1, 1024, 0, stream>>>(a.cu_seqlens, a.N, a.total_T, max_total, chunk_off, a.err,
+                                                       ring.ready, a.H * (kRing + 1));
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(sms));
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = O_SMEM;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        const cudaError_t e = cudaLaunchKernelEx(
+            &cfg, kda_chunk_overlap_kernel, mq, mk, mv, mo, a.g, a.beta, a.cu_seqlens,
+            static_cast<const int32_t*>(chunk_off), static_cast<int>(a.H), a.total_T, max_total, a.scale,
+            a.l2norm ? 1 : 0, a.scalar_decay ? 1 : 0, img, a.initial_state, a.final_state, a.o, a.err, a.slots,
+            static_cast<int>(a.num_slots), ring);
+        return e != cudaSuccess ? e : cudaGetLastError();
+    }
+
+    uint8_t* img = static_cast<uint8_t*>(scratch) + index_bytes(a.N);
+    kda_chunk_index_kernel<<<1, 1024, 0, stream>>>(a.cu_seqlens, a.N, a.total_T, max_total, chunk_off, a.err,
+                                                   nullptr, 0);
     const size_t items_ub = max_chunks(a.N, a.total_T) * static_cast<size_t>(a.H);
-    const size_t grid1 = items_ub < static_cast<size_t>(num_sms()) ? items_ub : static_cast<size_t>(num_sms());
+    const size_t grid1 = items_ub < static_cast<size_t>(sms) ? items_ub : static_cast<size_t>(sms);
     if (grid1 > 0)
         kda_chunk_prep_kernel<<<static_cast<unsigned>(grid1), kThreads, P_SMEM, stream>>>(
             mq, mk, mv, a.g, a.beta, a.cu_seqlens, chunk_off, a.N, a.H, max_total, a.scale, a.l2norm ? 1 : 0,
             a.scalar_decay ? 1 : 0, img, a.err);
     const long long blocks = (long long)a.N * a.H;
     kda_chunk_state_kernel<<<static_cast<unsigned>(blocks), kThreads, S_SMEM, stream>>>(
-        mo, img, chunk_off, a.cu_seqlens, a.total_T, a.H, max_total, a.initial_state, a.final_state, a.o, a.err, a.slots,
-        a.num_slots);
+        mo, img, chunk_off, a.cu_seqlens, a.total_T, a.H, max_total, a.initial_state, a.final_state, a.o, a.err,
+        a.slots, a.num_slots);
     return cudaGetLastError();
 }
 

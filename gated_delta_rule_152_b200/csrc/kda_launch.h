@@ -38,8 +38,11 @@ cudaError_t launch_chunk(const PrefillArgs& a, cudaStream_t stream);
 
 // Two-pass chunked prefill: a parallel pass over (chunk, head) that writes
 // each chunk's state-independent operands to scratch, then a sequential pass
-// per (sequence, head) that carries the state.  `scratch` (16-byte aligned)
-// must hold two_pass_scratch_bytes(N, total_T, H) bytes.
+// per (sequence, head) that carries the state; for a single sequence both
+// passes run overlapped in one cooperative launch through a ring of operand
+// slots.  `scratch` (16-byte aligned) must hold two_pass_scratch_bytes(N,
+// total_T, H) bytes.  Returns cudaErrorNotSupported, having launched nothing,
+// when the device cannot host the overlapped launch.
 size_t two_pass_scratch_bytes(int32_t N, int64_t total_T, int32_t H);
 cudaError_t launch_chunk_two_pass(const PrefillArgs& a, void* scratch, cudaStream_t stream);
 

@@ -27,6 +27,11 @@ __device__ __forceinline__ void st_tf32x4(uint8_t* smem, uint32_t off, float a, 
     *reinterpret_cast<float4*>(smem + off) = tf32x4(a, b, c, d);
 }
 
+// Barrier over a subset of the block's warps (ids 1..15; id 0 is __syncthreads).
+__device__ __forceinline__ void named_barrier(uint32_t id, uint32_t threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 // TMEM address of lane quarter `quarter` (lanes 32*quarter ..), column `col`.
 __device__ __forceinline__ uint32_t tm_lane(uint32_t tmem, int quarter, uint32_t col) {
     return tmem + (static_cast<uint32_t>(32 * quarter) << 16) + col;
