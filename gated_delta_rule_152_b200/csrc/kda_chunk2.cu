@@ -521,24 +521,31 @@ constexpr uint32_t S_DC = 65536;      // exp(Gamma_C), copied with [Qt ; W]
 constexpr uint32_t S_B2 = 66560;      // 48 KB [Kb^T ; P], then
 constexpr uint32_t S_U = 115712;      //   32 KB U ([token][value] fp32), copied together
 constexpr uint32_t S_DT = 148480;     // 32 KB delta^T: 128 value rows x 64 tokens, 2 K-blocks x 16 KB
-constexpr uint32_t S_MISC = 181248;   // barriers, TMEM slot
+constexpr uint32_t S_OS = 181248;     // 32 KB O of the previous chunk ([token][value] fp32), TMA store source
+constexpr uint32_t S_MISC = 214016;   // barriers, TMEM slot
 constexpr uint32_t S_SMEM = S_MISC + 1024 + 1024;
 constexpr uint32_t B2U_COPY = B2_COPY + 32768;
 static_assert(S_DC == S_B1 + IMG_DC && S_B2 % 1024 == 0 && S_U == S_B2 + B2_COPY && S_DT % 1024 == 0 &&
               IMG_U == IMG_B2 + B2_COPY, "layout");
 
 constexpr uint32_t TS_S = 0;      // 128 cols: S^T fp32 (lane = value column, column = key channel)
-constexpr uint32_t TS_Z = 128;    // 64 cols: Z^T, then O^T (column = token)
-constexpr uint32_t TS_Y = 192;    // 64 cols: Y^T
+constexpr uint32_t TS_Z = 128;    // 64 cols: Z^T, then O^T (column = token) of even chunks; Y^T follows;
+                                  //   odd chunks use the set 256 columns on (384 - 511)
 constexpr uint32_t TS_A = 256;    // 128 cols: St^T rounded to tf32, the A operand of the first product
 constexpr uint32_t TS_COLS = 512;
 constexpr uint32_t ID_N128 = idesc_tf32(128, 128, false, false);
-constexpr uint32_t ID_N192 = idesc_tf32(128, 192, false, false);
 constexpr int kOutThread = 128;   // issues the O stores, the L2 prefetches and the ring hand-back
                                   // (first thread of the O warps; not the MMA thread)
-constexpr bool kStageO = true;    // O leaves through shared memory and one TMA store per chunk
 
-// Pass 2 for sequence n, head h.
+// Pass 2 for sequence n, head h.  Per chunk c (k = c % 2 selects one of two
+// Z/Y column sets in TMEM):
+//   decay:  St = Diag(e^Gamma_C) S into TMEM (fp32) and, rounded to tf32, into
+//           the A-operand columns                                  (all warps)
+//   MMA1:   [Z_k | Y_k] = St^T [Qt ; W]^T        (A from TMEM, B = [Qt ; W])
+//           meanwhile O of chunk c-1 (set k^1) is read out and staged
+//   delta:  delta^T = U^T - Y_k^T                                  (all warps)
+//   MMA2a:  S^T += delta^T Kb   (the only product the next chunk waits for)
+//   MMA2b:  Z_k^T += delta^T P^T  = O^T of chunk c, read out during chunk c+1
 template <bool RING>
 __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_t* __restrict__ img,
                                            const int32_t* __restrict__ chunk_off, const int32_t* __restrict__ cu,
@@ -550,8 +557,9 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
     const uint32_t sb = smem_u32(smem);
     uint64_t* bar_b1 = reinterpret_cast<uint64_t*>(smem + S_MISC);
     uint64_t* bar_b2 = bar_b1 + 1;
-    uint64_t* bar_mma = bar_b1 + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_b1 + 3);
+    uint64_t* bar_mma = bar_b1 + 2;   // MMA1 and MMA2a of every chunk
+    uint64_t* bar_o = bar_b1 + 3;     // MMA2b of every chunk
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_b1 + 4);
     const float* dc_s = reinterpret_cast<const float*>(smem + S_DC);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -590,6 +598,7 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
         mbar_init(bar_b1, 1);
         mbar_init(bar_b2, 1);
         mbar_init(bar_mma, 1);
+        mbar_init(bar_o, 1);
         fence_mbar_init();
     }
     tc_fence_before();
@@ -617,87 +626,60 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
         for (int p = 0; p < 4; ++p) bulk_load(smem + S_B1 + p * 16384, src + p * 16384, 16384, bar_b1);
         bulk_load(smem + S_DC, src + IMG_DC, 512, bar_b1);
     };
-    auto load_b2 = [&](int c) {   // [Kb^T ; P] and U
+    // [Kb^T ; P] and U in two steps on one mbarrier phase (the first step
+    // registers all the bytes): Kb^T and U as soon as MMA2a of the previous
+    // chunk is done, P once MMA2b (which reads P) is done
+    auto load_b2_kbt_u = [&](int c) {
         mbar_arrive_expect_tx(bar_b2, B2U_COPY);
         const uint8_t* src = image(c) + IMG_B2;
 #pragma unroll
-        for (int p = 0; p < 5; ++p) bulk_load(smem + S_B2 + p * 16384, src + p * 16384, 16384, bar_b2);
+        for (int kb = 0; kb < 2; ++kb) bulk_load(smem + S_B2 + kb * KB_B2, src + kb * KB_B2, 128 * 128, bar_b2);
+        bulk_load(smem + S_U, src + B2_COPY, 32768, bar_b2);
+    };
+    auto load_b2_p = [&](int c) {
+        const uint8_t* src = image(c) + IMG_B2;
+#pragma unroll
+        for (int kb = 0; kb < 2; ++kb)
+            bulk_load(smem + S_B2 + kb * KB_B2 + 128 * 128, src + kb * KB_B2 + 128 * 128, 64 * 128, bar_b2);
+    };
+    auto load_b2 = [&](int c) {
+        load_b2_kbt_u(c);
+        load_b2_p(c);
     };
     if (tid == 0 && nch > 0 && (img_ok = await_image(0))) {
         load_b1(0);
         load_b2(0);
     }
-    // in-flight copies: pending flag and the chunk they belong to (its parity)
+    // in-flight copies and products: pending flag and the chunk (parity) they belong to
     bool ok = !__syncthreads_or(!img_ok);
-    bool b1_pending = ok && nch > 0, b2_pending = ok && nch > 0, mma_pending = false;
+    bool b1_pending = ok && nch > 0, b2_pending = ok && nch > 0, mma_pending = false, o_pending = false;
     int b1_chunk = 0, b2_chunk = 0;
     uint32_t mma_phase = 0;
     auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
         return !__syncthreads_or(!mbar_wait_bounded(bar, parity));
     };
-    // O^T of the chunk at t0 (lane = value column, columns = its 64 tokens), read
-    // by the warps of one half: into the DT tile as [token][value] (staged; DT
-    // is free between the second product of one chunk and the delta of the
-    // next), else straight to o
-    auto emit_o = [&](int64_t t0, int L, bool staged) {
-#pragma unroll
-        for (int part = 0; part < 2; ++part) {
-            float acc[32];
-            tmem_ld32(tm_lane(tmem, quarter, TS_Z + 32 * part), acc);
-            tmem_wait_ld();
-            if (staged) {
-                float* dst = reinterpret_cast<float*>(smem + S_DT) + (32 * part) * kD + e;
-#pragma unroll
-                for (int j = 0; j < 32; ++j) dst[j * kD] = acc[j];
-            } else {
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int r = 32 * part + j;
-                    if (r < L) o[((size_t)(t0 + r) * H + h) * kD + e] = acc[j];
-                }
-            }
-        }
-    };
+    auto zcol = [](int c) { return TS_Z + 256u * static_cast<uint32_t>(c & 1); };   // Z of chunk c; Y follows
     if (!RING && tid == kOutThread && nch > 1) prefetch_l2(image(1), IMG_BYTES);
 
     int64_t t_prev = bos;
-    int L_prev = 0;
     for (int c = 0; c < nch; ++c) {
         const int64_t t0 = bos + (int64_t)c * kC;
         const int L = static_cast<int>(eos - t0 < kC ? eos - t0 : (int64_t)kC);
-        const uint8_t* im = image(c);
 
-        // ---- the state of the chunk start is in TMEM: warps 4-7 read O of the
-        // previous chunk out while warps 0-3 decay the state to this chunk's end
-        // (back into TMEM, and as the A operand)
-        bool o_tma = false;
+        // ---- the state at the chunk start is in TMEM once MMA2a of chunk c-1 is done
         if (c > 0) {
             if (!(ok = wait_all(bar_mma, mma_phase))) break;
             mma_phase ^= 1;
             mma_pending = false;
             tc_fence_after();
-            if (tid == 0) load_b2(c);
+            if (tid == 0) load_b2_kbt_u(c);
             b2_pending = true;
             b2_chunk = c;
-            o_tma = L_prev == kC;
         }
         if (!RING && tid == kOutThread && c + 2 < nch) prefetch_l2(image(c + 2), IMG_BYTES);
-        // warps 4-7: O of the previous chunk out; a full chunk's tile leaves by
-        // one TMA store as soon as those four warps have written it
-        if (half == 1 && c > 0) {
-            emit_o(t_prev, L_prev, kStageO && o_tma);
-            if (kStageO && o_tma) {
-                fence_proxy_async_smem();
-                named_barrier(1, 128);
-                if (tid == kOutThread) {
-                    tma_store_3d(tm_o, smem + S_DT, 0, h, static_cast<int32_t>(t_prev));
-                    bulk_commit();
-                }
-            }
-        }
-        // all warps: the state decayed to this chunk's end (key channels
-        // 64*half ..): fp32 back into TMEM, and rounded to tf32 into the
-        // A-operand columns; it needs exp(Gamma_C), which comes with [Qt ; W]
+        if (tid == kOutThread) bulk_wait_read();   // the O staging tile is rewritten below
+        // decay (key channels 64*half ..): fp32 back into TMEM, rounded to tf32
+        // into the A-operand columns; it needs exp(Gamma_C), which comes with [Qt ; W]
         const bool b1_ok = mbar_wait_bounded(bar_b1, c & 1);
         if (b1_ok) {
             float st[2][32];
@@ -720,36 +702,61 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
             }
             tmem_wait_st();
         }
-        fence_proxy_async_smem();
         tc_fence_before();
         if (!(ok = !__syncthreads_or(!b1_ok))) break;
         b1_pending = false;
 
-        // ---- [Z^T | Y^T] = St^T [Qt ; W]^T; meanwhile O of the previous chunk leaves by TMA
+        // ---- MMA1: [Z_k^T | Y_k^T] = St^T [Qt ; W]^T
         if (tid == 0) {
             tc_fence_after();
             const uint64_t db = tdesc(sb, S_B1);
 #pragma unroll
             for (int s = 0; s < 16; ++s)
-                mma_tf32_ts(tmem + TS_Z, tmem + TS_A + 8 * s, kstep(db, KB_B1, s), ID_N128, s > 0);
+                mma_tf32_ts(tmem + zcol(c), tmem + TS_A + 8 * s, kstep(db, KB_B1, s), ID_N128, s > 0);
             mma_commit(bar_mma);
         }
         mma_pending = true;
-        if (kStageO && tid == kOutThread) bulk_wait_read();   // DT is written again below
-        if (!(ok = wait_all(bar_mma, mma_phase))) break;
+        // meanwhile (warps 4-7; thread 0 is busy issuing): O of chunk c-1 (a
+        // full chunk) into the staging tile; its product MMA2b also read P, so
+        // chunk c's copy of P waits for it
+        bool o_ok = true;
+        if (c > 0 && half == 1) {
+            o_ok = mbar_wait_bounded(bar_o, (c - 1) & 1);
+            if (o_ok) {
+                tc_fence_after();
+                if (tid == kOutThread) load_b2_p(c);
+#pragma unroll
+                for (int part = 0; part < 2; ++part) {
+                    float acc[32];
+                    tmem_ld32(tm_lane(tmem, quarter, zcol(c - 1) + 32 * part), acc);
+                    tmem_wait_ld();
+                    float* dst = reinterpret_cast<float*>(smem + S_OS) + (32 * part) * kD + e;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) dst[j * kD] = acc[j];
+                }
+            }
+            fence_proxy_async_smem();
+        }
+        tc_fence_before();
+        if (!(ok = !__syncthreads_or(!mbar_wait_bounded(bar_mma, mma_phase) || !o_ok))) break;
         mma_phase ^= 1;
         mma_pending = false;
+        if (c > 0) o_pending = false;
         tc_fence_after();
+        if (c > 0 && tid == kOutThread) {   // O of chunk c-1 leaves by one TMA store
+            tma_store_3d(tm_o, smem + S_OS, 0, h, static_cast<int32_t>(t_prev));
+            bulk_commit();
+        }
         if (tid == 0 && c + 1 < nch && (img_ok = await_image(c + 1))) load_b1(c + 1);
         b1_pending = c + 1 < nch;
         b1_chunk = c + 1;
 
-        // ---- delta^T = U^T - Y^T (tf32 operand, row = value column, K = token);
+        // ---- delta^T = U^T - Y_k^T (tf32 operand, row = value column, K = token);
         // U came with [Kb^T ; P]
         const bool b2_ok = mbar_wait_bounded(bar_b2, c & 1);
         if (b2_ok) {
             float y[32];
-            tmem_ld32(tm_lane(tmem, quarter, TS_Y + 32 * half), y);
+            tmem_ld32(tm_lane(tmem, quarter, zcol(c) + 64 + 32 * half), y);
             const float* us = reinterpret_cast<const float*>(smem + S_U) + (32 * half) * kD + e;
             float u[32];
 #pragma unroll
@@ -772,24 +779,41 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
         // completed), so the slot can be handed back with a plain store
         if (RING && tid == kOutThread) st_relaxed_gpu(ring.done + h, c + 1);
 
-        // ---- [S^T | O^T] += delta^T [Kb^T ; P]^T
+        // ---- MMA2a: S^T += delta^T Kb (thread 0);  MMA2b: Z_k^T += delta^T P^T,
+        // O of chunk c (kOutThread, so that neither issuing thread is held up
+        // by both)
         if (tid == 0) {
             tc_fence_after();
             const uint64_t da = tdesc(sb, S_DT), db = tdesc(sb, S_B2);
 #pragma unroll
             for (int s = 0; s < 8; ++s)
-                mma_tf32_ss(tmem + TS_S, kstep(da, 16384, s), kstep(db, KB_B2, s), ID_N192, 1);
+                mma_tf32_ss(tmem + TS_S, kstep(da, 16384, s), kstep(db, KB_B2, s), ID_N128, 1);
             mma_commit(bar_mma);
+        } else if (tid == kOutThread) {
+            tc_fence_after();
+            const uint64_t da = tdesc(sb, S_DT), dp = tdesc(sb, S_B2 + 128 * 128);
+#pragma unroll
+            for (int s = 0; s < 8; ++s)
+                mma_tf32_ss(tmem + zcol(c), kstep(da, 16384, s), kstep(dp, KB_B2, s), ID_N64, 1);
+            mma_commit(bar_o);
         }
         mma_pending = true;
+        o_pending = true;
         t_prev = t0;
-        L_prev = L;
-    }
-    if (ok && nch > 0) {
-        if ((ok = wait_all(bar_mma, mma_phase))) {
+        if (c + 1 == nch) {   // last chunk: O straight to o once MMA2b is done
+            if (!(ok = wait_all(bar_mma, mma_phase))) break;
             mma_pending = false;
+            if (!(ok = wait_all(bar_o, c & 1))) break;
+            o_pending = false;
             tc_fence_after();
-            if (half == 1) emit_o(t_prev, L_prev, false);
+            float acc[32];
+            tmem_ld32(tm_lane(tmem, quarter, zcol(c) + 32 * half), acc);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int r = 32 * half + j;
+                if (r < L) o[((size_t)(t0 + r) * H + h) * kD + e] = acc[j];
+            }
         }
     }
     if (ok) {
@@ -811,6 +835,7 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
         if (b1_pending) mbar_wait_bounded(bar_b1, b1_chunk & 1, 1u << 16);
         if (b2_pending) mbar_wait_bounded(bar_b2, b2_chunk & 1, 1u << 16);
         if (mma_pending) mbar_wait_bounded(bar_mma, mma_phase, 1u << 16);
+        if (o_pending) mbar_wait_bounded(bar_o, 0, 1u << 16), mbar_wait_bounded(bar_o, 1, 1u << 16);
     }
     if (tid == kOutThread) bulk_wait_all();
     tc_fence_before();

@@ -42,9 +42,10 @@ def assert_close(gpu, ref, tol, what):
 
 
 # The bf16 prefill has two tensor-core paths: the two-pass one (prep pass over
-# all chunks, then the sequential state pass) runs when the workspace holds
-# its scratch -- the binding's default -- and the fused single kernel runs
-# with the minimum workspace.
+# all chunks and the sequential state pass; for a single sequence both run
+# overlapped in one launch through a ring of operand slots) runs when the
+# workspace holds its scratch -- the binding's default -- and the fused single
+# kernel runs with the minimum workspace.
 PATHS = ["two_pass", "fused"]
 
 
@@ -359,6 +360,33 @@ def test_prefill_with_state_pool(mode):
     assert_close(pool_d[slots], s_ref, tol, "pooled final states")
     untouched = [i for i in range(6) if i not in slots]
     assert torch.equal(pool_d[untouched].cpu(), pool[untouched])
+
+
+def test_single_sequence_state_pool_overlapped_path():
+    # one sequence: the overlapped prep/state launch, reading and writing the
+    # state through a pool slot; 9 chunks wrap the 8-slot operand ring
+    dev = torch.device("cuda")
+    x = kin.make_custom_prefill(52, [9 * 64 - 5], heads=3, init_state_std=0.02)
+    pool = torch.randn(4, 3, 128, 128) * 0.02
+    pool[2] = x.initial_state[0]
+    pool_d = pool.to(dev)
+    xd = x.to(dev)
+    o = kda.kda_chunk_fwd_slots(xd.q, xd.k, xd.v, xd.g, xd.beta, xd.cu_seqlens, pool_d,
+                                torch.tensor([2], dtype=torch.int32, device=dev))
+    torch.cuda.synchronize()
+    o_ref, s_ref = oracle.kda_forward(x.q, x.k, x.v, x.g, x.beta, x.cu_seqlens, x.initial_state)
+    assert_close(o, o_ref, TOL_BF16, "o")
+    assert_close(pool_d[2:3], s_ref, TOL_BF16, "pooled final state")
+    assert torch.equal(pool_d[[0, 1, 3]].cpu(), pool[[0, 1, 3]])
+
+
+def test_single_sequence_with_many_heads_takes_the_two_launch_path():
+    # more heads than the overlapped launch gives state CTAs to: one sequence
+    # through the separate prep and state launches
+    x = kin.make_custom_prefill(53, [300], heads=100, init_state_std=0.02)
+    o, s, o_ref, s_ref = run_both(x, heads=[0, 57, 99])
+    assert_close(o, o_ref, TOL_BF16, "o")
+    assert_close(s, s_ref, TOL_BF16, "final state")
 
 
 def test_prefill_state_pool_rejects_bad_slot():
