@@ -48,15 +48,15 @@ STATE_BYTES = 4 * D * D
 PREFILL_FLOPS_PER_TOKEN_HEAD = (5 * 2 * 64 * 64 * D + 3 * 2 * 64 * D * D + 64 ** 3 // 3) // 64
 # Decode: state read + write, plus q, k, v (bf16), g (fp32), beta, o (fp32).
 DECODE_BYTES_PER_SEQ_HEAD = 2 * STATE_BYTES + 3 * 2 * D + 4 * D + 4 + 4 * D
-# One prefill call with the full workspace launches three kernels: the chunk
-# index, the parallel prep pass and the sequential state pass.  The prefill
-# roofline is taken over the whole call (algorithmic bytes of the call / its
-# CUDA-event time); the ncu launch list gives each kernel's share.
-PREFILL_KERNELS = ("kda_chunk_index_kernel", "kda_chunk_prep_kernel", "kda_chunk_state_kernel")
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one call, summed
-# over its kernels, from an ncu capture of the current kernel build on the
-# same workload; None whenever a kernel changed since it was captured.
-MEASURED_TRAFFIC_PREFILL = None
+# One prefill call of the 8K workload (one sequence, full workspace) launches
+# two kernels: the chunk index and the overlapped prep/state kernel.  The
+# prefill roofline is taken over the whole call (algorithmic bytes of the
+# call / its CUDA-event time); the ncu launch list gives each kernel's share.
+PREFILL_KERNELS = ("kda_chunk_index_kernel", "kda_chunk_overlap_kernel")
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one call, from
+# an ncu capture of the current kernel build on the same workload (the index
+# kernel's few KB left out); None whenever a kernel changed since it was captured.
+MEASURED_TRAFFIC_PREFILL = 337.748992e6 + 150.252800e6
 MEASURED_TRAFFIC_DECODE = 547.405312e6 + 486.942464e6
 
 
