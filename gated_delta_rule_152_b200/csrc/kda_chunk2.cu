@@ -123,9 +123,9 @@ constexpr uint32_t P_KB = 65536;     // 32 KB Kb: 64 rows x 128 channels, 4 K-bl
                                      //   TMA destination of the next item's raw q (16 KB) and k (16 KB)
 constexpr uint32_t P_KTT = 98304;    // 32 KB Kt^T: 128 channel rows x 64 tokens, 2 K-blocks x 16 KB
 constexpr uint32_t P_VT = 131072;    // 32 KB V^T: 128 value rows x 64 tokens, 2 K-blocks x 16 KB
-constexpr uint32_t P_RV = 163840;    // 16 KB raw v (bf16 [64 tokens][128]); after the prep, the P tile
-                                     //   (64 rows x 64 tokens, 2 K-blocks x 8 KB) on its way to the image
-constexpr uint32_t P_KBTS = 180224;  // 32 KB Kb^T (128 channel rows x 64 tokens) on its way to the image
+constexpr uint32_t P_RV = 163840;    // 16 KB raw v (bf16 [64 tokens][128])
+constexpr uint32_t P_KBTS = 180224;  // 32 KB Kb^T (128 channel rows x 64 tokens) on its way to the image,
+                                     //   then the P tile (64 rows x 64 tokens, 2 K-blocks x 8 KB)
 constexpr uint32_t P_MISC = 212992;  // beta[64] | xch[8][128] at +1024 | barriers at +5120
 constexpr uint32_t P_SMEM = P_MISC + 6144 + 1024;
 constexpr uint32_t P_KB_KB = 8192, P_KB_TP = 8192, P_KB_T = 16384;
@@ -300,7 +300,7 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
         load_pending = false;
         load_parity ^= 1;
 
-        // ============== prep: [Qt ; Kt] -> X, Kb -> KB, V^T -> VT, exp(Gamma_C) -> image
+        // ============== prep: [Qt ; Kt] -> X, Kb -> KB, exp(Gamma_C) -> image
         {
             float2 GC[2];
             prep_chunk_rows(smem + P_KB, smem + P_KB + kC * kD * 2, greg, xch, L, scale, l2norm != 0, GC,
@@ -313,23 +313,31 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
                 *reinterpret_cast<float4*>(im + IMG_DC + 16 * lane) =
                     make_float4(ex2(GC[0].x), ex2(GC[0].y), ex2(GC[1].x), ex2(GC[1].y));
             if (tid < kC) beta_s[tid] = breg;
-            // V^T from the raw v tile: thread = value column e, 32 tokens; rows past L are zero
-            const int e = tid & 127, tg = tid >> 7;
-            const __nv_bfloat16* rv = reinterpret_cast<const __nv_bfloat16*>(smem + P_RV);
-            float vv[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int i = 32 * tg + j;
-                vv[j] = (i < L) ? __bfloat162float(rv[i * kD + e]) : 0.f;
-            }
-#pragma unroll
-            for (int b = 0; b < 8; ++b)
-                *reinterpret_cast<float4*>(K_at(smem, P_VT, P_KB_T, e, 32 * tg + 4 * b)) =
-                    make_float4(vv[4 * b], vv[4 * b + 1], vv[4 * b + 2], vv[4 * b + 3]);
         }
+        fence_proxy_async_smem();
+        tc_fence_before();
         __syncthreads();
 
-        // ============== Kt^T -> KTT (shared), Kb^T -> image; thread = channel, 32 tokens
+        // ============== [Qt ; Kt] x Kb^T -> P (lanes 0-63), A (lanes 64-127); Qt -> image
+        if (tid == 0) {
+            tc_fence_after();
+            const uint64_t dx = tdesc(sb, P_X), dkb = tdesc(sb, P_KB);
+#pragma unroll
+            for (int s = 0; s < 16; ++s)
+                mma_tf32_ss(tmem + TP_AP, kstep(dx, KB_B1, s), kstep(dkb, P_KB_KB, s), ID_N64, s > 0);
+            mma_commit(bar_mma);
+        }
+        mma_pending = true;
+        if (tid == kStoreThread) {   // Qt -> rows 0-63 of [Qt ; W]
+            publish();
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb)
+                bulk_store(im + IMG_B1 + kb * KB_B1, smem + P_X + kb * KB_B1, 64 * 128);
+            bulk_commit();
+        }
+        // ============== while the Gram product runs (it only reads X and KB):
+        // Kt^T -> KTT and Kb^T -> staging (thread = channel, 32 tokens), V^T from the
+        // raw v tile (thread = value column, 32 tokens; rows past L are zero)
         {
             const int cch = tid & 127, tg = tid >> 7;
             float4 x[8], y[8];
@@ -351,33 +359,31 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
                 *reinterpret_cast<float4*>(K_at(smem, P_KTT, P_KB_T, cch, i0)) = x[b];
                 *reinterpret_cast<float4*>(K_at(smem, P_KBTS, P_KB_T, cch, i0)) = y[b];
             }
+            const __nv_bfloat16* rv = reinterpret_cast<const __nv_bfloat16*>(smem + P_RV);
+            float vv[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int i = 32 * tg + j;
+                vv[j] = (i < L) ? __bfloat162float(rv[i * kD + cch]) : 0.f;
+            }
+#pragma unroll
+            for (int b = 0; b < 8; ++b)
+                *reinterpret_cast<float4*>(K_at(smem, P_VT, P_KB_T, cch, 32 * tg + 4 * b)) =
+                    make_float4(vv[4 * b], vv[4 * b + 1], vv[4 * b + 2], vv[4 * b + 3]);
         }
         fence_proxy_async_smem();
-        tc_fence_before();
         __syncthreads();
-        if (tid == kStoreThread) {   // Kb^T -> image rows 0-127 of [Kb^T ; P]; Qt -> rows 0-63 of [Qt ; W]
-            publish();
+        if (tid == kStoreThread) {   // Kb^T -> rows 0-127 of [Kb^T ; P]; then X and the staging are free
 #pragma unroll
             for (int kb = 0; kb < 2; ++kb)
                 bulk_store(im + IMG_B2 + kb * KB_B2, smem + P_KBTS + kb * P_KB_T, P_KB_T);
-#pragma unroll
-            for (int kb = 0; kb < 4; ++kb)
-                bulk_store(im + IMG_B1 + kb * KB_B1, smem + P_X + kb * KB_B1, 64 * 128);
             bulk_commit();
+            bulk_wait_read();
         }
-
-        // ============== [Qt ; Kt] x Kb^T -> P (lanes 0-63), A (lanes 64-127)
-        if (tid == 0) {
-            tc_fence_after();
-            const uint64_t dx = tdesc(sb, P_X), dkb = tdesc(sb, P_KB);
-#pragma unroll
-            for (int s = 0; s < 16; ++s)
-                mma_tf32_ss(tmem + TP_AP, kstep(dx, KB_B1, s), kstep(dkb, P_KB_KB, s), ID_N64, s > 0);
-            mma_commit(bar_mma);
-        }
-        mma_pending = true;
-        if (tid == kStoreThread) bulk_wait_read();   // X is scratch from here on
         if (!(ok = wait_mma())) break;
+        // KB and RV are free: stage the next item's raw q, k, v
+        if (tid == 0 && has_next) issue_load(nxt);
+        load_pending = has_next;
 
         // ============== P -> staging tile (tf32, lower incl.), A -> M = strict_lower(beta A) (fp32)
         float* Mf = reinterpret_cast<float*>(smem + P_X);
@@ -388,12 +394,12 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
             float acc[32];
             tmem_ld32(tm_lane(tmem, quarter, TP_AP + 32 * half), acc);
             tmem_wait_ld();
-            if (quarter < 2) {   // P (lower incl.) -> the staging tile in RV (raw v is consumed)
+            if (quarter < 2) {   // P (lower incl.) -> the staging tile (Kb^T has left it)
                 const int r = 32 * quarter + lane;
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const int i0 = 32 * half + 4 * j;
-                    *reinterpret_cast<float4*>(smem + P_RV + half * P_KB_TP + sw128_off(r, j)) =
+                    *reinterpret_cast<float4*>(smem + P_KBTS + half * P_KB_TP + sw128_off(r, j)) =
                         tf32x4((i0 + 0 <= r) ? acc[4 * j + 0] : 0.f, (i0 + 1 <= r) ? acc[4 * j + 1] : 0.f,
                                (i0 + 2 <= r) ? acc[4 * j + 2] : 0.f, (i0 + 3 <= r) ? acc[4 * j + 3] : 0.f);
                 }
@@ -415,19 +421,15 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
         __syncthreads();
 
         // ============== T = (I + M)^-1, T' = T diag(beta) -> TP (tf32 operand, rows r, K = i);
-        // meanwhile the store thread sends P to the image and, once the staging
-        // tiles have been read, stages the next item's raw q, k, v (KB and RV are free)
+        // meanwhile the store thread sends P to the image
         ut_inverse64(Mf, Tf, Y1, Y2, tid, [&] {
             if (tid == kStoreThread) {
 #pragma unroll
                 for (int kb = 0; kb < 2; ++kb)
-                    bulk_store(im + IMG_B2 + kb * KB_B2 + 128 * 128, smem + P_RV + kb * P_KB_TP, P_KB_TP);
+                    bulk_store(im + IMG_B2 + kb * KB_B2 + 128 * 128, smem + P_KBTS + kb * P_KB_TP, P_KB_TP);
                 bulk_commit();
-                bulk_wait_read();
-                if (has_next) issue_load(nxt);
             }
         });
-        load_pending = has_next;
         {
             const int r = tid >> 2;
             float4 t4[4], b4[4];
