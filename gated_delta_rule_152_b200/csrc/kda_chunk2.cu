@@ -314,6 +314,8 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
                     make_float4(ex2(GC[0].x), ex2(GC[0].y), ex2(GC[1].x), ex2(GC[1].y));
             if (tid < kC) beta_s[tid] = breg;
         }
+        // the previous item's W and U have left the KTT / VT tiles rewritten below
+        if (tid == kStoreThread) bulk_wait_read();
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
@@ -467,17 +469,18 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
         if (!(ok = wait_mma())) break;
 
         // ============== W (tf32, a 64-row K-major tile) and U ([token][value],
-        // fp32) staged in X (free now), then bulk-stored to the image
+        // fp32) staged in KTT and VT (their products are done; the next item
+        // rewrites them only after its prep), then bulk-stored to the image
         {
             float acc[32];
             const int c = 32 * quarter + lane;   // channel (W) or value column (U)
             tmem_ld32(tm_lane(tmem, quarter, TP_W + 32 * half), acc);
             tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) *K_at(smem, P_X, P_KB_KB, 32 * half + j, c) = to_tf32(acc[j]);
+            for (int j = 0; j < 32; ++j) *K_at(smem, P_KTT, P_KB_KB, 32 * half + j, c) = to_tf32(acc[j]);
             tmem_ld32(tm_lane(tmem, quarter, TP_U + 32 * half), acc);
             tmem_wait_ld();
-            float* dst = reinterpret_cast<float*>(smem + P_X + 32768) + (32 * half) * kD + c;
+            float* dst = reinterpret_cast<float*>(smem + P_VT) + (32 * half) * kD + c;
 #pragma unroll
             for (int j = 0; j < 32; ++j) dst[j * kD] = acc[j];
         }
@@ -487,10 +490,9 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
         if (tid == kStoreThread) {
 #pragma unroll
             for (int kb = 0; kb < 4; ++kb)
-                bulk_store(im + IMG_B1 + kb * KB_B1 + 64 * 128, smem + P_X + kb * P_KB_KB, P_KB_KB);
-            bulk_store(im + IMG_U, smem + P_X + 32768, 32768);
+                bulk_store(im + IMG_B1 + kb * KB_B1 + 64 * 128, smem + P_KTT + kb * P_KB_KB, P_KB_KB);
+            bulk_store(im + IMG_U, smem + P_VT, 32768);
             bulk_commit();
-            bulk_wait_read();   // the next item's prep rewrites X
             if (RING) {
                 pub_flag = ring.ready + cur.h * kRing + (cur.c & (kRing - 1));
                 pub_val = cur.c + 1;
