@@ -155,7 +155,8 @@ struct Ring {
 // of head w % H, in the global chunk order of chunk_off).
 template <bool RING>
 __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
-                                          const float* __restrict__ g, const float* __restrict__ beta,
+                                          const CUtensorMap* tm_g, const float* __restrict__ g,
+                                          const float* __restrict__ beta,
                                           const int32_t* __restrict__ cu, const int32_t* __restrict__ chunk_off,
                                           int N, int H, int64_t max_total, float scale, int l2norm, int scalar_g,
                                           uint8_t* __restrict__ img, uint32_t* err, int64_t first, int64_t stride,
@@ -281,9 +282,10 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
     prefetch(cur);
 
     for (; ok && w < items; w += stride) {
-        const int64_t wn = w + stride;
-        const bool has_next = wn < items;
+        const int64_t wn = w + stride, w2 = wn + stride;
+        const bool has_next = wn < items, has_next2 = w2 < items;
         const Item nxt = has_next ? decode(wn) : cur;
+        const Item nxt2 = has_next2 ? decode(w2) : cur;   // only for an L2 prefetch below
         uint8_t* im = image_of(cur);
         const int L = cur.L;
 
@@ -383,8 +385,18 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
             bulk_wait_read();
         }
         if (!(ok = wait_mma())) break;
-        // KB and RV are free: stage the next item's raw q, k, v
-        if (tid == 0 && has_next) issue_load(nxt);
+        // KB and RV are free: stage the next item's raw q, k, v, and bring the
+        // item after it (its q, k, v and g) into L2 so that its loads find it there
+        if (tid == 0 && has_next) {
+            issue_load(nxt);
+            if (has_next2) {
+                const int32_t t2 = static_cast<int32_t>(nxt2.t0);
+                tma_prefetch_3d(tm_q, 0, nxt2.h, t2);
+                tma_prefetch_3d(tm_k, 0, nxt2.h, t2);
+                tma_prefetch_3d(tm_v, 0, nxt2.h, t2);
+                if (!scalar_g) tma_prefetch_3d(tm_g, 0, nxt2.h, t2);
+            }
+        }
         load_pending = has_next;
 
         // ============== P -> staging tile (tf32, lower incl.), A -> M = strict_lower(beta A) (fp32)
@@ -852,11 +864,12 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
 
 __global__ void __launch_bounds__(kThreads, 1)
 kda_chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                      const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ g,
+                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                      const float* __restrict__ g,
                       const float* __restrict__ beta, const int32_t* __restrict__ cu,
                       const int32_t* __restrict__ chunk_off, int N, int H, int64_t max_total, float scale,
                       int l2norm, int scalar_g, uint8_t* __restrict__ img, uint32_t* err) {
-    prep_role<false>(&tm_q, &tm_k, &tm_v, g, beta, cu, chunk_off, N, H, max_total, scale, l2norm, scalar_g, img,
+    prep_role<false>(&tm_q, &tm_k, &tm_v, &tm_g, g, beta, cu, chunk_off, N, H, max_total, scale, l2norm, scalar_g, img,
                      err, blockIdx.x, gridDim.x, Ring{nullptr, nullptr});
 }
 
@@ -874,7 +887,8 @@ kda_chunk_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t* 
 // ahead of them through the ring.
 __global__ void __launch_bounds__(kThreads, 1)
 kda_chunk_overlap_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                         const __grid_constant__ CUtensorMap tm_o,
                          const float* __restrict__ g, const float* __restrict__ beta, const int32_t* __restrict__ cu,
                          const int32_t* __restrict__ chunk_off, int H, int64_t total_T, int64_t max_total,
                          float scale, int l2norm, int scalar_g, uint8_t* __restrict__ img, const float* s0,
@@ -884,7 +898,7 @@ kda_chunk_overlap_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_
         state_role<true>(&tm_o, img, chunk_off, cu, total_T, H, max_total, s0, sT, o, err, slots, num_slots, 0,
                          blockIdx.x, ring);
     else
-        prep_role<true>(&tm_q, &tm_k, &tm_v, g, beta, cu, chunk_off, 1, H, max_total, scale, l2norm, scalar_g, img,
+        prep_role<true>(&tm_q, &tm_k, &tm_v, &tm_g, g, beta, cu, chunk_off, 1, H, max_total, scale, l2norm, scalar_g, img,
                         err, blockIdx.x - H, gridDim.x - H, ring);
 }
 
@@ -929,10 +943,13 @@ cudaError_t launch_chunk_two_pass(const PrefillArgs& a, void* scratch, cudaStrea
         if (attr_err == cudaSuccess) attr_err = set_smem(kda_chunk_overlap_kernel, O_SMEM);
     });
     if (attr_err != cudaSuccess) return attr_err;
-    CUtensorMap mq, mk, mv, mo;
+    CUtensorMap mq, mk, mv, mg, mo;
     if (!make_token_map(&mq, a.q, a.total_T, a.H) || !make_token_map(&mk, a.k, a.total_T, a.H) ||
         !make_token_map(&mv, a.v, a.total_T, a.H) || !make_token_map(&mo, a.o, a.total_T, a.H, true))
         return cudaErrorInvalidValue;
+    // g as [total_T, H, 128] fp32 for L2 prefetches (the scalar-decay form is not prefetched)
+    if (a.scalar_decay) mg = mo;
+    else if (!make_token_map(&mg, a.g, a.total_T, a.H, true)) return cudaErrorInvalidValue;
     int32_t* chunk_off = static_cast<int32_t*>(scratch);
     const int64_t max_total = static_cast<int64_t>(max_chunks(a.N, a.total_T));
     const int sms = num_sms();
@@ -962,7 +979,7 @@ cudaError_t launch_chunk_two_pass(const PrefillArgs& a, void* scratch, cudaStrea
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         const cudaError_t e = cudaLaunchKernelEx(
-            &cfg, kda_chunk_overlap_kernel, mq, mk, mv, mo, a.g, a.beta, a.cu_seqlens,
+            &cfg, kda_chunk_overlap_kernel, mq, mk, mv, mg, mo, a.g, a.beta, a.cu_seqlens,
             static_cast<const int32_t*>(chunk_off), static_cast<int>(a.H), a.total_T, max_total, a.scale,
             a.l2norm ? 1 : 0, a.scalar_decay ? 1 : 0, img, a.initial_state, a.final_state, a.o, a.err, a.slots,
             static_cast<int>(a.num_slots), ring);
@@ -976,7 +993,7 @@ cudaError_t launch_chunk_two_pass(const PrefillArgs& a, void* scratch, cudaStrea
     const size_t grid1 = items_ub < static_cast<size_t>(sms) ? items_ub : static_cast<size_t>(sms);
     if (grid1 > 0)
         kda_chunk_prep_kernel<<<static_cast<unsigned>(grid1), kThreads, P_SMEM, stream>>>(
-            mq, mk, mv, a.g, a.beta, a.cu_seqlens, chunk_off, a.N, a.H, max_total, a.scale, a.l2norm ? 1 : 0,
+            mq, mk, mv, mg, a.g, a.beta, a.cu_seqlens, chunk_off, a.N, a.H, max_total, a.scale, a.l2norm ? 1 : 0,
             a.scalar_decay ? 1 : 0, img, a.err);
     const long long blocks = (long long)a.N * a.H;
     kda_chunk_state_kernel<<<static_cast<unsigned>(blocks), kThreads, S_SMEM, stream>>>(
