@@ -223,35 +223,53 @@ def bench_gpu(args, world, rank, local):
     tf32_peak = bf16 * TF32_OVER_BF16
     achieved_tflops = flops_per_launch / (ms / 1e3) / 1e12
 
-    # end to end: pinned host inputs -> device, call, o + final state -> host
+    # end to end: pinned host inputs -> device, call, o + final state -> host,
+    # every step.  The result copies of step i run on a second stream while
+    # step i+1's inputs come in (PCIe is full duplex); outputs and their host
+    # copies are double-buffered so that no copy is overwritten in flight.
     pin = lambda t: t.pin_memory()
     hq, hk, hv, hg, hb, hcu = (pin(t) for t in (x.q, x.k, x.v, x.g, x.beta, x.cu_seqlens))
-    ho = torch.empty(T, H, D).pin_memory()
-    hs = torch.empty(1, H, D, D).pin_memory()
+    ho = [torch.empty(T, H, D).pin_memory() for _ in range(2)]
+    hs = [torch.empty(1, H, D, D).pin_memory() for _ in range(2)]
+    do = [o, torch.empty(T, H, D, device=dev)]
+    ds = [sT, torch.empty(1, H, D, D, device=dev)]
     dq, dk, dv, dg, db, dcu = (torch.empty_like(t, device=dev) for t in (hq, hk, hv, hg, hb, hcu))
+    out_stream = torch.cuda.Stream(dev)
+    out_done = [torch.cuda.Event(), torch.cuda.Event()]
+    for ev in out_done:
+        ev.record(out_stream)
 
-    def e2e_step():
+    def e2e_step(i):
+        b = i & 1
         for d_, h_ in ((dq, hq), (dk, hk), (dv, hv), (dg, hg), (db, hb), (dcu, hcu)):
             d_.copy_(h_, non_blocking=True)
-        kda.kda_chunk_fwd(dq, dk, dv, dg, db, dcu, final_state=sT, o=o, workspace=ws, stream=stream)
-        ho.copy_(o, non_blocking=True)
-        hs.copy_(sT, non_blocking=True)
+        stream.wait_event(out_done[b])   # step i-2's results have left buffer b
+        kda.kda_chunk_fwd(dq, dk, dv, dg, db, dcu, final_state=ds[b], o=do[b], workspace=ws, stream=stream)
+        computed = torch.cuda.Event()
+        computed.record(stream)
+        out_stream.wait_event(computed)
+        with torch.cuda.stream(out_stream):
+            ho[b].copy_(do[b], non_blocking=True)
+            hs[b].copy_(ds[b], non_blocking=True)
+        out_done[b].record(out_stream)
 
-    for _ in range(max(1, args.warmup)):
-        e2e_step()
+    for i in range(max(1, args.warmup)):
+        e2e_step(i)
     torch.cuda.synchronize(dev)
     barrier(world)
     torch.cuda.synchronize(dev)
     e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
+    for i in range(args.steps):
+        e2e_step(i)
+    for ev in out_done:   # the last results are on the host
+        stream.wait_event(ev)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hg, hb, hcu))
-    d2h = ho.numel() * 4 + hs.numel() * 4
-    del xd, dq, dk, dv, dg, db
+    d2h = ho[0].numel() * 4 + hs[0].numel() * 4
+    del xd, dq, dk, dv, dg, db, do, ds
     torch.cuda.empty_cache()
 
     # ---------------- decode (256 seq x 34 layers) -------------------------
