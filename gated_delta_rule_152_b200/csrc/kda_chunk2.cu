@@ -547,7 +547,6 @@ static_assert(S_DC == S_B1 + IMG_DC && S_B2 % 1024 == 0 && S_U == S_B2 + B2_COPY
 constexpr uint32_t TS_S = 0;      // 128 cols: S^T fp32 (lane = value column, column = key channel)
 constexpr uint32_t TS_Z = 128;    // 64 cols: Z^T, then O^T (column = token) of even chunks; Y^T follows;
                                   //   odd chunks use the set 256 columns on (384 - 511)
-constexpr uint32_t TS_A = 256;    // 128 cols: St^T rounded to tf32, the A operand of the first product
 constexpr uint32_t TS_COLS = 512;
 constexpr uint32_t ID_N128 = idesc_tf32(128, 128, false, false);
 constexpr int kOutThread = 128;   // issues the O stores, the L2 prefetches and the ring hand-back
@@ -555,9 +554,9 @@ constexpr int kOutThread = 128;   // issues the O stores, the L2 prefetches and 
 
 // Pass 2 for sequence n, head h.  Per chunk c (k = c % 2 selects one of two
 // Z/Y column sets in TMEM):
-//   decay:  St = Diag(e^Gamma_C) S into TMEM (fp32) and, rounded to tf32, into
-//           the A-operand columns                                  (all warps)
-//   MMA1:   [Z_k | Y_k] = St^T [Qt ; W]^T        (A from TMEM, B = [Qt ; W])
+//   decay:  St = Diag(e^Gamma_C) S in place in TMEM (fp32)         (all warps)
+//   MMA1:   [Z_k | Y_k] = St^T [Qt ; W]^T        (A = the state in TMEM, read as
+//           tf32; B = [Qt ; W])
 //           meanwhile O of chunk c-1 (set k^1) is read out and staged
 //   delta:  delta^T = U^T - Y_k^T                                  (all warps)
 //   MMA2a:  S^T += delta^T Kb   (the only product the next chunk waits for)
@@ -694,8 +693,10 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
         }
         if (!RING && tid == kOutThread && c + 2 < nch) prefetch_l2(image(c + 2), IMG_BYTES);
         if (tid == kOutThread) bulk_wait_read();   // the O staging tile is rewritten below
-        // decay (key channels 64*half ..): fp32 back into TMEM, rounded to tf32
-        // into the A-operand columns; it needs exp(Gamma_C), which comes with [Qt ; W]
+        // decay (key channels 64*half ..) in place; the fp32 state is also the A
+        // operand of MMA1, which reads it as tf32 (the low mantissa bits are
+        // dropped; measured on the CPU against the fp64 oracle: no change in the
+        // error of o or S); it needs exp(Gamma_C), which comes with [Qt ; W]
         const bool b1_ok = mbar_wait_bounded(bar_b1, c & 1);
         if (b1_ok) {
             float st[2][32];
@@ -712,9 +713,6 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
                     st[part][4 * j + 2] *= d4.z; st[part][4 * j + 3] *= d4.w;
                 }
                 tmem_st32(tm_lane(tmem, quarter, TS_S + c0), st[part]);
-#pragma unroll
-                for (int j = 0; j < 32; ++j) st[part][j] = to_tf32(st[part][j]);
-                tmem_st32(tm_lane(tmem, quarter, TS_A + c0), st[part]);
             }
             tmem_wait_st();
         }
@@ -728,7 +726,7 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
             const uint64_t db = tdesc(sb, S_B1);
 #pragma unroll
             for (int s = 0; s < 16; ++s)
-                mma_tf32_ts(tmem + zcol(c), tmem + TS_A + 8 * s, kstep(db, KB_B1, s), ID_N128, s > 0);
+                mma_tf32_ts(tmem + zcol(c), tmem + TS_S + 8 * s, kstep(db, KB_B1, s), ID_N128, s > 0);
             mma_commit(bar_mma);
         }
         mma_pending = true;
