@@ -175,9 +175,16 @@ def cpu_baseline(x: kin.PrefillInputs, target_s: float = 10.0):
     tokens = int(min(x.total_T, max(probe_tokens, probe_tokens * target_s / max(dt, 1e-6))))
     tokens = max(64, (tokens // 64) * 64)
     dt, tokens = oracle_prefill_sample(x, tokens)
-    return {"value": tokens / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": f"first {tokens} of 8192 tokens x 32 heads of prefill_bf16_T8192_H32, fp64, "
-                      f"{cores} OpenMP threads over (sequence, head) pairs, {dt:.1f} s"}
+    # when the whole workload takes well under the target, repeat whole
+    # passes so the rate is taken over about target_s of work
+    passes, total = 1, dt
+    while tokens == x.total_T and total < target_s and passes < 32:
+        dt, _ = oracle_prefill_sample(x, tokens)
+        passes, total = passes + 1, total + dt
+    what = (f"{passes} passes over all {tokens}" if passes > 1 else f"first {tokens} of {x.total_T}")
+    return {"value": tokens * passes / total, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{what} tokens x 32 heads of prefill_bf16_T8192_H32, fp64, "
+                      f"{cores} OpenMP threads over (sequence, head) pairs, {total:.1f} s"}
 
 
 # ---------------------------------------------------------------- GPU arm

@@ -13,6 +13,7 @@ from .kda import (  # noqa: F401
     kda_chunk_fwd_workspace_size_min,
     kda_decode_step,
     kda_decode_step_slots,
+    kda_selftest_bounded_waits,
     kda_status_string,
     kda_verify_fwd,
     kda_workspace_error,

@@ -37,6 +37,7 @@ KDA_DEVERR_SLOT = 4
 EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd_workspace_size_min", "kda_chunk_fwd",
             "kda_decode_step",
             "kda_chunk_fwd_slots", "kda_decode_step_slots", "kda_verify_fwd", "kda_workspace_error",
+            "kda_selftest_bounded_waits",
             "kda_status_string")
 
 _lock = threading.Lock()
@@ -81,6 +82,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.kda_verify_fwd.restype = ctypes.c_int
         lib.kda_workspace_error.argtypes = [P, ctypes.POINTER(U32), P]
         lib.kda_workspace_error.restype = ctypes.c_int
+        lib.kda_selftest_bounded_waits.argtypes = [P, SZ, U32, P]
+        lib.kda_selftest_bounded_waits.restype = ctypes.c_int
         lib.kda_status_string.argtypes = [ctypes.c_int]
         lib.kda_status_string.restype = ctypes.c_char_p
         _lib = lib
@@ -330,6 +333,15 @@ def kda_verify_fwd(q, k, v, g, beta, cu_seqlens, *, initial_state: Optional[torc
     if st != KDA_OK:
         raise KdaError(st, "kda_verify_fwd")
     return o, snapshots
+
+
+def kda_selftest_bounded_waits(workspace: torch.Tensor, polls: int = 4096, stream=None) -> None:
+    """Enqueue the self-test whose bounded waits must give up (see the header);
+    read the outcome with kda_workspace_error(workspace)."""
+    st = load_library().kda_selftest_bounded_waits(_ptr(workspace), workspace.numel() * workspace.element_size(),
+                                                   int(polls), _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_selftest_bounded_waits")
 
 
 def kda_workspace_error(workspace: torch.Tensor, stream=None) -> int:

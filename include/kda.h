@@ -242,6 +242,20 @@ KDA_API int kda_verify_fwd(const void *q, const void *k, const void *v, const fl
  */
 KDA_API int kda_workspace_error(const void *workspace, uint32_t *out, kda_stream_t stream);
 
+/*
+ * Self-test of the kernels' bounded waits (no counterpart on the pages; it
+ * exists so that the failure path can be exercised without a GPU fault).
+ * Launches one small kernel that waits, `polls` times at most each, for a
+ * global flag that nothing sets (workspace word 1, cleared by this call) and
+ * for an mbarrier phase that never completes; each wait that gives up sets
+ * KDA_DEVERR_TIMEOUT in workspace word 0 (cleared by this call) and the
+ * kernel returns normally, so the context stays usable.  workspace: device
+ * memory, 16-byte aligned, at least 256 bytes.  Returns KDA_OK once the
+ * kernel is enqueued; read the outcome with kda_workspace_error().
+ */
+KDA_API int kda_selftest_bounded_waits(void *workspace, size_t workspace_bytes, uint32_t polls,
+                                       kda_stream_t stream);
+
 /* Static English description of a kda_status value. */
 KDA_API const char *kda_status_string(int status);
 

@@ -117,3 +117,10 @@ def test_binding_rejects_cpu_tensors():
     x = torch.zeros(4, 2, 128)
     with pytest.raises(ValueError):
         kda.kda_chunk_fwd(x, x, x, x, torch.zeros(4, 2), torch.tensor([0, 4], dtype=torch.int32))
+
+
+def test_selftest_rejects_bad_workspace(lib):
+    P = ctypes.c_void_p
+    assert lib.kda_selftest_bounded_waits(None, 256, 16, None) == kda.KDA_ERR_WORKSPACE
+    assert lib.kda_selftest_bounded_waits(P(A), 64, 16, None) == kda.KDA_ERR_WORKSPACE
+    assert lib.kda_selftest_bounded_waits(P(MIS), 256, 16, None) == kda.KDA_ERR_MISALIGNED

@@ -448,3 +448,47 @@ def test_verify_snapshots_match_prefix_states(dtype):
             _, s_ref = oracle.kda_forward(x.q[sl], x.k[sl], x.v[sl], x.g[sl], x.beta[sl], [0, t + 1 - cu[n]],
                                           x.initial_state[n:n + 1])
             assert_close(snaps[t:t + 1], s_ref[:, :], TOL_FP32, f"snapshot of token {t}")
+
+
+def test_bounded_waits_give_up_with_an_error_and_the_context_survives():
+    # a flag nobody sets and an mbarrier phase that never completes: both
+    # bounded waits give up, report KDA_DEVERR_TIMEOUT, and later work runs
+    dev = torch.device("cuda")
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    kda.kda_selftest_bounded_waits(ws, polls=4096)
+    assert kda.kda_workspace_error(ws) & kda.KDA_DEVERR_TIMEOUT
+    x = kin.make_custom_prefill(62, [130], heads=2, init_state_std=0.02)
+    o, s, o_ref, s_ref = run_both(x)
+    assert_close(o, o_ref, TOL_BF16, "o after the self-test")
+    assert_close(s, s_ref, TOL_BF16, "final state after the self-test")
+
+
+@pytest.mark.parametrize("lengths", [[700], [300, 450]])
+def test_prefill_replays_from_a_cuda_graph(lengths):
+    # the overlapped (one sequence) and two-launch (two sequences) paths,
+    # captured once and replayed: the same bits as the eager call
+    dev = torch.device("cuda")
+    x = kin.make_custom_prefill(61, lengths, heads=4, init_state_std=0.02).to(dev)
+    T, H, d = x.q.shape
+    N = len(lengths)
+    ws = torch.zeros(kda.kda_chunk_fwd_workspace_size(N, T, H), dtype=torch.uint8, device=dev)
+    o = torch.empty(T, H, d, device=dev)
+    sT = torch.empty(N, H, d, d, device=dev)
+    call = lambda: kda.kda_chunk_fwd(x.q, x.k, x.v, x.g, x.beta, x.cu_seqlens, initial_state=x.initial_state,
+                                     final_state=sT, o=o, workspace=ws)
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        call()
+    torch.cuda.current_stream(dev).wait_stream(side)
+    torch.cuda.synchronize()
+    o_ref, s_ref = o.clone(), sT.clone()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call()
+    o.zero_()
+    sT.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_ref) and torch.equal(sT, s_ref)
+    assert kda.kda_workspace_error(ws) == 0
