@@ -13,16 +13,23 @@
 // Everything except the last line is independent of the state.  Pass 1
 // (kda_chunk_prep_kernel) therefore runs over all (chunk, head) pairs in
 // parallel and writes, per pair, ready-made tensor-core operand images of
-// [Qt ; W] and [Kb^T ; P], and U and e^Gamma_C, to scratch.  Pass 2
+// [Qt ; W], Kb and P, and U and e^Gamma_C, to scratch.  Pass 2
 // (kda_chunk_state_kernel) walks the chunks of one (sequence, head) in order
 // and only carries the state:
 //     [Z^T | Y^T] = St^T [Qt ; W]^T            (M = 128 value columns, N = 128)
 //     delta^T = U^T - Y^T
-//     [S_next^T | O^T] = [St^T | Z^T] + delta^T [Kb^T ; P]^T    (N = 192)
+//     S_next^T = St^T + delta^T Kb,   O^T = Z^T + delta^T P^T
 // The state is kept transposed in tensor memory (lane = value column, column
-// = key channel), so it is the A operand of the first product and the
-// accumulator of the second, and the readout O^T lands with the value
+// = key channel), so it is the A operand of the first products and the
+// accumulator of the update, and the readout O^T lands with the value
 // column in the lane, which is the contiguous axis of o in global memory.
+//
+// Operand tiles have 128-byte rows.  K-major tiles (the reduction axis
+// contiguous) permute 16-byte chunks by the row index mod 8; MN-major tf32
+// tiles (the other axis contiguous), which the tensor core reads with a
+// different swizzle, permute 32-byte granules by the row index mod 4.  Pass 1
+// writes Kt, Kb and V in the token-row orientation it produces them in and
+// lets the products read them MN-major, so no tile is transposed.
 //
 // Precision: as the fused kernel -- tf32 operands (rounded to nearest),
 // fp32 accumulation, fp32 state; U is kept in fp32.
@@ -39,17 +46,21 @@ namespace {
 constexpr int kC = 64;
 constexpr int kThreads = 256;
 
-// ---- per (chunk, head) operand image in scratch (byte offsets); tiles are
-// K-major with the 128-byte swizzle, exactly as they sit in shared memory.
-constexpr uint32_t IMG_B1 = 0;        // [Qt ; W]: rows 0-63 Qt, 64-127 W (token) x 128 channels, 4 K-blocks x 16 KB
+// ---- per (chunk, head) operand image in scratch (byte offsets), tiles
+// exactly as the state pass holds them in shared memory.
+constexpr uint32_t IMG_B1 = 0;        // [Qt ; W]: rows 0-63 Qt, 64-127 W (token) x 128 channels, K-major,
+                                      //   4 K-blocks x 16 KB
 constexpr uint32_t IMG_DC = 65536;    // exp(Gamma_C): 128 fp32 (+ 512 B pad)
-constexpr uint32_t IMG_B2 = 66560;    // [Kb^T ; P]: rows 0-127 Kb^T (channel), 128-191 P (token) x 64 tokens, 2 K-blocks x 24 KB
-constexpr uint32_t IMG_U = 115712;    // U: [token][value column] fp32, 64 x 128
+constexpr uint32_t IMG_KB = 66560;    // Kb: 64 token rows x 128 channels, MN-major, 4 blocks of 32 channels x 8 KB
+constexpr uint32_t IMG_P = 99328;     // P: 64 token rows x 64 tokens, K-major, 2 K-blocks x 8 KB
+constexpr uint32_t IMG_U = 115712;    // U^T: 128 value rows x 64 tokens fp32, 16-byte chunks permuted as
+                                      //   K-major tiles, 2 blocks of 32 tokens x 16 KB
 constexpr uint32_t IMG_BYTES = 148480;
-constexpr uint32_t KB_B1 = 16384, KB_B2 = 24576;
+constexpr uint32_t KB_B1 = 16384, IMG_BLK = 8192;   // K-block of [Qt ; W]; 64 rows x 128 B
 constexpr uint32_t B1_COPY = IMG_DC + 512;   // [Qt ; W] and exp(Gamma_C) in one copy
-constexpr uint32_t B2_COPY = 49152;
-static_assert(IMG_B2 % 1024 == 0 && IMG_U == IMG_B2 + B2_COPY && IMG_BYTES == IMG_U + 32768, "image layout");
+constexpr uint32_t B2_COPY = IMG_BYTES - IMG_KB;   // Kb, P and U on one mbarrier phase
+static_assert(IMG_KB % 1024 == 0 && IMG_P == IMG_KB + 32768 && IMG_U == IMG_P + 16384 &&
+              IMG_BYTES == IMG_U + 32768, "image layout");
 
 __device__ __forceinline__ bool seq_bounds(const int32_t* cu, int n, int64_t total_T, int64_t& bos, int64_t& eos) {
     bos = cu[n];
@@ -116,33 +127,40 @@ __global__ void __launch_bounds__(1024) kda_chunk_index_kernel(const int32_t* __
 
 // ============================================================ pass 1
 // Shared memory (byte offsets from a 1024-aligned base).
-constexpr uint32_t P_X = 0;          // 64 KB [Qt ; Kt]: 128 rows x 128 channels, 4 K-blocks x 16 KB.
-                                     //   After the Gram MMA: triangular-solve scratch, and T' at P_TP.
-constexpr uint32_t P_TP = 49152;     // 16 KB T': 64 rows (token r) x 64 (token i), 2 K-blocks x 8 KB
-constexpr uint32_t P_KB = 65536;     // 32 KB Kb: 64 rows x 128 channels, 4 K-blocks x 8 KB; also the
+constexpr uint32_t P_X = 0;          // 64 KB [Qt ; Kt]: 128 rows x 128 channels, K-major, 4 K-blocks x 16 KB
+                                     //   (A of the Gram product).  After it: the triangular-solve scratch
+                                     //   (from 0), T' (at P_TP), then P on its way to the image (from 0)
+constexpr uint32_t P_TP = 49152;     // 16 KB T': 64 rows (token r) x 64 (token i), K-major, 2 K-blocks x 8 KB
+constexpr uint32_t P_KB = 65536;     // 32 KB Kb: 64 rows x 128 channels, K-major, 4 K-blocks x 8 KB; also the
                                      //   TMA destination of the next item's raw q (16 KB) and k (16 KB)
-constexpr uint32_t P_KTT = 98304;    // 32 KB Kt^T: 128 channel rows x 64 tokens, 2 K-blocks x 16 KB
-constexpr uint32_t P_VT = 131072;    // 32 KB V^T: 128 value rows x 64 tokens, 2 K-blocks x 16 KB
-constexpr uint32_t P_RV = 163840;    // 16 KB raw v (bf16 [64 tokens][128])
-constexpr uint32_t P_KBTS = 180224;  // 32 KB Kb^T (128 channel rows x 64 tokens) on its way to the image,
-                                     //   then the P tile (64 rows x 64 tokens, 2 K-blocks x 8 KB)
+constexpr uint32_t P_KTM = 98304;    // 32 KB Kt MN-major: 64 token rows x 128 channels, 4 blocks x 8 KB
+                                     //   (Kt^T for W^T)
+constexpr uint32_t P_WST = 131072;   // 32 KB W (K-major, 4 K-blocks x 8 KB) on its way to the image
+constexpr uint32_t P_V = 163840;     // 32 KB V MN-major: 64 token rows x 128 values, 4 blocks x 8 KB
+                                     //   (V^T for U^T); then U^T on its way out
+constexpr uint32_t P_RV = 196608;    // 16 KB raw v (bf16 [64 tokens][128])
 constexpr uint32_t P_MISC = 212992;  // beta[64] | xch[8][128] at +1024 | barriers at +5120
 constexpr uint32_t P_SMEM = P_MISC + 6144 + 1024;
-constexpr uint32_t P_KB_KB = 8192, P_KB_TP = 8192, P_KB_T = 16384;
-constexpr int kStoreThread = 128;    // issues the bulk stores and the next item's TMA loads
-static_assert(kUtScratchBytes <= P_TP, "solve scratch overlaps T'");
+constexpr uint32_t P_KB_KB = 8192, P_KB_TP = 8192, P_MN_KB = 8192;
+// Issues the bulk stores and the ring hand-over.  Its warp (quarter 3) reads
+// no P, so the hand-over overlaps the W / U product.  Bulk-store groups per
+// item: P (from X), then W and U (from WST and V).
+constexpr int kStoreThread = 224;
+static_assert(kUtScratchBytes <= P_TP - P_X, "solve scratch");
 
 constexpr uint32_t TP_AP = 0;     // 64 cols: P (lanes 0-63) | A (lanes 64-127)
 constexpr uint32_t TP_W = 64;     // 64 cols: W^T (lane = channel, column = token)
 constexpr uint32_t TP_U = 128;    // 64 cols: U^T (lane = value column, column = token)
 constexpr uint32_t TP_COLS = 256;
 constexpr uint32_t ID_N64 = idesc_tf32(128, 64, false, false);
+constexpr uint32_t ID_N64_AMN = idesc_tf32(128, 64, true, false);   // A read MN-major
+
 
 // Overlapped mode (one sequence): the prep role writes each (chunk, head)
 // image into a ring of kRing slots per head instead of its own place in the
 // scratch, and the two roles hand slots over through flags in global memory:
-//   ready[h * kRing + s] = c + 1 once chunk c's image sits complete in slot s,
-//   done[h]              = number of chunks of head h the state role has read.
+//   ready(h, s) = c + 1 once chunk c's image sits complete in slot s,
+//   done(h)     = number of chunks of head h the state role has read.
 // A slot is rewritten only after its previous chunk was read, so the ring
 // (kRing x H x IMG_BYTES, 37 MB for 32 heads) stays in L2.
 constexpr int kRing = 8;
@@ -150,6 +168,13 @@ struct Ring {
     int32_t* ready;
     int32_t* done;
 };
+// The flags of one head sit in a 128-byte line of their own, so that waiting
+// producers and the state CTAs of other heads do not contend for it.
+constexpr int kFlagStride = 32;
+__device__ __forceinline__ int32_t* ready_flag(const Ring& r, int h, int c) {
+    return r.ready + h * kFlagStride + (c & (kRing - 1));
+}
+__device__ __forceinline__ int32_t* done_flag(const Ring& r, int h) { return r.done + h * kFlagStride; }
 
 // Pass 1 for the work items first, first + stride, ... (item w = chunk w / H
 // of head w % H, in the global chunk order of chunk_off).
@@ -221,19 +246,25 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
                                  : static_cast<size_t>(it.gc) * H + it.h;
         return img + slot * IMG_BYTES;
     };
-    // ring mode: the image of the previous item is announced once its bulk
-    // stores have completed (checked when the store thread next issues stores)
+    // ring mode: the image of an item (Qt, Kb and exp(Gamma_C) written with
+    // plain stores before the item's block barriers, the rest by bulk stores)
+    // is announced by the store thread once those bulk stores have completed:
+    // a proxy fence, then a gpu-scope release, which also covers the plain
+    // stores of the other threads (ordered before it by the barriers).  That
+    // happens while the next item's W / U product runs, or before the store
+    // thread blocks on a slot.
     int32_t* pub_flag = nullptr;
     int32_t pub_val = 0;
     auto publish = [&]() {
+        bulk_wait_all();
         if (RING && pub_flag) {
-            bulk_wait_all();
             fence_proxy_async_global();
-            __threadfence();
             st_release_gpu(pub_flag, pub_val);
             pub_flag = nullptr;
         }
     };
+    // store thread: done[] of the item's head, read one item ahead
+    int32_t done_seen = 0;
     float greg[8][4];
     float breg;
     auto prefetch = [&](const Item& it) {
@@ -277,6 +308,8 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
 
     int64_t w = first;
     Item cur = decode(w);
+    Item nxt = w + stride < items ? decode(w + stride) : cur;
+    Item nxt2 = w + 2 * stride < items ? decode(w + 2 * stride) : cur;   // only for an L2 prefetch
     if (tid == 0) issue_load(cur);
     load_pending = true;
     prefetch(cur);
@@ -284,8 +317,6 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
     for (; ok && w < items; w += stride) {
         const int64_t wn = w + stride, w2 = wn + stride;
         const bool has_next = wn < items, has_next2 = w2 < items;
-        const Item nxt = has_next ? decode(wn) : cur;
-        const Item nxt2 = has_next2 ? decode(w2) : cur;   // only for an L2 prefetch below
         uint8_t* im = image_of(cur);
         const int L = cur.L;
 
@@ -293,36 +324,46 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
         // producer never blocks on it while holding an unannounced image (the
         // state role that it waits for may need exactly that image).
         bool slot_free = true;
-        if (RING && tid == kStoreThread && cur.c >= kRing &&
-            ld_acquire_gpu(ring.done + cur.h) < cur.c - kRing + 1) {
+        if (RING && tid == kStoreThread && cur.c >= kRing && done_seen < cur.c - kRing + 1 &&
+            ld_acquire_gpu(done_flag(ring, cur.h)) < cur.c - kRing + 1) {
             publish();
-            slot_free = wait_flag_ge(ring.done + cur.h, cur.c - kRing + 1);
+            slot_free = wait_flag_ge(done_flag(ring, cur.h), cur.c - kRing + 1, 1u << 20, 256);
         }
+        // the previous item's P has left X, which is rewritten below
+        if (tid == kStoreThread) bulk_wait_read_but<1>();
         if (!(ok = !__syncthreads_or(!mbar_wait_bounded(bar_load, load_parity) || !slot_free))) break;
         load_pending = false;
         load_parity ^= 1;
 
-        // ============== prep: [Qt ; Kt] -> X, Kb -> KB, exp(Gamma_C) -> image
+        // ============== prep: [Qt ; Kt] -> X, Kb -> KB (K-major), Kt -> KTM (MN-major);
+        // Qt (K-major), Kb (MN-major) and exp(Gamma_C) -> image (a warp stores four
+        // whole 128-byte rows at a time)
         {
             float2 GC[2];
             prep_chunk_rows(smem + P_KB, smem + P_KB + kC * kD * 2, greg, xch, L, scale, l2norm != 0, GC,
                             [&](int r, int kbi, int ch, float4 kt, float4 qt, float4 kb) {
-                                st_tf32x4(smem, P_X + kbi * KB_B1 + sw128_off(r, ch), qt.x, qt.y, qt.z, qt.w);
-                                st_tf32x4(smem, P_X + kbi * KB_B1 + sw128_off(64 + r, ch), kt.x, kt.y, kt.z, kt.w);
-                                st_tf32x4(smem, P_KB + kbi * P_KB_KB + sw128_off(r, ch), kb.x, kb.y, kb.z, kb.w);
+                                const float4 q4 = tf32x4(qt.x, qt.y, qt.z, qt.w);
+                                const float4 k4 = tf32x4(kt.x, kt.y, kt.z, kt.w);
+                                const float4 b4 = tf32x4(kb.x, kb.y, kb.z, kb.w);
+                                *reinterpret_cast<float4*>(smem + P_X + kbi * KB_B1 + sw128_off(r, ch)) = q4;
+                                *reinterpret_cast<float4*>(smem + P_X + kbi * KB_B1 + sw128_off(64 + r, ch)) = k4;
+                                *reinterpret_cast<float4*>(smem + P_KB + kbi * P_KB_KB + sw128_off(r, ch)) = b4;
+                                *reinterpret_cast<float4*>(smem + P_KTM + kbi * P_MN_KB + sw32g_off(r, ch)) = k4;
+                                *reinterpret_cast<float4*>(im + IMG_B1 + kbi * KB_B1 + sw128_off(r, ch)) = q4;
+                                *reinterpret_cast<float4*>(im + IMG_KB + kbi * IMG_BLK + sw32g_off(r, ch)) = b4;
                             });
             if (warp == 0)
                 *reinterpret_cast<float4*>(im + IMG_DC + 16 * lane) =
                     make_float4(ex2(GC[0].x), ex2(GC[0].y), ex2(GC[1].x), ex2(GC[1].y));
             if (tid < kC) beta_s[tid] = breg;
         }
-        // the previous item's W and U have left the KTT / VT tiles rewritten below
+        // the previous item's U has left V, which is rewritten below
         if (tid == kStoreThread) bulk_wait_read();
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
 
-        // ============== [Qt ; Kt] x Kb^T -> P (lanes 0-63), A (lanes 64-127); Qt -> image
+        // ============== [Qt ; Kt] x Kb^T -> P (lanes 0-63), A (lanes 64-127)
         if (tid == 0) {
             tc_fence_after();
             const uint64_t dx = tdesc(sb, P_X), dkb = tdesc(sb, P_KB);
@@ -332,58 +373,22 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
             mma_commit(bar_mma);
         }
         mma_pending = true;
-        if (tid == kStoreThread) {   // Qt -> rows 0-63 of [Qt ; W]
-            publish();
+        // ============== meanwhile: V (MN-major; bf16 is exact in tf32) from the raw
+        // tile, rows past L zero; a 32-byte granule holds the 8 values of a raw chunk
 #pragma unroll
-            for (int kb = 0; kb < 4; ++kb)
-                bulk_store(im + IMG_B1 + kb * KB_B1, smem + P_X + kb * KB_B1, 64 * 128);
-            bulk_commit();
-        }
-        // ============== while the Gram product runs (it only reads X and KB):
-        // Kt^T -> KTT and Kb^T -> staging (thread = channel, 32 tokens), V^T from the
-        // raw v tile (thread = value column, 32 tokens; rows past L are zero)
-        {
-            const int cch = tid & 127, tg = tid >> 7;
-            float4 x[8], y[8];
-#pragma unroll
-            for (int b = 0; b < 8; ++b) {
-                const int i0 = 32 * tg + 4 * b;
-                x[b].x = *K_at(smem, P_X, KB_B1, 64 + i0 + 0, cch);
-                x[b].y = *K_at(smem, P_X, KB_B1, 64 + i0 + 1, cch);
-                x[b].z = *K_at(smem, P_X, KB_B1, 64 + i0 + 2, cch);
-                x[b].w = *K_at(smem, P_X, KB_B1, 64 + i0 + 3, cch);
-                y[b].x = *K_at(smem, P_KB, P_KB_KB, i0 + 0, cch);
-                y[b].y = *K_at(smem, P_KB, P_KB_KB, i0 + 1, cch);
-                y[b].z = *K_at(smem, P_KB, P_KB_KB, i0 + 2, cch);
-                y[b].w = *K_at(smem, P_KB, P_KB_KB, i0 + 3, cch);
-            }
-#pragma unroll
-            for (int b = 0; b < 8; ++b) {
-                const int i0 = 32 * tg + 4 * b;
-                *reinterpret_cast<float4*>(K_at(smem, P_KTT, P_KB_T, cch, i0)) = x[b];
-                *reinterpret_cast<float4*>(K_at(smem, P_KBTS, P_KB_T, cch, i0)) = y[b];
-            }
-            const __nv_bfloat16* rv = reinterpret_cast<const __nv_bfloat16*>(smem + P_RV);
-            float vv[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int i = 32 * tg + j;
-                vv[j] = (i < L) ? __bfloat162float(rv[i * kD + cch]) : 0.f;
-            }
-#pragma unroll
-            for (int b = 0; b < 8; ++b)
-                *reinterpret_cast<float4*>(K_at(smem, P_VT, P_KB_T, cch, 32 * tg + 4 * b)) =
-                    make_float4(vv[4 * b], vv[4 * b + 1], vv[4 * b + 2], vv[4 * b + 3]);
+        for (int qd = 0; qd < 4; ++qd) {
+            const int id = qd * kThreads + tid, r = id >> 4, j = id & 15;   // row r, values 8 j .. 8 j + 7
+            uint4 u = make_uint4(0u, 0u, 0u, 0u);
+            if (r < L) u = *reinterpret_cast<const uint4*>(smem + P_RV + r * (kD * 2) + 16 * j);
+            uint8_t* dst = smem + P_V + (j >> 2) * P_MN_KB;
+            *reinterpret_cast<float4*>(dst + sw32g_off(r, 2 * (j & 3))) =
+                make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
+                            __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u));
+            *reinterpret_cast<float4*>(dst + sw32g_off(r, 2 * (j & 3) + 1)) =
+                make_float4(__uint_as_float(u.z << 16), __uint_as_float(u.z & 0xFFFF0000u),
+                            __uint_as_float(u.w << 16), __uint_as_float(u.w & 0xFFFF0000u));
         }
         fence_proxy_async_smem();
-        __syncthreads();
-        if (tid == kStoreThread) {   // Kb^T -> rows 0-127 of [Kb^T ; P]; then X and the staging are free
-#pragma unroll
-            for (int kb = 0; kb < 2; ++kb)
-                bulk_store(im + IMG_B2 + kb * KB_B2, smem + P_KBTS + kb * P_KB_T, P_KB_T);
-            bulk_commit();
-            bulk_wait_read();
-        }
         if (!(ok = wait_mma())) break;
         // KB and RV are free: stage the next item's raw q, k, v, and bring the
         // item after it (its q, k, v and g) into L2 so that its loads find it there
@@ -399,51 +404,31 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
         }
         load_pending = has_next;
 
-        // ============== P -> staging tile (tf32, lower incl.), A -> M = strict_lower(beta A) (fp32)
+        // ============== A -> M = strict_lower(beta A) (fp32, in X); P stays in TMEM
         float* Mf = reinterpret_cast<float*>(smem + P_X);
         float* Tf = Mf + 64 * kLd;
         float* Y1 = Tf + 64 * kLd;
         float* Y2 = Y1 + 2 * 16 * kLd1;
-        {
+        if (quarter >= 2) {
             float acc[32];
             tmem_ld32(tm_lane(tmem, quarter, TP_AP + 32 * half), acc);
             tmem_wait_ld();
-            if (quarter < 2) {   // P (lower incl.) -> the staging tile (Kb^T has left it)
-                const int r = 32 * quarter + lane;
+            const int r = 32 * quarter + lane - 64;
+            const float br = beta_s[r];
+            float* mrow = Mf + r * kLd + 32 * half;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int i0 = 32 * half + 4 * j;
-                    *reinterpret_cast<float4*>(smem + P_KBTS + half * P_KB_TP + sw128_off(r, j)) =
-                        tf32x4((i0 + 0 <= r) ? acc[4 * j + 0] : 0.f, (i0 + 1 <= r) ? acc[4 * j + 1] : 0.f,
-                               (i0 + 2 <= r) ? acc[4 * j + 2] : 0.f, (i0 + 3 <= r) ? acc[4 * j + 3] : 0.f);
-                }
-            } else {
-                const int r = 32 * quarter + lane - 64;
-                const float br = beta_s[r];
-                float* mrow = Mf + r * kLd + 32 * half;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int i0 = 32 * half + 4 * j;
-                    *reinterpret_cast<float4*>(mrow + 4 * j) =
-                        make_float4((i0 + 0 < r) ? br * acc[4 * j + 0] : 0.f, (i0 + 1 < r) ? br * acc[4 * j + 1] : 0.f,
-                                    (i0 + 2 < r) ? br * acc[4 * j + 2] : 0.f, (i0 + 3 < r) ? br * acc[4 * j + 3] : 0.f);
-                }
+            for (int j = 0; j < 8; ++j) {
+                const int i0 = 32 * half + 4 * j;
+                *reinterpret_cast<float4*>(mrow + 4 * j) =
+                    make_float4((i0 + 0 < r) ? br * acc[4 * j + 0] : 0.f, (i0 + 1 < r) ? br * acc[4 * j + 1] : 0.f,
+                                (i0 + 2 < r) ? br * acc[4 * j + 2] : 0.f, (i0 + 3 < r) ? br * acc[4 * j + 3] : 0.f);
             }
         }
-        fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
 
-        // ============== T = (I + M)^-1, T' = T diag(beta) -> TP (tf32 operand, rows r, K = i);
-        // meanwhile the store thread sends P to the image
-        ut_inverse64(Mf, Tf, Y1, Y2, tid, [&] {
-            if (tid == kStoreThread) {
-#pragma unroll
-                for (int kb = 0; kb < 2; ++kb)
-                    bulk_store(im + IMG_B2 + kb * KB_B2 + 128 * 128, smem + P_KBTS + kb * P_KB_TP, P_KB_TP);
-                bulk_commit();
-            }
-        });
+        // ============== T = (I + M)^-1, T' = T diag(beta) -> TP (tf32 operand, rows r, K = i)
+        ut_inverse64(Mf, Tf, Y1, Y2, tid, [] {});
         {
             const int r = tid >> 2;
             float4 t4[4], b4[4];
@@ -465,36 +450,66 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
         tc_fence_before();
         __syncthreads();
 
-        // ============== W^T = Kt^T T'^T,  U^T = V^T T'^T
+        // ============== W^T = Kt^T T'^T,  U^T = V^T T'^T  (Kt and V read MN-major)
         if (tid == 0) {
             tc_fence_after();
-            const uint64_t dkt = tdesc(sb, P_KTT), dvt = tdesc(sb, P_VT), dtp = tdesc(sb, P_TP);
+            const uint64_t dkt = sdesc_mn32(sb + P_KTM, P_MN_KB), dv = sdesc_mn32(sb + P_V, P_MN_KB);
+            const uint64_t dtp = tdesc(sb, P_TP);
 #pragma unroll
             for (int s = 0; s < 8; ++s) {
-                mma_tf32_ss(tmem + TP_W, kstep(dkt, P_KB_T, s), kstep(dtp, P_KB_TP, s), ID_N64, s > 0);
-                mma_tf32_ss(tmem + TP_U, kstep(dvt, P_KB_T, s), kstep(dtp, P_KB_TP, s), ID_N64, s > 0);
+                mma_tf32_ss(tmem + TP_W, mn_kstep(dkt, s), kstep(dtp, P_KB_TP, s), ID_N64_AMN, s > 0);
+                mma_tf32_ss(tmem + TP_U, mn_kstep(dv, s), kstep(dtp, P_KB_TP, s), ID_N64_AMN, s > 0);
             }
             mma_commit(bar_mma);
         }
         mma_pending = true;
         if (has_next) prefetch(nxt);
+        if (tid == kStoreThread) {
+            publish();   // the previous item's image (its stores are long complete)
+            if (RING && has_next) done_seen = ld_relaxed_gpu(done_flag(ring, nxt.h));
+        }
+        // ============== meanwhile P (lower incl., tf32, K-major) from TMEM -> X (free
+        // since T' was built): lanes 0-31 by warp 4, lanes 32-63 by warps 1 and 5
+        if (warp == 1 || warp == 4 || warp == 5) {
+            const int r = 32 * quarter + lane;
+            const int hb = warp == 5 ? 1 : 0, he = warp == 1 ? 1 : 2;
+            for (int hh = hb; hh < he; ++hh) {
+                float acc[32];
+                tmem_ld32(tm_lane(tmem, quarter, TP_AP + 32 * hh), acc);
+                tmem_wait_ld();
+                uint8_t* dst = smem + P_X + hh * IMG_BLK;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int i0 = 32 * hh + 4 * j;
+                    *reinterpret_cast<float4*>(dst + sw128_off(r, j)) =
+                        tf32x4((i0 + 0 <= r) ? acc[4 * j + 0] : 0.f, (i0 + 1 <= r) ? acc[4 * j + 1] : 0.f,
+                               (i0 + 2 <= r) ? acc[4 * j + 2] : 0.f, (i0 + 3 <= r) ? acc[4 * j + 3] : 0.f);
+                }
+            }
+        }
+        fence_proxy_async_smem();
         if (!(ok = wait_mma())) break;
+        if (tid == kStoreThread) {
+            bulk_store(im + IMG_P, smem + P_X, 2 * IMG_BLK);
+            bulk_commit();
+        }
 
-        // ============== W (tf32, a 64-row K-major tile) and U ([token][value],
-        // fp32) staged in KTT and VT (their products are done; the next item
-        // rewrites them only after its prep), then bulk-stored to the image
+        // ============== W (tf32, K-major [token][channel]) -> WST and U^T (fp32,
+        // row = value column) -> V (its product is done); then both to the image
         {
             float acc[32];
             const int c = 32 * quarter + lane;   // channel (W) or value column (U)
             tmem_ld32(tm_lane(tmem, quarter, TP_W + 32 * half), acc);
             tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) *K_at(smem, P_KTT, P_KB_KB, 32 * half + j, c) = to_tf32(acc[j]);
+            for (int j = 0; j < 32; ++j) *K_at(smem, P_WST, IMG_BLK, 32 * half + j, c) = to_tf32(acc[j]);
             tmem_ld32(tm_lane(tmem, quarter, TP_U + 32 * half), acc);
             tmem_wait_ld();
-            float* dst = reinterpret_cast<float*>(smem + P_VT) + (32 * half) * kD + c;
+            uint8_t* ut = smem + P_V + half * (2 * IMG_BLK);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) dst[j * kD] = acc[j];
+            for (int j = 0; j < 8; ++j)
+                *reinterpret_cast<float4*>(ut + sw128_off(c, j)) =
+                    make_float4(acc[4 * j], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]);
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -502,20 +517,22 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
         if (tid == kStoreThread) {
 #pragma unroll
             for (int kb = 0; kb < 4; ++kb)
-                bulk_store(im + IMG_B1 + kb * KB_B1 + 64 * 128, smem + P_KTT + kb * P_KB_KB, P_KB_KB);
-            bulk_store(im + IMG_U, smem + P_VT, 32768);
+                bulk_store(im + IMG_B1 + kb * KB_B1 + IMG_BLK, smem + P_WST + kb * IMG_BLK, IMG_BLK);
+            bulk_store(im + IMG_U, smem + P_V, 4 * IMG_BLK);
             bulk_commit();
             if (RING) {
-                pub_flag = ring.ready + cur.h * kRing + (cur.c & (kRing - 1));
+                pub_flag = ready_flag(ring, cur.h, cur.c);
                 pub_val = cur.c + 1;
             }
         }
         cur = nxt;
+        nxt = nxt2;
+        if (w2 + stride < items) nxt2 = decode(w2 + stride);
     }
 
     if (tid == kStoreThread) {
-        if (ok) publish();
         bulk_wait_all();
+        if (ok) publish();
     }
     tc_fence_before();
     __syncthreads();
@@ -532,23 +549,26 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
 }
 
 // ============================================================ pass 2
+// The state pass keeps the image layout: shared-memory offsets equal image offsets.
 constexpr uint32_t S_B1 = 0;          // 64 KB [Qt ; W] of the current chunk
 constexpr uint32_t S_DC = 65536;      // exp(Gamma_C), copied with [Qt ; W]
-constexpr uint32_t S_B2 = 66560;      // 48 KB [Kb^T ; P], then
-constexpr uint32_t S_U = 115712;      //   32 KB U ([token][value] fp32), copied together
+constexpr uint32_t S_KB = 66560;      // 32 KB Kb (MN-major), copied with U, then
+constexpr uint32_t S_P = 99328;       //   16 KB P (K-major)
+constexpr uint32_t S_U = 115712;      // 32 KB U^T
 constexpr uint32_t S_DT = 148480;     // 32 KB delta^T: 128 value rows x 64 tokens, 2 K-blocks x 16 KB
 constexpr uint32_t S_OS = 181248;     // 32 KB O of the previous chunk ([token][value] fp32), TMA store source
 constexpr uint32_t S_MISC = 214016;   // barriers, TMEM slot
 constexpr uint32_t S_SMEM = S_MISC + 1024 + 1024;
-constexpr uint32_t B2U_COPY = B2_COPY + 32768;
-static_assert(S_DC == S_B1 + IMG_DC && S_B2 % 1024 == 0 && S_U == S_B2 + B2_COPY && S_DT % 1024 == 0 &&
-              IMG_U == IMG_B2 + B2_COPY, "layout");
+static_assert(S_B1 == IMG_B1 && S_DC == IMG_DC && S_KB == IMG_KB && S_P == IMG_P && S_U == IMG_U &&
+              S_DT == IMG_BYTES && S_DT % 1024 == 0, "layout");
 
 constexpr uint32_t TS_S = 0;      // 128 cols: S^T fp32 (lane = value column, column = key channel)
 constexpr uint32_t TS_Z = 128;    // 64 cols: Z^T, then O^T (column = token) of even chunks; Y^T follows;
                                   //   odd chunks use the set 256 columns on (384 - 511)
 constexpr uint32_t TS_COLS = 512;
 constexpr uint32_t ID_N128 = idesc_tf32(128, 128, false, false);
+constexpr uint32_t ID_N128_BMN = idesc_tf32(128, 128, false, true);   // B read MN-major
+constexpr int kImgThread = 32;    // waits for the next chunk's image during MMA1 and copies it in
 constexpr int kOutThread = 128;   // issues the O stores, the L2 prefetches and the ring hand-back
                                   // (first thread of the O warps; not the MMA thread)
 
@@ -559,7 +579,7 @@ constexpr int kOutThread = 128;   // issues the O stores, the L2 prefetches and 
 //           tf32; B = [Qt ; W])
 //           meanwhile O of chunk c-1 (set k^1) is read out and staged
 //   delta:  delta^T = U^T - Y_k^T                                  (all warps)
-//   MMA2a:  S^T += delta^T Kb   (the only product the next chunk waits for)
+//   MMA2a:  S^T += delta^T Kb   (Kb read MN-major; the only product the next chunk waits for)
 //   MMA2b:  Z_k^T += delta^T P^T  = O^T of chunk c, read out during chunk c+1
 template <bool RING>
 __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_t* __restrict__ img,
@@ -599,7 +619,7 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
     // ring mode: chunk c's image must be complete before its first copy is issued
     auto await_image = [&](int c) -> bool {
         if (!RING) return true;
-        const bool good = wait_flag_ge(ring.ready + h * kRing + (c & (kRing - 1)), c + 1);
+        const bool good = wait_flag_ge(ready_flag(ring, h, c), c + 1);
         fence_proxy_async_global();
         return good;
     };
@@ -641,24 +661,18 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
         for (int p = 0; p < 4; ++p) bulk_load(smem + S_B1 + p * 16384, src + p * 16384, 16384, bar_b1);
         bulk_load(smem + S_DC, src + IMG_DC, 512, bar_b1);
     };
-    // [Kb^T ; P] and U in two steps on one mbarrier phase (the first step
-    // registers all the bytes): Kb^T and U as soon as MMA2a of the previous
+    // Kb, P and U in two steps on one mbarrier phase (the first step
+    // registers all the bytes): Kb and U as soon as MMA2a of the previous
     // chunk is done, P once MMA2b (which reads P) is done
-    auto load_b2_kbt_u = [&](int c) {
-        mbar_arrive_expect_tx(bar_b2, B2U_COPY);
-        const uint8_t* src = image(c) + IMG_B2;
-#pragma unroll
-        for (int kb = 0; kb < 2; ++kb) bulk_load(smem + S_B2 + kb * KB_B2, src + kb * KB_B2, 128 * 128, bar_b2);
-        bulk_load(smem + S_U, src + B2_COPY, 32768, bar_b2);
+    auto load_b2_kb_u = [&](int c) {
+        mbar_arrive_expect_tx(bar_b2, B2_COPY);
+        const uint8_t* src = image(c);
+        bulk_load(smem + S_KB, src + IMG_KB, 4 * IMG_BLK, bar_b2);
+        bulk_load(smem + S_U, src + IMG_U, 4 * IMG_BLK, bar_b2);
     };
-    auto load_b2_p = [&](int c) {
-        const uint8_t* src = image(c) + IMG_B2;
-#pragma unroll
-        for (int kb = 0; kb < 2; ++kb)
-            bulk_load(smem + S_B2 + kb * KB_B2 + 128 * 128, src + kb * KB_B2 + 128 * 128, 64 * 128, bar_b2);
-    };
+    auto load_b2_p = [&](int c) { bulk_load(smem + S_P, image(c) + IMG_P, 2 * IMG_BLK, bar_b2); };
     auto load_b2 = [&](int c) {
-        load_b2_kbt_u(c);
+        load_b2_kb_u(c);
         load_b2_p(c);
     };
     if (tid == 0 && nch > 0 && (img_ok = await_image(0))) {
@@ -687,7 +701,7 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
             mma_phase ^= 1;
             mma_pending = false;
             tc_fence_after();
-            if (tid == 0) load_b2_kbt_u(c);
+            if (tid == 0) load_b2_kb_u(c);
             b2_pending = true;
             b2_chunk = c;
         }
@@ -730,9 +744,11 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
             mma_commit(bar_mma);
         }
         mma_pending = true;
-        // meanwhile (warps 4-7; thread 0 is busy issuing): O of chunk c-1 (a
-        // full chunk) into the staging tile; its product MMA2b also read P, so
-        // chunk c's copy of P waits for it
+        // meanwhile: the next chunk's image is awaited (its copy waits for MMA1,
+        // which reads the tile it lands in), off the issuing thread
+        if (tid == kImgThread && c + 1 < nch) img_ok = await_image(c + 1);
+        // and (warps 4-7) O of chunk c-1 (a full chunk) goes into the staging
+        // tile; its product MMA2b also read P, so chunk c's copy of P waits for it
         bool o_ok = true;
         if (c > 0 && half == 1) {
             o_ok = mbar_wait_bounded(bar_o, (c - 1) & 1);
@@ -761,20 +777,23 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
             tma_store_3d(tm_o, smem + S_OS, 0, h, static_cast<int32_t>(t_prev));
             bulk_commit();
         }
-        if (tid == 0 && c + 1 < nch && (img_ok = await_image(c + 1))) load_b1(c + 1);
+        if (tid == kImgThread && c + 1 < nch && img_ok) load_b1(c + 1);
         b1_pending = c + 1 < nch;
         b1_chunk = c + 1;
 
         // ---- delta^T = U^T - Y_k^T (tf32 operand, row = value column, K = token);
-        // U came with [Kb^T ; P]
+        // U^T came with Kb
         const bool b2_ok = mbar_wait_bounded(bar_b2, c & 1);
         if (b2_ok) {
             float y[32];
             tmem_ld32(tm_lane(tmem, quarter, zcol(c) + 64 + 32 * half), y);
-            const float* us = reinterpret_cast<const float*>(smem + S_U) + (32 * half) * kD + e;
+            const uint8_t* us = smem + S_U + half * (2 * IMG_BLK);
             float u[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) u[j] = us[j * kD];
+            for (int j = 0; j < 8; ++j) {
+                const float4 x = *reinterpret_cast<const float4*>(us + sw128_off(e, j));
+                u[4 * j] = x.x; u[4 * j + 1] = x.y; u[4 * j + 2] = x.z; u[4 * j + 3] = x.w;
+            }
             tmem_wait_ld();
 #pragma unroll
             for (int j = 0; j < 8; ++j)
@@ -791,24 +810,24 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
         b2_pending = false;
         // chunk c's slot is read: both copies have landed (their mbarriers
         // completed), so the slot can be handed back with a plain store
-        if (RING && tid == kOutThread) st_relaxed_gpu(ring.done + h, c + 1);
+        if (RING && tid == kOutThread) st_relaxed_gpu(done_flag(ring, h), c + 1);
 
         // ---- MMA2a: S^T += delta^T Kb (thread 0);  MMA2b: Z_k^T += delta^T P^T,
         // O of chunk c (kOutThread, so that neither issuing thread is held up
-        // by both)
+        // by both; P of the next chunk is copied in once MMA2b is done)
         if (tid == 0) {
             tc_fence_after();
-            const uint64_t da = tdesc(sb, S_DT), db = tdesc(sb, S_B2);
+            const uint64_t da = tdesc(sb, S_DT), db = sdesc_mn32(sb + S_KB, IMG_BLK);
 #pragma unroll
             for (int s = 0; s < 8; ++s)
-                mma_tf32_ss(tmem + TS_S, kstep(da, 16384, s), kstep(db, KB_B2, s), ID_N128, 1);
+                mma_tf32_ss(tmem + TS_S, kstep(da, 16384, s), mn_kstep(db, s), ID_N128_BMN, 1);
             mma_commit(bar_mma);
         } else if (tid == kOutThread) {
             tc_fence_after();
-            const uint64_t da = tdesc(sb, S_DT), dp = tdesc(sb, S_B2 + 128 * 128);
+            const uint64_t da = tdesc(sb, S_DT), dp = tdesc(sb, S_P);
 #pragma unroll
             for (int s = 0; s < 8; ++s)
-                mma_tf32_ss(tmem + zcol(c), kstep(da, 16384, s), kstep(dp, KB_B2, s), ID_N64, 1);
+                mma_tf32_ss(tmem + zcol(c), kstep(da, 16384, s), kstep(dp, IMG_BLK, s), ID_N64, 1);
             mma_commit(bar_o);
         }
         mma_pending = true;
@@ -913,7 +932,7 @@ size_t index_bytes(int32_t N) { return (static_cast<size_t>(N + 1) * 4 + 1023) &
 constexpr int kMinPrepCtas = 16;
 constexpr int kMaxRingHeads = 96;
 bool ring_eligible(int32_t N, int32_t H) { return N == 1 && H <= kMaxRingHeads; }
-size_t ring_flag_bytes(int32_t H) { return (static_cast<size_t>(H) * (kRing + 1) * 4 + 1023) & ~size_t(1023); }
+size_t ring_flag_bytes(int32_t H) { return (static_cast<size_t>(H) * 2 * kFlagStride * 4 + 1023) & ~size_t(1023); }
 
 template <class K>
 cudaError_t set_smem(K kernel, uint32_t bytes) {
@@ -962,10 +981,10 @@ cudaError_t launch_chunk_two_pass(const PrefillArgs& a, void* scratch, cudaStrea
             return cudaGetLastError();
         if (!coop || per_sm < 1 || a.H + kMinPrepCtas > sms) return cudaErrorNotSupported;
         uint8_t* flags = static_cast<uint8_t*>(scratch) + index_bytes(a.N);
-        Ring ring{reinterpret_cast<int32_t*>(flags), reinterpret_cast<int32_t*>(flags) + a.H * kRing};
+        Ring ring{reinterpret_cast<int32_t*>(flags), reinterpret_cast<int32_t*>(flags) + a.H * kFlagStride};
         uint8_t* img = flags + ring_flag_bytes(a.H);
         kda_chunk_index_kernel<<<1, 1024, 0, stream>>>(a.cu_seqlens, a.N, a.total_T, max_total, chunk_off, a.err,
-                                                       ring.ready, a.H * (kRing + 1));
+                                                       ring.ready, a.H * 2 * kFlagStride);
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(static_cast<unsigned>(sms));
         cfg.blockDim = dim3(kThreads);

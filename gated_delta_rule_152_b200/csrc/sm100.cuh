@@ -41,6 +41,10 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                  ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -113,6 +117,11 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // Wait until every committed group of this thread has completed.
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// The same, leaving the N most recently committed groups pending.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read_but() { asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_all_but() { asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory"); }
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -269,6 +278,11 @@ __device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t* p) {
     asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
+__device__ __forceinline__ int32_t ld_relaxed_gpu(const int32_t* p) {
+    int32_t v;
+    asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
 __device__ __forceinline__ void st_release_gpu(int32_t* p, int32_t v) {
     asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
@@ -282,10 +296,11 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 }
 // Bounded wait until *p >= target (acquire); false if it gave up (after about
 // a second: each poll is an L2 round trip plus a short sleep).
-__device__ __forceinline__ bool wait_flag_ge(const int32_t* p, int32_t target, uint32_t limit = (1u << 21)) {
+__device__ __forceinline__ bool wait_flag_ge(const int32_t* p, int32_t target, uint32_t limit = (1u << 21),
+                                             uint32_t sleep_ns = 64) {
     for (uint32_t i = 0; i < limit; ++i) {
         if (ld_acquire_gpu(p) >= target) return true;
-        __nanosleep(64);
+        __nanosleep(sleep_ns);
     }
     return false;
 }
@@ -326,5 +341,21 @@ __device__ __forceinline__ float ex2(float x) {
 __device__ __forceinline__ uint32_t sw128_off(uint32_t row, uint32_t chunk) {
     return row * 128u + ((chunk ^ (row & 7u)) << 4);
 }
+
+// MN-major tf32 operands take a different form: 128-byte rows (32 elements of
+// the M or N axis) whose 32-byte granules are permuted by the row index mod 4,
+// rows grouped by 4 (512 B).  Byte offset of 16-byte chunk `chunk` (0..7) of
+// row `row`, for a tile based on a 512-byte boundary.
+__device__ __forceinline__ uint32_t sw32g_off(uint32_t row, uint32_t chunk) {
+    return row * 128u + ((((chunk >> 1) ^ (row & 3u)) << 5) | ((chunk & 1u) << 4));
+}
+// Descriptor of such a tile: 32-element blocks of the M (or N) axis lbo bytes
+// apart, 4-row groups of K contiguous (512 B apart); layout type 1.  K step s
+// (8 rows) starts 1 KB further on (mn_kstep).
+__device__ __forceinline__ uint64_t sdesc_mn32(uint32_t smem_addr, uint32_t lbo_bytes) {
+    const uint64_t d = sdesc_sw128(smem_addr, lbo_bytes, 512);
+    return (d & ~(static_cast<uint64_t>(7u) << 61)) | (static_cast<uint64_t>(1u) << 61);
+}
+__device__ __forceinline__ uint64_t mn_kstep(uint64_t d, int s) { return d + 64u * static_cast<uint32_t>(s); }
 
 }  // namespace kda
