@@ -389,6 +389,17 @@ def test_single_sequence_with_many_heads_takes_the_two_launch_path():
     assert_close(s, s_ref, TOL_BF16, "final state")
 
 
+@pytest.mark.parametrize("heads,tokens", [(96, 1280), (1, 2000)])
+def test_overlapped_path_at_the_extremes_of_heads(heads, tokens):
+    # one sequence through the overlapped launch with the most heads it takes
+    # (fewest preparing CTAs) and with one head (most producers waiting for
+    # its ring slots, which wrap many times)
+    x = kin.make_custom_prefill(54, [tokens], heads=heads, init_state_std=0.02)
+    o, s, o_ref, s_ref = run_both(x, heads=sorted({0, heads // 2, heads - 1}))
+    assert_close(o, o_ref, TOL_BF16, "o")
+    assert_close(s, s_ref, TOL_BF16, "final state")
+
+
 def test_prefill_state_pool_rejects_bad_slot():
     dev = torch.device("cuda")
     x = kin.make_custom_prefill(52, [40, 30], heads=2).to(dev)
