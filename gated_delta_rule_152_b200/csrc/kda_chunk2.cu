@@ -155,7 +155,6 @@ constexpr uint32_t TP_COLS = 256;
 constexpr uint32_t ID_N64 = idesc_tf32(128, 64, false, false);
 constexpr uint32_t ID_N64_AMN = idesc_tf32(128, 64, true, false);   // A read MN-major
 
-
 // Overlapped mode (one sequence): the prep role writes each (chunk, head)
 // image into a ring of kRing slots per head instead of its own place in the
 // scratch, and the two roles hand slots over through flags in global memory:
