@@ -188,6 +188,52 @@ def cpu_baseline(x: kin.PrefillInputs, target_s: float = 10.0):
 
 
 # ---------------------------------------------------------------- GPU arm
+def time_prefill_config(spec, dev, stream, steps, warmup, hbm, world):
+    """Device time of one prefill call on another synthetic prefill config
+    (inputs resident in HBM, larger than L2), with its own clock record."""
+    from gated_delta_rule_152_b200 import kda
+    x = kin.make_prefill(spec)
+    xd = x.to(dev)
+    T, H = x.total_T, x.heads
+    N = x.cu_seqlens.numel() - 1
+    o = torch.empty(T, H, D, device=dev)
+    sT = torch.empty(N, H, D, D, device=dev)
+    ws = torch.empty(max(kda.kda_chunk_fwd_workspace_size(N, T, H), 256), dtype=torch.uint8, device=dev)
+
+    def step():
+        kda.kda_chunk_fwd(xd.q, xd.k, xd.v, xd.g, xd.beta, xd.cu_seqlens, initial_state=xd.initial_state,
+                          final_state=sT, o=o, workspace=ws, stream=stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clk = clocks.stop()
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, world)
+    state_io = N * H * STATE_BYTES * (2 if x.initial_state is not None else 1)
+    nbytes = T * H * PREFILL_BYTES_PER_TOKEN_HEAD + state_io
+    gbs = nbytes / (ms / 1e3) / 1e9
+    overlapped = N == 1 and H <= 96
+    del xd, o, sT, ws
+    torch.cuda.empty_cache()
+    return {"workload": spec.name, "value": world * T / (ms / 1e3), "unit": "tokens/s", "ms_per_call": ms,
+            "sequences": N, "tokens": T, "heads": H, "steps": steps, "warmup": warmup,
+            "path": "overlapped" if overlapped else "two-launch (index, prep, state kernels)",
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                         "bytes_per_launch": nbytes},
+            "clocks": clk}, steps * (2 if overlapped else 3)
+
+
 def bench_gpu(args, world, rank, local):
     from gated_delta_rule_152_b200 import kda
     dev = torch.device("cuda", local if world > 1 else 0)
@@ -320,6 +366,13 @@ def bench_gpu(args, world, rank, local):
     del states
     torch.cuda.empty_cache()
 
+    # ---------------- the other prefill configs (not in --quick) -----------
+    extras, extra_launches = {}, 0
+    if not args.quick:
+        for key, xspec in (("long_context", kin.PREFILL_128K), ("varlen", kin.VARLEN_16)):
+            extras[key], n_l = time_prefill_config(xspec, dev, stream, 30, max(args.warmup, 3), hbm, world)
+            extra_launches += n_l
+
     line = {
         "metric": METRIC,
         "value": prefill_tok_s,
@@ -351,9 +404,10 @@ def bench_gpu(args, world, rank, local):
                                 "bytes_per_launch": dec_bytes}},
         "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps * 2 * len(PREFILL_KERNELS) + dsteps,
+        "gpu_launches": args.steps * 2 * len(PREFILL_KERNELS) + dsteps + extra_launches,
         "clocks": clk,
     }
+    line.update(extras)
     if rank == 0 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(x)
     return line
