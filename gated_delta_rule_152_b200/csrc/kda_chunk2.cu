@@ -356,7 +356,7 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
                     make_float4(ex2(GC[0].x), ex2(GC[0].y), ex2(GC[1].x), ex2(GC[1].y));
             if (tid < kC) beta_s[tid] = breg;
         }
-        // the previous item's U has left V, which is rewritten below
+        // the previous item's U and W have left V and WST (V is rewritten below)
         if (tid == kStoreThread) bulk_wait_read();
         fence_proxy_async_smem();
         tc_fence_before();
