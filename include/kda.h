@@ -90,10 +90,13 @@ enum {
 
 /*
  * Bytes of device workspace with which kda_chunk_fwd (and _slots) runs its
- * fastest path for these sizes: the error word, a chunk index, and the
- * state-independent tensor-core operands of every (64-token chunk, head)
- * pair, about 145 KiB per pair (8192 tokens x 32 heads: 608 MB).  Returns 0
- * for invalid sizes.
+ * fastest path for these sizes: the error word, a chunk index, and room for
+ * the state-independent tensor-core operands of the (64-token chunk, head)
+ * pairs, 145 KiB per pair.  One sequence with at most 96 heads needs a ring
+ * of 8 such slots per head plus one 128-byte flag line per head and
+ * direction (32 heads: about 38 MB, whatever the length); otherwise every
+ * pair has its own slot (2 x 8192 tokens x 32 heads: about 613 MB).
+ * Returns 0 for invalid sizes.
  */
 KDA_API size_t kda_chunk_fwd_workspace_size(int32_t N, int64_t total_T, int32_t H, int32_t d,
                                     kda_dtype dt);

@@ -51,6 +51,18 @@ def test_workspace_size(lib):
     assert lib.kda_chunk_fwd_workspace_size(-1, 1000, 32, 128, 0) == 0
 
 
+def test_workspace_size_ring_and_per_pair_scratch(lib):
+    slot = 145 * 1024   # operands of one (64-token chunk, head) pair
+    one = lib.kda_chunk_fwd_workspace_size(1, 8192, 32, 128, 0)
+    assert 32 * 8 * slot <= one < 64 << 20           # one sequence: a ring of 8 slots per head
+    assert lib.kda_chunk_fwd_workspace_size(1, 131072, 32, 128, 0) == one   # independent of length
+    two = lib.kda_chunk_fwd_workspace_size(2, 8192, 32, 128, 0)
+    assert two >= 128 * 32 * slot                    # several sequences: a slot per pair
+    many_heads = lib.kda_chunk_fwd_workspace_size(1, 8192, 100, 128, 0)
+    assert many_heads >= 128 * 100 * slot            # too many heads for the ring
+    assert lib.kda_chunk_fwd_workspace_size_min(1, 8192, 32, 128, 0) < 4096
+
+
 def _chunk(lib, **kw):
     args = dict(q=A, k=A, v=A, g=A, beta=A, cu=A, N=2, T=100, H=4, d=128, dt=0, scale=1.0, flags=1,
                 s0=None, sT=None, o=A, ws=A, wsb=4096, stream=None)
