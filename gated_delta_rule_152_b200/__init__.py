@@ -8,6 +8,7 @@ seeded synthetic workloads.
 from .kda import (  # noqa: F401
     KdaError,
     kda_chunk_fwd,
+    kda_chunk_fwd_noalloc,
     kda_chunk_fwd_slots,
     kda_chunk_fwd_workspace_size,
     kda_chunk_fwd_workspace_size_min,

@@ -35,7 +35,7 @@ KDA_DEVERR_TIMEOUT = 2
 KDA_DEVERR_SLOT = 4
 
 EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd_workspace_size_min", "kda_chunk_fwd",
-            "kda_decode_step",
+            "kda_chunk_fwd_noalloc", "kda_decode_step",
             "kda_chunk_fwd_slots", "kda_decode_step_slots", "kda_verify_fwd", "kda_workspace_error",
             "kda_selftest_bounded_waits",
             "kda_status_string")
@@ -69,6 +69,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.kda_chunk_fwd.argtypes = [P, P, P, P, P, P, I32, I64, I32, I32, ctypes.c_int, F32, U32,
                                       P, P, P, P, SZ, P]
         lib.kda_chunk_fwd.restype = ctypes.c_int
+        lib.kda_chunk_fwd_noalloc.argtypes = [P, P, P, P, P, P, I32, I64, I32, I32, ctypes.c_int, F32, U32,
+                                              P, P, P, P]
+        lib.kda_chunk_fwd_noalloc.restype = ctypes.c_int
         lib.kda_decode_step.argtypes = [P, P, P, P, P, P, P, I32, I32, I32, ctypes.c_int, F32, U32, P]
         lib.kda_decode_step.restype = ctypes.c_int
         lib.kda_chunk_fwd_slots.argtypes = [P, P, P, P, P, P, I32, I64, I32, I32, ctypes.c_int, F32, U32,
@@ -188,6 +191,49 @@ def kda_chunk_fwd(q, k, v, g, beta, cu_seqlens, *, scale: float = 1.0, l2norm: b
                            _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     if st != KDA_OK:
         raise KdaError(st, "kda_chunk_fwd")
+    return o, final_state
+
+
+def kda_chunk_fwd_noalloc(q, k, v, g, beta, cu_seqlens, *, scale: float = 1.0, l2norm: bool = True,
+                          initial_state: Optional[torch.Tensor] = None, final_state=True,
+                          o: Optional[torch.Tensor] = None, recurrent: bool = False,
+                          scalar_decay: bool = False, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """kda_chunk_fwd on the library's built-in scratch instead of a workspace
+    (see the header: at most KDA_NOALLOC_MAX_SEQS sequences, calls on one
+    stream, the first call before any stream capture).  The outputs are
+    allocated here if not given; the library call itself allocates nothing.
+    Same arguments and results as kda_chunk_fwd."""
+    lib = load_library()
+    dev = q.device
+    if dev.type != "cuda":
+        raise ValueError("kda_chunk_fwd_noalloc needs CUDA tensors")
+    T, H, d = q.shape
+    dt = _dtype_code(q)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check(t, name, (T, H, d), q.dtype, dev)
+    _check(g, "g", (T, H) if scalar_decay else (T, H, d), torch.float32, dev)
+    _check(beta, "beta", (T, H), torch.float32, dev)
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 or cu_seqlens.device != dev:
+        raise ValueError("cu_seqlens must be a 1-D int32 tensor on the same device")
+    N = cu_seqlens.numel() - 1
+    if initial_state is not None:
+        _check(initial_state, "initial_state", (N, H, d, d), torch.float32, dev)
+    if final_state is True:
+        final_state = torch.empty((N, H, d, d), dtype=torch.float32, device=dev)
+    elif final_state is False:
+        final_state = None
+    elif final_state is not None:
+        _check(final_state, "final_state", (N, H, d, d), torch.float32, dev)
+    if o is None:
+        o = torch.empty((T, H, d), dtype=torch.float32, device=dev)
+    _check(o, "o", (T, H, d), torch.float32, dev)
+    flags = ((KDA_FLAG_L2NORM_QK if l2norm else 0) | (KDA_FLAG_RECURRENT if recurrent else 0) |
+             (KDA_FLAG_SCALAR_DECAY if scalar_decay else 0))
+    st = lib.kda_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), N, T, H,
+                                   d, dt, float(scale), flags, _ptr(initial_state), _ptr(final_state), _ptr(o),
+                                   _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_chunk_fwd_noalloc")
     return o, final_state
 
 

@@ -131,6 +131,14 @@ def test_binding_rejects_cpu_tensors():
         kda.kda_chunk_fwd(x, x, x, x, torch.zeros(4, 2), torch.tensor([0, 4], dtype=torch.int32))
 
 
+def test_noalloc_binding_rejects_cpu_tensors_and_bad_shapes():
+    import torch
+    x = torch.zeros(4, 2, 128)
+    cu = torch.tensor([0, 4], dtype=torch.int32)
+    with pytest.raises(ValueError):
+        kda.kda_chunk_fwd_noalloc(x, x, x, x, torch.zeros(4, 2), cu)
+
+
 def test_selftest_rejects_bad_workspace(lib):
     P = ctypes.c_void_p
     assert lib.kda_selftest_bounded_waits(None, 256, 16, None) == kda.KDA_ERR_WORKSPACE
