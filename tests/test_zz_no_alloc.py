@@ -73,3 +73,22 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row():
         assert torch.isfinite(o).all() and torch.isfinite(s).all()
         assert _ratio(o, o_ref) <= TOL_BF16
         assert _ratio(s, s_ref) <= TOL_BF16
+
+
+@pytest.mark.gpu
+def test_noalloc_python_binding_matches_the_raw_entry_point():
+    # the Python function of the same name, after the raw entry point above
+    # has done the one-time device set-up: the same bits on the same inputs
+    dev = torch.device("cuda")
+    x = kin.make_custom_prefill(33, [200, 7, 64], heads=2, init_state_std=0.02).to(dev)
+    T, H, d = x.q.shape
+    N = x.cu_seqlens.numel() - 1
+    o, s = kda.kda_chunk_fwd_noalloc(x.q, x.k, x.v, x.g, x.beta, x.cu_seqlens, initial_state=x.initial_state)
+    o2 = torch.full_like(o, float("nan"))
+    s2 = torch.full_like(s, float("nan"))
+    st = _entry()(_p(x.q), _p(x.k), _p(x.v), _p(x.g), _p(x.beta), _p(x.cu_seqlens), N, T, H, d,
+                  kda.KDA_DTYPE_BF16, 1.0, kda.KDA_FLAG_L2NORM_QK, _p(x.initial_state), _p(s2), _p(o2),
+                  ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == kda.KDA_OK
+    torch.cuda.synchronize()
+    assert torch.equal(o, o2) and torch.equal(s, s2)
