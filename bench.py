@@ -336,7 +336,7 @@ def bench_gpu(args, world, rank, local):
         return layer
 
     from concurrent.futures import ThreadPoolExecutor
-    with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as pool:
+    with ThreadPoolExecutor(max_workers=max(1, min(8, (os.cpu_count() or 1) // world))) as pool:
         list(pool.map(fill, range(L)))
     torch.cuda.synchronize(dev)
     toks = [kin.make_decode_tokens(spec, layer).to(dev) for layer in range(L)]
@@ -366,9 +366,10 @@ def bench_gpu(args, world, rank, local):
     del states
     torch.cuda.empty_cache()
 
-    # ---------------- the other prefill configs (not in --quick) -----------
+    # ---------------- the other prefill configs (one GPU, not in --quick) ---
+    # their host inputs take about 10 GB each, too much to hold once per rank
     extras, extra_launches = {}, 0
-    if not args.quick:
+    if not args.quick and world == 1:
         for key, xspec in (("long_context", kin.PREFILL_128K), ("varlen", kin.VARLEN_16)):
             extras[key], n_l = time_prefill_config(xspec, dev, stream, 30, max(args.warmup, 3), hbm, world)
             extra_launches += n_l
