@@ -19,8 +19,13 @@
 // Unrolling the per-token rule inside the chunk gives the triangular system
 // (I + M) delta = diag(beta) (V - Y) for the rank-one corrections delta_r,
 // from which the outputs and the end state follow.  Every exponent is taken
-// relative to the chunk end, so all factors are finite as long as a channel's
-// decay inside one chunk, -sum(g), stays below ~87.
+// relative to the chunk end, so the factors stay inside the fp32 range while a
+// channel's decay inside one chunk, -sum(g), stays below 100 log2 units (about
+// 69 nats; level 0 of kda_tile.cuh).  A chunk that decays more in some
+// channel -- the page lets every channel decay at its own data-dependent
+// rate, so nothing bounds it -- sends its (sequence, head, slice) to the
+// token-by-token recurrence (serial_slice, kda_serial.cuh), which restarts from
+// the initial state; the two-pass kernels handle such chunks in place.
 //
 // Precision: operands are rounded to tf32 (10-bit mantissa) and accumulated in
 // fp32.  bf16 operands were measured (CPU emulation against the fp64 oracle)
@@ -40,6 +45,7 @@
 // touch tensor-memory lanes 32*(warp%4) .. +31.
 #include "kda_common.cuh"
 #include "kda_launch.h"
+#include "kda_serial.cuh"
 #include "kda_tile.cuh"
 #include "sm100.cuh"
 
@@ -95,6 +101,7 @@ constexpr uint32_t ID_N32 = idesc_tf32(128, 32, false, false);
 
 __global__ void __launch_bounds__(kThreads, 1)
 kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                  const __nv_bfloat16* __restrict__ v, const float* __restrict__ g,
                  const float* __restrict__ beta, const int32_t* __restrict__ cu_seqlens,
                  int64_t total_T, int H, float scale, int l2norm, int scalar_g, const float* s0,
@@ -203,19 +210,25 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
     // Prep of one chunk (state independent): Gamma, L2 norms, the tf32 tiles
     // Kt, Qt (XQ), Kb (rows 0-63 of KS) and V^T, plus beta and exp(Gamma_C).
-    // Contains one block barrier; every thread must call it.
-    auto prep = [&](int L) {
-        float2 GC[2];
-        prep_chunk_rows(smem + OFF_KS, smem + OFF_KS + kC * kD * 2, greg, xch, L, scale, l2norm != 0, GC,
-                        [&](int r, int kbi, int ch, float4 kt, float4 qt, float4 kb) {
-                            st_tf32x4(smem, OFF_XQ + kbi * KB_XQ + sw128_off(r, ch), kt.x, kt.y, kt.z, kt.w);
-                            st_tf32x4(smem, OFF_XQ + kbi * KB_XQ + sw128_off(64 + r, ch), qt.x, qt.y, qt.z, qt.w);
-                            st_tf32x4(smem, OFF_KS + kbi * KB_KS + sw128_off(r, ch), kb.x, kb.y, kb.z, kb.w);
-                        });
-        if (warp == 0) {
-            dc_s[4 * lane + 0] = ex2(GC[0].x); dc_s[4 * lane + 1] = ex2(GC[0].y);
-            dc_s[4 * lane + 2] = ex2(GC[1].x); dc_s[4 * lane + 3] = ex2(GC[1].y);
-        }
+    // Returns the chunk's Gram level (kda_tile.cuh); this kernel's single
+    // reference point per chunk serves level 0 only.  Contains one block
+    // barrier; every thread must call it.
+    auto prep = [&](int L) -> int {
+        float4 gc;
+        const int level = prep_chunk_rows(
+            smem + OFF_KS, smem + OFF_KS + kC * kD * 2, greg, xch, L, scale, l2norm != 0,
+            [&](const ChunkChannels& cc, int) { gc = cc.rho[3]; },
+            [&](int r, int kbi, int ch, float4 qn, float4 kn, float4 gr) {
+            // a = Gamma_r - Gamma_C >= 0 (the decay is cumulative, g <= 0): E = 2^a >= 1, F = 2^-a <= 1
+            const float4 a = sub4(gr, gc);
+            const float4 E = ex2x4(make_float4(fminf(a.x, 126.f), fminf(a.y, 126.f), fminf(a.z, 126.f), fminf(a.w, 126.f)));
+            const float4 F = ex2x4(make_float4(-a.x, -a.y, -a.z, -a.w));
+            const float4 kt = mul4(kn, E), qt = mul4(qn, E), kb = mul4(kn, F);
+            st_tf32x4(smem, OFF_XQ + kbi * KB_XQ + sw128_off(r, ch), kt.x, kt.y, kt.z, kt.w);
+            st_tf32x4(smem, OFF_XQ + kbi * KB_XQ + sw128_off(64 + r, ch), qt.x, qt.y, qt.z, qt.w);
+            st_tf32x4(smem, OFF_KS + kbi * KB_KS + sw128_off(r, ch), kb.x, kb.y, kb.z, kb.w);
+        });
+        if (warp == 0) *reinterpret_cast<float4*>(dc_s + 4 * lane) = ex2x4(gc);
         if (tid < kC) beta_s[tid] = breg;
         {   // V^T: token tid/4, value columns 8*(tid%4) .. +7 (exact bf16 -> fp32)
             const int r = tid >> 2, j0 = 8 * (tid & 3);
@@ -226,6 +239,7 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 *K_at(smem, OFF_VT, KB_VT, j0 + 2 * x + 1, r) = __uint_as_float(w4[x] & 0xFFFF0000u);
             }
         }
+        return level;
     };
 
     bool ok = true;
@@ -241,6 +255,10 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         return good;
     };
 
+    // level of the chunk prepared last: a chunk whose decay is too strong for the
+    // chunk-end reference point sends the whole (sequence, head, slice) to the
+    // token-by-token recurrence instead (serial_slice, from the initial state)
+    int lvl_next = 0;
     if (nchunks > 0) {   // prologue: stage and prep chunk 0
         if (tid == 0) issue_load(bos);
         load_pending = true;
@@ -248,11 +266,16 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         ok = !__syncthreads_or(!mbar_wait_bounded(bar_load, 0));
         if (ok) {
             load_pending = false;
-            prep(static_cast<int>(len < kC ? len : (int64_t)kC));
+            lvl_next = prep(static_cast<int>(len < kC ? len : (int64_t)kC));
         }
     }
 
+    bool serial = false;
     for (int c = 0; ok && c < nchunks; ++c) {
+        if (lvl_next != 0) {   // nothing is in flight here: chunk c's load was consumed by its prep
+            serial = true;
+            break;
+        }
         const int64_t t0 = bos + (int64_t)c * kC;
         const int L = static_cast<int>(eos - t0 < kC ? eos - t0 : (int64_t)kC);
         const bool has_next = c + 1 < nchunks;
@@ -437,7 +460,7 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (has_next) {
             if (!(ok = !__syncthreads_or(!mbar_wait_bounded(bar_load, (c + 1) & 1)))) break;
             load_pending = false;
-            prep(Ln);
+            lvl_next = prep(Ln);
         }
         if (!(ok = wait_mma())) break;
 
@@ -458,7 +481,14 @@ kda_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
     tc_fence_before();
     __syncthreads();
-    if (ok) {
+    if (ok && serial) {
+        // the recurrence over the whole sequence from the initial state (which this
+        // CTA has not written yet), in the now idle shared memory
+        if (warp < 4)
+            serial_slice(q, k, v, g, beta, bos, eos, H, h, slice, scale, l2norm != 0, scalar_g != 0, s0, sT, state_off,
+                         o, nullptr, reinterpret_cast<float*>(smem), tid, 1u);
+        __syncthreads();
+    } else if (ok) {
         if (sT && warp < 4) {
             float acc[32];
             tc_fence_after();
@@ -536,7 +566,8 @@ cudaError_t launch_chunk(const PrefillArgs& a, cudaStream_t stream) {
         return cudaErrorInvalidValue;
     const long long blocks = (long long)a.N * a.H * kSplit;
     kda_chunk_kernel<<<static_cast<unsigned>(blocks), kThreads, SMEM_BYTES, stream>>>(
-        mq, mk, static_cast<const __nv_bfloat16*>(a.v), a.g, a.beta, a.cu_seqlens, a.total_T, a.H, a.scale,
+        mq, mk, static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
+        static_cast<const __nv_bfloat16*>(a.v), a.g, a.beta, a.cu_seqlens, a.total_T, a.H, a.scale,
         a.l2norm ? 1 : 0, a.scalar_decay ? 1 : 0, a.initial_state, a.final_state, a.o, a.err, a.slots,
         a.num_slots);
     return cudaGetLastError();

@@ -5,20 +5,29 @@
 // layer remember without rereading?"):
 //     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,
 //     o_t = scale * S_t^T q_t.
-// Evaluated 64 tokens at a time with the chunk algebra of kda_chunk.cu
-// (Gamma, E, F, Kt, Qt, Kb, A, P, M, T' as defined there).  With
-//     W = T' Kt   and   U = T' V,
-// the correction of a chunk is delta = T' (V - Kt St) = U - W St, so
-//     O = Qt St + P delta,    S_next = St + Kb^T delta,    St = Diag(e^Gamma_C) S.
+// Evaluated 64 tokens at a time.  For one chunk with entry state S (rows =
+// key channels), Gamma_r = g_0 + ... + g_r per channel and Gamma_C its value
+// at the chunk's last token, the state side takes every exponent relative to
+// the chunk START, so each of its factors lies in (0, 1] whatever the decay:
+//     Qs = scale q^ e^Gamma_r,  Ks = k^ e^Gamma_r,  Kb = k^ e^(Gamma_C - Gamma_r),
+//     T' = (I + strict_lower(diag(beta) A))^-1 diag(beta),  P = lower_incl(...),
+//     W = T' Ks,  U = T' V,
+//     delta = U - W S,   O = Qs S + P delta,   S_next = Diag(e^Gamma_C) S + Kb^T delta,
+// with A_ri = sum_c k^_rc k^_ic e^(Gamma_rc - Gamma_ic) and P_ri the same with
+// scale q^_r: the intra-chunk Gram matrices, taken at the level the chunk's
+// decay allows (kda_tile.cuh: one tensor-core product through the chunk end,
+// 16-token block references, or pairwise exponentials).  Unrolling the
+// per-token rule inside the chunk gives (I + M) delta = diag(beta)(V - Ks S)
+// for the rank-one corrections delta_r, from which O and S_next follow.
 // Everything except the last line is independent of the state.  Pass 1
 // (kda_chunk_prep_kernel) therefore runs over all (chunk, head) pairs in
 // parallel and writes, per pair, ready-made tensor-core operand images of
-// [Qt ; W], Kb and P, and U and e^Gamma_C, to scratch.  Pass 2
+// [Qs ; W], Kb and P, and U and e^Gamma_C, to scratch.  Pass 2
 // (kda_chunk_state_kernel) walks the chunks of one (sequence, head) in order
 // and only carries the state:
-//     [Z^T | Y^T] = St^T [Qt ; W]^T            (M = 128 value columns, N = 128)
-//     delta^T = U^T - Y^T
-//     S_next^T = St^T + delta^T Kb,   O^T = Z^T + delta^T P^T
+//     [Z^T | Y^T] = S^T [Qs ; W]^T             (M = 128 value columns, N = 128)
+//     delta^T = U^T - Y^T,   S^T <- S^T Diag(e^Gamma_C)
+//     S_next^T = S^T + delta^T Kb,   O^T = Z^T + delta^T P^T
 // The state is kept transposed in tensor memory (lane = value column, column
 // = key channel), so it is the A operand of the first products and the
 // accumulator of the update, and the readout O^T lands with the value
@@ -28,11 +37,11 @@
 // contiguous) permute 16-byte chunks by the row index mod 8; MN-major tf32
 // tiles (the other axis contiguous), which the tensor core reads with a
 // different swizzle, permute 32-byte granules by the row index mod 4.  Pass 1
-// writes Kt, Kb and V in the token-row orientation it produces them in and
+// writes Ks, Kb and V in the token-row orientation it produces them in and
 // lets the products read them MN-major, so no tile is transposed.
 //
 // Precision: as the fused kernel -- tf32 operands (rounded to nearest),
-// fp32 accumulation, fp32 state; U is kept in fp32.
+// fp32 accumulation, fp32 state (decayed on CUDA cores); U is kept in fp32.
 #include "kda_common.cuh"
 #include "kda_launch.h"
 #include "kda_tile.cuh"
@@ -48,7 +57,7 @@ constexpr int kThreads = 256;
 
 // ---- per (chunk, head) operand image in scratch (byte offsets), tiles
 // exactly as the state pass holds them in shared memory.
-constexpr uint32_t IMG_B1 = 0;        // [Qt ; W]: rows 0-63 Qt, 64-127 W (token) x 128 channels, K-major,
+constexpr uint32_t IMG_B1 = 0;        // [Qs ; W]: rows 0-63 Qs, 64-127 W (token) x 128 channels, K-major,
                                       //   4 K-blocks x 16 KB
 constexpr uint32_t IMG_DC = 65536;    // exp(Gamma_C): 128 fp32 (+ 512 B pad)
 constexpr uint32_t IMG_KB = 66560;    // Kb: 64 token rows x 128 channels, MN-major, 4 blocks of 32 channels x 8 KB
@@ -56,8 +65,8 @@ constexpr uint32_t IMG_P = 99328;     // P: 64 token rows x 64 tokens, K-major, 
 constexpr uint32_t IMG_U = 115712;    // U^T: 128 value rows x 64 tokens fp32, 16-byte chunks permuted as
                                       //   K-major tiles, 2 blocks of 32 tokens x 16 KB
 constexpr uint32_t IMG_BYTES = 148480;
-constexpr uint32_t KB_B1 = 16384, IMG_BLK = 8192;   // K-block of [Qt ; W]; 64 rows x 128 B
-constexpr uint32_t B1_COPY = IMG_DC + 512;   // [Qt ; W] and exp(Gamma_C) in one copy
+constexpr uint32_t KB_B1 = 16384, IMG_BLK = 8192;   // K-block of [Qs ; W]; 64 rows x 128 B
+constexpr uint32_t B1_COPY = IMG_DC + 512;   // [Qs ; W] and exp(Gamma_C) in one copy
 constexpr uint32_t B2_COPY = IMG_BYTES - IMG_KB;   // Kb, P and U on one mbarrier phase
 static_assert(IMG_KB % 1024 == 0 && IMG_P == IMG_KB + 32768 && IMG_U == IMG_P + 16384 &&
               IMG_BYTES == IMG_U + 32768, "image layout");
@@ -127,15 +136,18 @@ __global__ void __launch_bounds__(1024) kda_chunk_index_kernel(const int32_t* __
 
 // ============================================================ pass 1
 // Shared memory (byte offsets from a 1024-aligned base).
-constexpr uint32_t P_X = 0;          // 64 KB [Qt ; Kt]: 128 rows x 128 channels, K-major, 4 K-blocks x 16 KB
-                                     //   (A of the Gram product).  After it: the triangular-solve scratch
-                                     //   (from 0), T' (at P_TP), then P on its way to the image (from 0)
+constexpr uint32_t P_X = 0;          // 64 KB Gram operand: 128 rows (Q-side, K-side) x 128 channels, K-major,
+                                     //   4 K-blocks x 16 KB.  After it: [P ; A] staging (levels 1, 2), the
+                                     //   triangular-solve scratch (from 0), T' (at P_TP), then P on its way
+                                     //   to the image (from 0)
 constexpr uint32_t P_TP = 49152;     // 16 KB T': 64 rows (token r) x 64 (token i), K-major, 2 K-blocks x 8 KB
-constexpr uint32_t P_KB = 65536;     // 32 KB Kb: 64 rows x 128 channels, K-major, 4 K-blocks x 8 KB; also the
-                                     //   TMA destination of the next item's raw q (16 KB) and k (16 KB)
-constexpr uint32_t P_KTM = 98304;    // 32 KB Kt MN-major: 64 token rows x 128 channels, 4 blocks x 8 KB
-                                     //   (Kt^T for W^T)
-constexpr uint32_t P_WST = 131072;   // 32 KB W (K-major, 4 K-blocks x 8 KB) on its way to the image
+constexpr uint32_t P_KB = 65536;     // 32 KB second Gram operand: 64 rows x 128 channels, K-major, 4 K-blocks
+                                     //   x 8 KB; also the TMA destination of the next item's raw q (16 KB)
+                                     //   and k (16 KB)
+constexpr uint32_t P_KTM = 98304;    // 32 KB Ks MN-major: 64 token rows x 128 channels, 4 blocks x 8 KB
+                                     //   (Ks^T for W^T)
+constexpr uint32_t P_WST = 131072;   // 32 KB W (K-major, 4 K-blocks x 8 KB) on its way to the image; before
+                                     //   that the exact Gram's Z table (levels 1, 2)
 constexpr uint32_t P_V = 163840;     // 32 KB V MN-major: 64 token rows x 128 values, 4 blocks x 8 KB
                                      //   (V^T for U^T); then U^T on its way out
 constexpr uint32_t P_RV = 196608;    // 16 KB raw v (bf16 [64 tokens][128])
@@ -245,7 +257,7 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
                                  : static_cast<size_t>(it.gc) * H + it.h;
         return img + slot * IMG_BYTES;
     };
-    // ring mode: the image of an item (Qt, Kb and exp(Gamma_C) written with
+    // ring mode: the image of an item (Qs, Kb and exp(Gamma_C) written with
     // plain stores before the item's block barriers, the rest by bulk stores)
     // is announced by the store thread once those bulk stores have completed:
     // a proxy fence, then a gpu-scope release, which also covers the plain
@@ -334,26 +346,72 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
         load_pending = false;
         load_parity ^= 1;
 
-        // ============== prep: [Qt ; Kt] -> X, Kb -> KB (K-major), Kt -> KTM (MN-major);
-        // Qt (K-major), Kb (MN-major) and exp(Gamma_C) -> image (a warp stores four
-        // whole 128-byte rows at a time)
+        // ============== prep.  The state side takes the chunk-start form (every factor in
+        // (0, 1]): Qs = q^ 2^Gamma_r -> image rows 0-63 of [Qs ; W] (K-major), Ks = k^ 2^Gamma_r
+        // -> KTM (MN-major, for W), Kb = k^ 2^(Gamma_C - Gamma_r) -> image (MN-major), and
+        // 2^Gamma_C -> image.  The Gram operands in X (128 rows, Q-side then K-side) and KB
+        // (64 rows), both K-major, depend on the chunk's level (kda_tile.cuh):
+        //   0: [Qs ; Ks] 2^-Gamma_C and Kb, tf32 (the tensor-core product through the chunk end);
+        //   1: [q^ X ; k^ X] and k^ Y, fp32 (block references);
+        //   2: [q^ ; k^] and Gamma, fp32.
+        // A warp stores four whole 128-byte rows of the image at a time.
+        int level = 0;
+        float4 rho0, rho1, rho2, rho3;   // block ends of the thread's channels (for the exact Gram's table)
         {
-            float2 GC[2];
-            prep_chunk_rows(smem + P_KB, smem + P_KB + kC * kD * 2, greg, xch, L, scale, l2norm != 0, GC,
-                            [&](int r, int kbi, int ch, float4 kt, float4 qt, float4 kb) {
-                                const float4 q4 = tf32x4(qt.x, qt.y, qt.z, qt.w);
-                                const float4 k4 = tf32x4(kt.x, kt.y, kt.z, kt.w);
-                                const float4 b4 = tf32x4(kb.x, kb.y, kb.z, kb.w);
-                                *reinterpret_cast<float4*>(smem + P_X + kbi * KB_B1 + sw128_off(r, ch)) = q4;
-                                *reinterpret_cast<float4*>(smem + P_X + kbi * KB_B1 + sw128_off(64 + r, ch)) = k4;
-                                *reinterpret_cast<float4*>(smem + P_KB + kbi * P_KB_KB + sw128_off(r, ch)) = b4;
-                                *reinterpret_cast<float4*>(smem + P_KTM + kbi * P_MN_KB + sw32g_off(r, ch)) = k4;
-                                *reinterpret_cast<float4*>(im + IMG_B1 + kbi * KB_B1 + sw128_off(r, ch)) = q4;
-                                *reinterpret_cast<float4*>(im + IMG_KB + kbi * IMG_BLK + sw32g_off(r, ch)) = b4;
-                            });
-            if (warp == 0)
-                *reinterpret_cast<float4*>(im + IMG_DC + 16 * lane) =
-                    make_float4(ex2(GC[0].x), ex2(GC[0].y), ex2(GC[1].x), ex2(GC[1].y));
+            // per-channel factors: 2^-Gamma_C (level 0); 2^rho_{a-1} and 2^(Gamma_C - rho_a) of the
+            // thread's block a = warp / 2 (level 1)
+            float4 gc, bprev, bcur, inv, es, ef;
+            auto setup = [&](const ChunkChannels& cc, int lvl) {
+                level = lvl;
+                gc = cc.rho[3];
+                bprev = cc.bstart;
+                bcur = cc.bend;
+                rho0 = cc.rho[0];
+                rho1 = cc.rho[1];
+                rho2 = cc.rho[2];
+                rho3 = cc.rho[3];
+                inv = ex2x4(make_float4(fminf(-gc.x, 126.f), fminf(-gc.y, 126.f), fminf(-gc.z, 126.f),
+                                        fminf(-gc.w, 126.f)));
+                es = ex2x4(bprev);
+                ef = ex2x4(sub4(gc, bcur));
+            };
+            prep_chunk_rows(smem + P_KB, smem + P_KB + kC * kD * 2, greg, xch, L, scale, l2norm != 0, setup,
+                            [&](int r, int kbi, int ch, float4 qn, float4 kn, float4 gr) {
+                float4 qs, ks, kb, xq, xk, y;
+                if (level == 1) {
+                    const float4 X = ex2x4(sub4(gr, bprev)), Y = ex2x4(sub4(bcur, gr));
+                    xq = mul4(qn, X);
+                    xk = mul4(kn, X);
+                    y = mul4(kn, Y);
+                    qs = mul4(xq, es);
+                    ks = mul4(xk, es);
+                    kb = mul4(y, ef);
+                } else {
+                    const float4 e0 = ex2x4(gr), f = ex2x4(sub4(gc, gr));
+                    qs = mul4(qn, e0);
+                    ks = mul4(kn, e0);
+                    kb = mul4(kn, f);
+                    if (level == 0) {
+                        xq = tf32x4(qs.x * inv.x, qs.y * inv.y, qs.z * inv.z, qs.w * inv.w);
+                        xk = tf32x4(ks.x * inv.x, ks.y * inv.y, ks.z * inv.z, ks.w * inv.w);
+                        y = tf32x4(kb.x, kb.y, kb.z, kb.w);
+                    } else {
+                        xq = qn;
+                        xk = kn;
+                        y = gr;
+                    }
+                }
+                const float4 q4 = tf32x4(qs.x, qs.y, qs.z, qs.w);
+                const float4 k4 = tf32x4(ks.x, ks.y, ks.z, ks.w);
+                const float4 b4 = tf32x4(kb.x, kb.y, kb.z, kb.w);
+                *reinterpret_cast<float4*>(smem + P_X + kbi * KB_B1 + sw128_off(r, ch)) = xq;
+                *reinterpret_cast<float4*>(smem + P_X + kbi * KB_B1 + sw128_off(64 + r, ch)) = xk;
+                *reinterpret_cast<float4*>(smem + P_KB + kbi * P_KB_KB + sw128_off(r, ch)) = y;
+                *reinterpret_cast<float4*>(smem + P_KTM + kbi * P_MN_KB + sw32g_off(r, ch)) = k4;
+                *reinterpret_cast<float4*>(im + IMG_B1 + kbi * KB_B1 + sw128_off(r, ch)) = q4;
+                *reinterpret_cast<float4*>(im + IMG_KB + kbi * IMG_BLK + sw32g_off(r, ch)) = b4;
+            });
+            if (warp == 0) *reinterpret_cast<float4*>(im + IMG_DC + 16 * lane) = ex2x4(gc);
             if (tid < kC) beta_s[tid] = breg;
         }
         // the previous item's U and W have left V and WST (V is rewritten below)
@@ -362,8 +420,10 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
         tc_fence_before();
         __syncthreads();
 
-        // ============== [Qt ; Kt] x Kb^T -> P (lanes 0-63), A (lanes 64-127)
-        if (tid == 0) {
+        // ============== [P ; A]: level 0 by one tensor-core product [Qs ; Ks] 2^-Gamma_C x Kb^T
+        // (P in lanes 0-63, A in lanes 64-127 of TP_AP), levels 1 and 2 on CUDA cores and
+        // mma.sync (gram_exact), staged into the same tensor-memory columns
+        if (level == 0 && tid == 0) {
             tc_fence_after();
             const uint64_t dx = tdesc(sb, P_X), dkb = tdesc(sb, P_KB);
 #pragma unroll
@@ -371,7 +431,13 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
                 mma_tf32_ss(tmem + TP_AP, kstep(dx, KB_B1, s), kstep(dkb, P_KB_KB, s), ID_N64, s > 0);
             mma_commit(bar_mma);
         }
-        mma_pending = true;
+        if (level == 0) mma_pending = true;
+        if (level != 0 && warp == 0) {   // block ends of the thread's channels -> [4][128] table in xch
+            *reinterpret_cast<float4*>(xch + 0 * kD + 4 * lane) = rho0;
+            *reinterpret_cast<float4*>(xch + 1 * kD + 4 * lane) = rho1;
+            *reinterpret_cast<float4*>(xch + 2 * kD + 4 * lane) = rho2;
+            *reinterpret_cast<float4*>(xch + 3 * kD + 4 * lane) = rho3;
+        }
         // ============== meanwhile: V (MN-major; bf16 is exact in tf32) from the raw
         // tile, rows past L zero; a 32-byte granule holds the 8 values of a raw chunk
 #pragma unroll
@@ -388,18 +454,44 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
                             __uint_as_float(u.w << 16), __uint_as_float(u.w & 0xFFFF0000u));
         }
         fence_proxy_async_smem();
-        if (!(ok = wait_mma())) break;
-        // KB and RV are free: stage the next item's raw q, k, v, and bring the
-        // item after it (its q, k, v and g) into L2 so that its loads find it there
-        if (tid == 0 && has_next) {
-            issue_load(nxt);
-            if (has_next2) {
-                const int32_t t2 = static_cast<int32_t>(nxt2.t0);
-                tma_prefetch_3d(tm_q, 0, nxt2.h, t2);
-                tma_prefetch_3d(tm_k, 0, nxt2.h, t2);
-                tma_prefetch_3d(tm_v, 0, nxt2.h, t2);
-                if (!scalar_g) tma_prefetch_3d(tm_g, 0, nxt2.h, t2);
+        // KB and RV are free once the Gram inputs are read: stage the next item's raw
+        // q, k, v, and bring the item after it (its q, k, v and g) into L2 so that its
+        // loads find it there
+        auto next_loads = [&]() {
+            if (tid == 0 && has_next) {
+                issue_load(nxt);
+                if (has_next2) {
+                    const int32_t t2 = static_cast<int32_t>(nxt2.t0);
+                    tma_prefetch_3d(tm_q, 0, nxt2.h, t2);
+                    tma_prefetch_3d(tm_k, 0, nxt2.h, t2);
+                    tma_prefetch_3d(tm_v, 0, nxt2.h, t2);
+                    if (!scalar_g) tma_prefetch_3d(tm_g, 0, nxt2.h, t2);
+                }
             }
+        };
+        if (level == 0) {
+            if (!(ok = wait_mma())) break;
+            next_loads();
+        } else {
+            __syncthreads();   // the block-end table is written
+            float* st = reinterpret_cast<float*>(smem + P_X);
+            gram_exact(smem + P_X, KB_B1, smem + P_KB, P_KB_KB, xch, reinterpret_cast<float*>(smem + P_WST), st,
+                       level, tid, next_loads);
+            // [P ; A] -> tensor memory: lane quarter q, value columns 32 * half ..
+            {
+                float acc[32];
+                const float* row = st + (32 * quarter + lane) * kStLd + 32 * half;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float4 x = *reinterpret_cast<const float4*>(row + 4 * j);
+                    acc[4 * j] = x.x; acc[4 * j + 1] = x.y; acc[4 * j + 2] = x.z; acc[4 * j + 3] = x.w;
+                }
+                tmem_st32(tm_lane(tmem, quarter, TP_AP + 32 * half), acc);
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            __syncthreads();
+            tc_fence_after();
         }
         load_pending = has_next;
 
@@ -449,7 +541,7 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
         tc_fence_before();
         __syncthreads();
 
-        // ============== W^T = Kt^T T'^T,  U^T = V^T T'^T  (Kt and V read MN-major)
+        // ============== W^T = Ks^T T'^T,  U^T = V^T T'^T  (Ks and V read MN-major)
         if (tid == 0) {
             tc_fence_after();
             const uint64_t dkt = sdesc_mn32(sb + P_KTM, P_MN_KB), dv = sdesc_mn32(sb + P_V, P_MN_KB);
@@ -549,8 +641,8 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
 
 // ============================================================ pass 2
 // The state pass keeps the image layout: shared-memory offsets equal image offsets.
-constexpr uint32_t S_B1 = 0;          // 64 KB [Qt ; W] of the current chunk
-constexpr uint32_t S_DC = 65536;      // exp(Gamma_C), copied with [Qt ; W]
+constexpr uint32_t S_B1 = 0;          // 64 KB [Qs ; W] of the current chunk
+constexpr uint32_t S_DC = 65536;      // exp(Gamma_C), copied with [Qs ; W]
 constexpr uint32_t S_KB = 66560;      // 32 KB Kb (MN-major), copied with U, then
 constexpr uint32_t S_P = 99328;       //   16 KB P (K-major)
 constexpr uint32_t S_U = 115712;      // 32 KB U^T
@@ -573,10 +665,10 @@ constexpr int kOutThread = 128;   // issues the O stores, the L2 prefetches and 
 
 // Pass 2 for sequence n, head h.  Per chunk c (k = c % 2 selects one of two
 // Z/Y column sets in TMEM):
-//   decay:  St = Diag(e^Gamma_C) S in place in TMEM (fp32)         (all warps)
-//   MMA1:   [Z_k | Y_k] = St^T [Qt ; W]^T        (A = the state in TMEM, read as
-//           tf32; B = [Qt ; W])
+//   MMA1:   [Z_k | Y_k] = S^T [Qs ; W]^T         (A = the state at the chunk start in
+//           TMEM, read as tf32; B = [Qs ; W])
 //           meanwhile O of chunk c-1 (set k^1) is read out and staged
+//   decay:  S = Diag(e^Gamma_C) S in place in TMEM (fp32)          (all warps)
 //   delta:  delta^T = U^T - Y_k^T                                  (all warps)
 //   MMA2a:  S^T += delta^T Kb   (Kb read MN-major; the only product the next chunk waits for)
 //   MMA2b:  Z_k^T += delta^T P^T  = O^T of chunk c, read out during chunk c+1
@@ -595,6 +687,7 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
     uint64_t* bar_o = bar_b1 + 3;     // MMA2b of every chunk
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_b1 + 4);
     const float* dc_s = reinterpret_cast<const float*>(smem + S_DC);
+    float* dc_keep = reinterpret_cast<float*>(smem + S_MISC + 512);   // 2^Gamma_C of the current chunk
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quarter = warp & 3, half = warp >> 2;
@@ -674,9 +767,12 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
         load_b2_kb_u(c);
         load_b2_p(c);
     };
-    if (tid == 0 && nch > 0 && (img_ok = await_image(0))) {
-        load_b1(0);
-        load_b2(0);
+    if (tid == 0 && nch > 0) {
+        img_ok = await_image(0);
+        if (img_ok) {
+            load_b1(0);
+            load_b2(0);
+        }
     }
     // in-flight copies and products: pending flag and the chunk (parity) they belong to
     bool ok = !__syncthreads_or(!img_ok);
@@ -706,34 +802,18 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
         }
         if (!RING && tid == kOutThread && c + 2 < nch) prefetch_l2(image(c + 2), IMG_BYTES);
         if (tid == kOutThread) bulk_wait_read();   // the O staging tile is rewritten below
-        // decay (key channels 64*half ..) in place; the fp32 state is also the A
-        // operand of MMA1, which reads it as tf32 (the low mantissa bits are
-        // dropped; measured on the CPU against the fp64 oracle: no change in the
-        // error of o or S); it needs exp(Gamma_C), which comes with [Qt ; W]
+        // [Qs ; W] and 2^Gamma_C of chunk c have landed; 2^Gamma_C is kept aside for
+        // the decay after MMA1 (the next chunk's copy lands on top of it before then)
         const bool b1_ok = mbar_wait_bounded(bar_b1, c & 1);
-        if (b1_ok) {
-            float st[2][32];
-#pragma unroll
-            for (int part = 0; part < 2; ++part) tmem_ld32(tm_lane(tmem, quarter, TS_S + 64 * half + 32 * part), st[part]);
-            tmem_wait_ld();
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                const int c0 = 64 * half + 32 * part;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const float4 d4 = *reinterpret_cast<const float4*>(dc_s + c0 + 4 * j);
-                    st[part][4 * j] *= d4.x; st[part][4 * j + 1] *= d4.y;
-                    st[part][4 * j + 2] *= d4.z; st[part][4 * j + 3] *= d4.w;
-                }
-                tmem_st32(tm_lane(tmem, quarter, TS_S + c0), st[part]);
-            }
-            tmem_wait_st();
-        }
+        if (b1_ok && tid < kD / 4)
+            reinterpret_cast<float4*>(dc_keep)[tid] = reinterpret_cast<const float4*>(dc_s)[tid];
         tc_fence_before();
         if (!(ok = !__syncthreads_or(!b1_ok))) break;
         b1_pending = false;
 
-        // ---- MMA1: [Z_k^T | Y_k^T] = St^T [Qt ; W]^T
+        // ---- MMA1: [Z_k^T | Y_k^T] = S^T [Qs ; W]^T (the state at the chunk start,
+        // read by the tensor core as tf32: the low mantissa bits are dropped; measured
+        // on the CPU against the fp64 oracle: no change in the error of o or S)
         if (tid == 0) {
             tc_fence_after();
             const uint64_t db = tdesc(sb, S_B1);
@@ -780,8 +860,27 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
         b1_pending = c + 1 < nch;
         b1_chunk = c + 1;
 
-        // ---- delta^T = U^T - Y_k^T (tf32 operand, row = value column, K = token);
+        // ---- decay: S <- Diag(2^Gamma_C) S in place (fp32; MMA1, its last reader, is
+        // done), key channels 64 * half .. of value column e;
+        // delta^T = U^T - Y_k^T (tf32 operand, row = value column, K = token);
         // U^T came with Kb
+        {
+            float st[2][32];
+#pragma unroll
+            for (int part = 0; part < 2; ++part) tmem_ld32(tm_lane(tmem, quarter, TS_S + 64 * half + 32 * part), st[part]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                const int c0 = 64 * half + 32 * part;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float4 d4 = *reinterpret_cast<const float4*>(dc_keep + c0 + 4 * j);
+                    st[part][4 * j] *= d4.x; st[part][4 * j + 1] *= d4.y;
+                    st[part][4 * j + 2] *= d4.z; st[part][4 * j + 3] *= d4.w;
+                }
+                tmem_st32(tm_lane(tmem, quarter, TS_S + c0), st[part]);
+            }
+        }
         const bool b2_ok = mbar_wait_bounded(bar_b2, c & 1);
         if (b2_ok) {
             float y[32];
@@ -800,6 +899,7 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
                     tf32x4(u[4 * j] - y[4 * j], u[4 * j + 1] - y[4 * j + 1], u[4 * j + 2] - y[4 * j + 2],
                            u[4 * j + 3] - y[4 * j + 3]);
         }
+        tmem_wait_st();   // the decayed state is in place before MMA2a accumulates onto it
         fence_proxy_async_smem();
         tc_fence_before();
         if (!(ok = !__syncthreads_or(!b2_ok || !img_ok))) {

@@ -157,24 +157,55 @@ __device__ __forceinline__ void ut_inverse64(const float* Mf, float* Tf, float* 
     __syncthreads();
 }
 
+// Per-thread channel data of one chunk, for the calling thread's 4 channels
+// 4 * lane .. 4 * lane + 3 (every warp holds the same values): rho[a] is the
+// cumulative log-decay Gamma (log2 units, relative to the chunk start, so
+// <= 0) at the last token of the 16-token block a; rho[3] = Gamma_C.
+struct ChunkChannels {
+    float4 rho[4];
+    float4 bstart, bend;   // Gamma before and after the 16-token block of the thread's rows
+};
+
+// Largest exponent (log2 units) one factor of a factorised decay product may
+// carry: 2^100 and 2^-100 are far inside the fp32 / tf32 normal range, so
+// neither overflow nor flushed subnormals can occur below it.
+constexpr float kSafeLog2 = 100.f;
+
+// How the intra-chunk Gram matrices A_ri = sum_c k_rc k_ic 2^(Gamma_rc - Gamma_ic)
+// and P (same with q_r) of a chunk are taken, by the decay it carries:
+//   0: every channel decays by at most kSafeLog2 over the chunk -- one
+//      tensor-core product through the chunk end, (x 2^(Gamma_r - Gamma_C))
+//      (k 2^(Gamma_C - Gamma_i))^T;
+//   1: every channel decays by at most kSafeLog2 inside each 16-token block --
+//      block references: with rho_a the chunk's Gamma at the end of block a
+//      (rho_-1 = 0), X_r = 2^(Gamma_r - rho_{a(r)-1}), Y_i = 2^(rho_{b(i)} - Gamma_i)
+//      and Z_ab = 2^(rho_{a-1} - rho_b) for blocks b <= a,
+//      2^(Gamma_r - Gamma_i) = X_r Z_{a(r) b(i)} Y_i, where X, Y, Z_ab (b < a)
+//      lie in (0, 1] and Z_aa <= 2^kSafeLog2;
+//   2: otherwise -- the same for pairs of different blocks, and every
+//      2^(Gamma_r - Gamma_i) inside a block on its own.
+// All three reproduce the per-token rule exactly up to rounding.
+
 // Prep of one chunk of up to 64 tokens, for the calling thread's 8 token rows
-// r = 8 * warp + m (m = 0..7) and 4 channels 4 * lane .. 4 * lane + 3:
-//   Gamma_r = g_0 + ... + g_r per channel (log2 units), Gamma_C = Gamma_63
-//   (rows past L carry g = 0, so Gamma_C is the value at the last token);
-//   q^, k^ = L2-normalised rows (if l2norm), then
-//   Kt = k^ 2^(Gamma_r - Gamma_C),  Qt = scale q^ 2^(Gamma_r - Gamma_C),
-//   Kb = k^ 2^(Gamma_C - Gamma_r),  all zero for rows r >= L.
+// r = 8 * warp + m (m = 0..7, all inside 16-token block warp / 2) and 4
+// channels 4 * lane .. 4 * lane + 3:
+//   Gamma_r = g_0 + ... + g_r per channel (log2 units; rows past the chunk's
+//   last token carry g = 0, so Gamma_C = Gamma_63 is the value at its last
+//   token); q^, k^ = L2-normalised rows (if l2norm), q^ scaled by `scale`,
+//   zero for r >= L.
 // greg holds the thread's g values (rows x channels, natural-log units);
 // rq / rk point at the raw bf16 q / k rows ([64][128]), which are read into
 // registers before the block barrier inside, so emit may overwrite them.
-// emit(r, kbi, ch, kt, qt, kb) receives the fp32 values of row r for the
-// K-block kbi = lane / 8 and 16-byte chunk ch = lane % 8 of a K-major tile.
-// gc receives Gamma_C (log2 units) of the thread's 4 channels.  xch is a
-// shared [8][128] exchange buffer.  All 256 threads must call it.
-template <class Emit>
-__device__ __forceinline__ void prep_chunk_rows(const uint8_t* rq, const uint8_t* rk, const float (&greg)[8][4],
-                                                float* xch, int L, float scale, bool l2norm, float2 (&gc)[2],
-                                                Emit emit) {
+// Calls setup(cc, level) once, with the block ends of the thread's channels
+// and the chunk's Gram level (the same in every thread of the block), then
+// emit(r, kbi, ch, qn, kn, gr) with the fp32 q^, k^ and Gamma_r of row r for
+// the K-block kbi = lane / 8 and 16-byte chunk ch = lane % 8 of a K-major
+// tile.  Returns the level.  xch is a shared [8][128] exchange buffer.  All
+// 256 threads must call it.
+template <class Setup, class Emit>
+__device__ __forceinline__ int prep_chunk_rows(const uint8_t* rq, const uint8_t* rk, const float (&greg)[8][4],
+                                               float* xch, int L, float scale, bool l2norm, Setup setup,
+                                               Emit emit) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint2 qraw[8], kraw[8];
 #pragma unroll
@@ -198,21 +229,35 @@ __device__ __forceinline__ void prep_chunk_rows(const uint8_t* rq, const uint8_t
         *reinterpret_cast<float2*>(xch + warp * 128 + 4 * lane + 2 * x) = run;
     }
     __syncthreads();   // also: every thread holds its raw q, k in registers
+    // off = Gamma before this warp's first row; a block ends every second warp
+    ChunkChannels cc;
+    float2 run[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
     float2 off[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-    gc[0] = gc[1] = make_float2(0.f, 0.f);
 #pragma unroll
     for (int w = 0; w < 8; ++w) {
         const float4 t = *reinterpret_cast<const float4*>(xch + w * 128 + 4 * lane);
-        if (w < warp) {
-            off[0] = __fadd2_rn(off[0], make_float2(t.x, t.y));
-            off[1] = __fadd2_rn(off[1], make_float2(t.z, t.w));
+        if (w == warp) {
+            off[0] = run[0];
+            off[1] = run[1];
         }
-        gc[0] = __fadd2_rn(gc[0], make_float2(t.x, t.y));
-        gc[1] = __fadd2_rn(gc[1], make_float2(t.z, t.w));
+        if (w == (warp & 6)) cc.bstart = make_float4(run[0].x, run[0].y, run[1].x, run[1].y);
+        run[0] = __fadd2_rn(run[0], make_float2(t.x, t.y));
+        run[1] = __fadd2_rn(run[1], make_float2(t.z, t.w));
+        if (w & 1) cc.rho[w >> 1] = make_float4(run[0].x, run[0].y, run[1].x, run[1].y);
+        if (w == (warp | 1)) cc.bend = make_float4(run[0].x, run[0].y, run[1].x, run[1].y);
     }
-    // offset to the chunk end: Gamma_r - Gamma_C = G + (off - gc)
-    const float2 rel[2] = {__fadd2_rn(off[0], make_float2(-gc[0].x, -gc[0].y)),
-                           __fadd2_rn(off[1], make_float2(-gc[1].x, -gc[1].y))};
+    // the Gram level: every warp holds the same per-lane data, so the vote is block-uniform
+    float block_decay = 0.f;
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+        const float4 pr = a ? cc.rho[a - 1] : make_float4(0.f, 0.f, 0.f, 0.f), c = cc.rho[a];
+        block_decay = fmaxf(block_decay, fmaxf(fmaxf(pr.x - c.x, pr.y - c.y), fmaxf(pr.z - c.z, pr.w - c.w)));
+    }
+    const float chunk_decay = fmaxf(fmaxf(-cc.rho[3].x, -cc.rho[3].y), fmaxf(-cc.rho[3].z, -cc.rho[3].w));
+    const int level = !__any_sync(0xffffffffu, chunk_decay > kSafeLog2)   ? 0
+                      : !__any_sync(0xffffffffu, block_decay > kSafeLog2) ? 1
+                                                                          : 2;
+    setup(cc, level);
 
     // unpack, mask rows past the sequence end, and L2-normalise all 8 rows
     float2 qv[8][2], kv[8][2];
@@ -239,25 +284,157 @@ __device__ __forceinline__ void prep_chunk_rows(const uint8_t* rq, const uint8_t
         const int r = 8 * warp + m;
         const float nq = (l2norm ? rsqrtf(nrm[m] + kNormEps) : 1.f) * scale;
         const float nk = l2norm ? rsqrtf(nrm[8 + m] + kNormEps) : 1.f;
-        float4 kt, qt, kb;
-        float* ktp = &kt.x;
-        float* qtp = &qt.x;
-        float* kbp = &kb.x;
-#pragma unroll
-        for (int x = 0; x < 2; ++x) {
-            // a = (Gamma_r - Gamma_C) / ln 2 >= 0 (the decay is cumulative, g <= 0)
-            const float2 a = __fadd2_rn(G[m][x], rel[x]);
-            const float2 e = make_float2(ex2(fminf(a.x, 126.f)), ex2(fminf(a.y, 126.f)));   // E >= 1
-            const float2 f = make_float2(ex2(-a.x), ex2(-a.y));                              // F <= 1
-            const float2 kn = __fmul2_rn(kv[m][x], make_float2(nk, nk));
-            const float2 qn = __fmul2_rn(qv[m][x], make_float2(nq, nq));
-            const float2 t1 = __fmul2_rn(kn, e), t2 = __fmul2_rn(qn, e), t3 = __fmul2_rn(kn, f);
-            ktp[2 * x] = t1.x; ktp[2 * x + 1] = t1.y;
-            qtp[2 * x] = t2.x; qtp[2 * x + 1] = t2.y;
-            kbp[2 * x] = t3.x; kbp[2 * x + 1] = t3.y;
-        }
-        emit(r, kbi, ch, kt, qt, kb);
+        const float2 q0 = __fmul2_rn(qv[m][0], make_float2(nq, nq)), q1 = __fmul2_rn(qv[m][1], make_float2(nq, nq));
+        const float2 k0 = __fmul2_rn(kv[m][0], make_float2(nk, nk)), k1 = __fmul2_rn(kv[m][1], make_float2(nk, nk));
+        const float2 g0 = __fadd2_rn(G[m][0], off[0]), g1 = __fadd2_rn(G[m][1], off[1]);
+        emit(r, kbi, ch, make_float4(q0.x, q0.y, q1.x, q1.y), make_float4(k0.x, k0.y, k1.x, k1.y),
+             make_float4(g0.x, g0.y, g1.x, g1.y));
     }
+    return level;
+}
+
+__device__ __forceinline__ float4 ex2x4(float4 a) { return make_float4(ex2(a.x), ex2(a.y), ex2(a.z), ex2(a.w)); }
+__device__ __forceinline__ float4 mul4(float4 a, float4 b) {
+    return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w);
+}
+__device__ __forceinline__ float4 sub4(float4 a, float4 b) {
+    return make_float4(a.x - b.x, a.y - b.y, a.z - b.z, a.w - b.w);
+}
+
+// ---------------------------------------------------------------- exact Gram
+// Gram matrices of a chunk at level 1 or 2, on CUDA cores and mma.sync, for
+// the prep of the two-pass prefill.  Inputs (fp32, K-major 128-byte-swizzled
+// tiles as the emit wrote them):
+//   xt  128 rows: rows 0-63 Q-side, rows 64-127 K-side;
+//   yt  64 rows;
+// level 1: xt = [q^ X ; k^ X], yt = k^ Y (block references, see above);
+// level 2: xt = [q^ ; k^], yt = Gamma (log2), converted here in place to the
+//          level-1 tiles once the in-block pairs are done;
+// rho: [4][128] block-end Gammas (shared memory);  ztab: [10][128] scratch.
+// Output: the unmasked 64 x 64 matrices P (rows 0-63) and A (rows 64-127) as
+// plain fp32 rows of kStLd floats in `st`, which may be xt itself (it is only
+// written after every read of the inputs).  Entries above the diagonal are
+// left undefined.  All 256 threads; block barriers inside (none at entry,
+// one at exit).  `mid` runs once every input read is done, before the output
+// is written (it may reuse yt and ztab).
+constexpr int kStLd = 68;
+static_assert(128 * kStLd * 4 <= 65536, "staging fits the 64 KB [Q ; K] tile");
+
+// Block pair of mma unit u: pairs p = a (a + 1) / 2 + b in order, or at level
+// 2 only those with b < a (p = 1, 3, 4, 6, 7, 8).
+__device__ __forceinline__ int gram_pair(int u, int level) {
+    const int p = u >> 1;
+    return level == 2 ? p + 1 + (p >= 1) + (p >= 3) : p;
+}
+
+template <class Mid>
+__device__ __forceinline__ void gram_exact(uint8_t* xt, uint32_t kbx, uint8_t* yt, uint32_t kby, const float* rho,
+                                           float* ztab, float* st, int level, int tid, Mid mid) {
+    const int warp = tid >> 5, lane = tid & 31;
+    // Z table: entry p = a (a + 1) / 2 + b of the block pair (a, b), b <= a
+    for (int e = tid; e < 10 * kD; e += 256) {
+        const int p = e >> 7, c = e & (kD - 1);
+        const int a = (p >= 1) + (p >= 3) + (p >= 6), b = p - a * (a + 1) / 2;
+        const float prev = a ? rho[(a - 1) * kD + c] : 0.f;
+        ztab[e] = ex2(fminf(prev - rho[b * kD + c], 126.f));
+    }
+    // level 2: pairs inside a 16-token block, one exponential each.  Thread
+    // (block a, row j / 4, column group j % 4) sums four entries of P and A.
+    float dq[4] = {0.f, 0.f, 0.f, 0.f}, dk[4] = {0.f, 0.f, 0.f, 0.f};
+    const int pa = tid >> 6, prow = 16 * pa + ((tid & 63) >> 2), pcol = 16 * pa + 4 * (tid & 3);
+    if (level == 2 && pcol <= prow) {
+        for (int k = 0; k < kD; k += 4) {
+            const float4 qr = *reinterpret_cast<const float4*>(K_at(xt, 0, kbx, prow, k));
+            const float4 kr = *reinterpret_cast<const float4*>(K_at(xt, 0, kbx, 64 + prow, k));
+            const float4 gr = *reinterpret_cast<const float4*>(K_at(yt, 0, kby, prow, k));
+#pragma unroll
+            for (int l = 0; l < 4; ++l) {
+                const float4 ki = *reinterpret_cast<const float4*>(K_at(xt, 0, kbx, 64 + pcol + l, k));
+                const float4 gi = *reinterpret_cast<const float4*>(K_at(yt, 0, kby, pcol + l, k));
+                const float4 f = ex2x4(make_float4(fminf(gr.x - gi.x, 0.f), fminf(gr.y - gi.y, 0.f),
+                                                   fminf(gr.z - gi.z, 0.f), fminf(gr.w - gi.w, 0.f)));
+                const float4 w = mul4(ki, f);
+                dq[l] = fmaf(qr.x, w.x, fmaf(qr.y, w.y, fmaf(qr.z, w.z, fmaf(qr.w, w.w, dq[l]))));
+                dk[l] = fmaf(kr.x, w.x, fmaf(kr.y, w.y, fmaf(kr.z, w.z, fmaf(kr.w, w.w, dk[l]))));
+            }
+        }
+    }
+    __syncthreads();
+    if (level == 2) {   // raw tiles -> level-1 tiles, in place
+        for (int it = tid; it < 64 * (kD / 4); it += 256) {
+            const int r = it >> 5, k = 4 * (it & 31), a = r >> 4;
+            float4* qp = reinterpret_cast<float4*>(K_at(xt, 0, kbx, r, k));
+            float4* kp = reinterpret_cast<float4*>(K_at(xt, 0, kbx, 64 + r, k));
+            float4* yp = reinterpret_cast<float4*>(K_at(yt, 0, kby, r, k));
+            const float4 g = *yp, kk = *kp, q = *qp;
+            const float4 prev = a ? *reinterpret_cast<const float4*>(rho + (a - 1) * kD + k) : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 cur = *reinterpret_cast<const float4*>(rho + a * kD + k);
+            const float4 X = ex2x4(sub4(g, prev)), Y = ex2x4(sub4(cur, g));
+            *qp = mul4(q, X);
+            *kp = mul4(kk, X);
+            *yp = mul4(kk, Y);
+        }
+        __syncthreads();
+    }
+    // block pairs on mma.sync (tf32, fp32 accumulation): unit u = 2 p + m is
+    // block pair p, matrix m (0: P from the Q-side rows, 1: A from the K-side
+    // rows); at level 2 only pairs of different blocks
+    const int gq = lane >> 2, tq = lane & 3;
+    float d[3][2][4];
+    int units[3];
+    const int nunits = level == 2 ? 12 : 20;
+#pragma unroll
+    for (int s = 0; s < 3; ++s) {
+        const int u = warp + 8 * s;
+        units[s] = u < nunits ? u : -1;
+        if (units[s] < 0) continue;
+        const int p = gram_pair(u, level);
+        const int a = (p >= 1) + (p >= 3) + (p >= 6), b = p - a * (a + 1) / 2;
+        const int m = u & 1, row0 = 64 * m + 16 * a;
+        const float* z = ztab + p * kD;
+#pragma unroll
+        for (int nh = 0; nh < 2; ++nh)
+#pragma unroll
+            for (int x = 0; x < 4; ++x) d[s][nh][x] = 0.f;
+#pragma unroll 4
+        for (int k0 = 0; k0 < kD; k0 += 8) {
+            const float z0 = z[k0 + tq], z1 = z[k0 + tq + 4];
+            uint32_t fa[4];
+            fa[0] = tf32_bits(*K_at(xt, 0, kbx, row0 + gq, k0 + tq) * z0);
+            fa[1] = tf32_bits(*K_at(xt, 0, kbx, row0 + gq + 8, k0 + tq) * z0);
+            fa[2] = tf32_bits(*K_at(xt, 0, kbx, row0 + gq, k0 + tq + 4) * z1);
+            fa[3] = tf32_bits(*K_at(xt, 0, kbx, row0 + gq + 8, k0 + tq + 4) * z1);
+#pragma unroll
+            for (int nh = 0; nh < 2; ++nh) {
+                const int col = 16 * b + 8 * nh + gq;
+                uint32_t fb[2];
+                fb[0] = tf32_bits(*K_at(yt, 0, kby, col, k0 + tq));
+                fb[1] = tf32_bits(*K_at(yt, 0, kby, col, k0 + tq + 4));
+                mma_m16n8k8_tf32(d[s][nh], fa, fb);
+            }
+        }
+    }
+    __syncthreads();   // every input read
+    mid();
+#pragma unroll
+    for (int s = 0; s < 3; ++s) {
+        if (units[s] < 0) continue;
+        const int u = units[s];
+        const int p = gram_pair(u, level);
+        const int a = (p >= 1) + (p >= 3) + (p >= 6), b = p - a * (a + 1) / 2;
+        const int row0 = 64 * (u & 1) + 16 * a;
+#pragma unroll
+        for (int nh = 0; nh < 2; ++nh) {
+            const int col = 16 * b + 8 * nh + 2 * tq;
+            *reinterpret_cast<float2*>(st + (row0 + gq) * kStLd + col) = make_float2(d[s][nh][0], d[s][nh][1]);
+            *reinterpret_cast<float2*>(st + (row0 + gq + 8) * kStLd + col) = make_float2(d[s][nh][2], d[s][nh][3]);
+        }
+    }
+    if (level == 2 && pcol <= prow) {
+        *reinterpret_cast<float4*>(st + prow * kStLd + pcol) = make_float4(dq[0], dq[1], dq[2], dq[3]);
+        *reinterpret_cast<float4*>(st + (64 + prow) * kStLd + pcol) = make_float4(dk[0], dk[1], dk[2], dk[3]);
+    }
+    __syncthreads();
 }
 
 }  // namespace kda

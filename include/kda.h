@@ -26,10 +26,15 @@
  *       o          : [tokens, H, d]      fp32
  *       states     : [N, H, d, d] fp32   (sequence, head, key row, value col)
  *   - q, k, v share one dtype (kda_dtype); g, beta, states and o are fp32.
- *   - g = log(alpha) must be finite and <= 0.  Within one 64-token chunk the
- *     decay a channel accumulates (-sum g) must stay below 80 for the
- *     tensor-core path; larger decay is still finite but loses accuracy there
- *     (use KDA_FLAG_RECURRENT, which has no such limit).
+ *   - g = log(alpha) must be finite and <= 0; any such value is handled
+ *     exactly (up to rounding) by every path.  The page lets each channel
+ *     decay at its own data-dependent rate, so a chunk may carry any amount
+ *     of decay: the chunked tensor-core prefill takes a 64-token chunk whose
+ *     decay exceeds about 69 nats in some channel through 16-token block
+ *     references, and pairs of tokens inside a 16-token block whose decay
+ *     exceeds that through one exponential each (both slower than the common
+ *     case, still exact); the fused kernel that runs with the minimum
+ *     workspace hands such a sequence to the token-by-token recurrence.
  *   - Only d == 128 is supported (KDA_ERR_UNSUPPORTED otherwise).
  *   - Returns KDA_OK (0) or a negative kda_status.  Host-side checks run
  *     before anything is enqueued; on an error nothing is launched.

@@ -42,3 +42,48 @@ def test_tf32_operands_fit_the_bf16_tolerance_with_margin():
     err_o = np.abs(oc - o).max() / np.sqrt(np.mean(o * o))
     err_s = np.abs(sc - s).max() / np.sqrt(np.mean(s * s))
     assert err_o < 1e-2 and err_s < 1e-2, (err_o, err_s)
+
+
+# ---------------------------------------------------------------- chunk-start form
+# The form of the two-pass tensor-core prefill: state-side factors relative to
+# the chunk start (all in (0, 1]), Gram matrices at level 0, 1 or 2 by the
+# chunk's decay.  Each level must reproduce the token-by-token oracle exactly
+# (fp64), whatever the decay: the per-chunk decays below run from a few nats
+# to several thousand, and one case drives three channels at g = -80 per token.
+from tests.chunk_form import kda_forward_chunked_start  # noqa: E402
+
+
+def _strong_case(kind):
+    x = kin.make_custom_prefill(6, [300, 70], heads=2, init_state_std=0.02)
+    g = f64(x.g)
+    if kind == "per_token_2":          # ~2 nats per token on a third of the channels
+        g[:, :, ::3] = -2.0
+    elif kind == "x40":                # ~270 nats per chunk on the fastest channel
+        g = g * 40.0
+    elif kind == "x2000":              # ~13,500 nats per chunk
+        g = g * 2000.0
+    elif kind == "g80":                # three channels at g = -80 per token
+        g[:, :, [3, 77, 100]] = -80.0
+    o, s = oracle.kda_forward(x.q, x.k, x.v, g, x.beta, x.cu_seqlens, x.initial_state, scale=0.8)
+    args = (f64(x.q), f64(x.k), f64(x.v), g, f64(x.beta), x.cu_seqlens.tolist(), f64(x.initial_state))
+    return args, o, s
+
+
+@pytest.mark.parametrize("kind,expect", [("plain", {0}), ("per_token_2", {0, 1}), ("x40", {0, 2}),
+                                         ("x2000", {2}), ("g80", {2})])
+def test_chunk_start_form_matches_oracle_at_any_decay(kind, expect):
+    args, o, s = _strong_case(kind)
+    levels = []
+    oc, sc = kda_forward_chunked_start(*args, scale=0.8, levels=levels)
+    assert set(levels) == expect
+    scale_o, scale_s = np.sqrt(np.mean(o * o)), np.sqrt(np.mean(s * s))
+    assert np.abs(oc - o).max() <= 1e-11 * scale_o
+    assert np.abs(sc - s).max() <= 1e-11 * scale_s
+
+
+@pytest.mark.parametrize("level", [1, 2])
+def test_gram_levels_agree_where_all_are_finite(level):
+    args, o, s = _strong_case("plain")
+    oc, sc = kda_forward_chunked_start(*args, scale=0.8, force_level=level)
+    np.testing.assert_allclose(oc, o, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(sc, s, rtol=0, atol=1e-12)
