@@ -554,23 +554,21 @@ bool make_token_map(CUtensorMap* map, const void* base, int64_t total_T, int H, 
 cudaError_t launch_chunk(const PrefillArgs& a, cudaStream_t stream) {
     if (a.N == 0 || a.H == 0) return cudaSuccess;
     if (a.total_T <= 0) return cudaErrorInvalidValue;   // callers route empty batches elsewhere
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(kda_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        static_cast<int>(SMEM_BYTES));
+    static PerDeviceOnce attr_once;
+    const cudaError_t attr_err = attr_once.run([] {
+        return cudaFuncSetAttribute(kda_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(SMEM_BYTES));
     });
     if (attr_err != cudaSuccess) return attr_err;
     CUtensorMap mq, mk;
     if (!make_token_map(&mq, a.q, a.total_T, a.H) || !make_token_map(&mk, a.k, a.total_T, a.H))
         return cudaErrorInvalidValue;
     const long long blocks = (long long)a.N * a.H * kSplit;
-    kda_chunk_kernel<<<static_cast<unsigned>(blocks), kThreads, SMEM_BYTES, stream>>>(
+    return launch_kernel(kda_chunk_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), SMEM_BYTES, stream,
         mq, mk, static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
         static_cast<const __nv_bfloat16*>(a.v), a.g, a.beta, a.cu_seqlens, a.total_T, a.H, a.scale,
         a.l2norm ? 1 : 0, a.scalar_decay ? 1 : 0, a.initial_state, a.final_state, a.o, a.err, a.slots,
         a.num_slots);
-    return cudaGetLastError();
 }
 
 }  // namespace kda

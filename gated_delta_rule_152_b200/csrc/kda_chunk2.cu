@@ -253,7 +253,7 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
     };
     // the item's image: its own place in the scratch, or its head's ring slot
     auto image_of = [&](const Item& it) {
-        const size_t slot = RING ? static_cast<size_t>(it.h) * kRing + (it.c & (kRing - 1))
+        const size_t slot = RING ? static_cast<size_t>(it.h) * kRing + (it.gc & (kRing - 1))
                                  : static_cast<size_t>(it.gc) * H + it.h;
         return img + slot * IMG_BYTES;
     };
@@ -335,10 +335,11 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
         // producer never blocks on it while holding an unannounced image (the
         // state role that it waits for may need exactly that image).
         bool slot_free = true;
-        if (RING && tid == kStoreThread && cur.c >= kRing && done_seen < cur.c - kRing + 1 &&
-            ld_acquire_gpu(done_flag(ring, cur.h)) < cur.c - kRing + 1) {
+        const int32_t gcur = static_cast<int32_t>(cur.gc);   // the head's ring counts global chunks
+        if (RING && tid == kStoreThread && gcur >= kRing && done_seen < gcur - kRing + 1 &&
+            ld_acquire_gpu(done_flag(ring, cur.h)) < gcur - kRing + 1) {
             publish();
-            slot_free = wait_flag_ge(done_flag(ring, cur.h), cur.c - kRing + 1, 1u << 20, 256);
+            slot_free = wait_flag_ge(done_flag(ring, cur.h), gcur - kRing + 1, 1u << 20, 256);
         }
         // the previous item's P has left X, which is rewritten below
         if (tid == kStoreThread) bulk_wait_read_but<1>();
@@ -351,8 +352,9 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
         // -> KTM (MN-major, for W), Kb = k^ 2^(Gamma_C - Gamma_r) -> image (MN-major), and
         // 2^Gamma_C -> image.  The Gram operands in X (128 rows, Q-side then K-side) and KB
         // (64 rows), both K-major, depend on the chunk's level (kda_tile.cuh):
-        //   0: [Qs ; Ks] 2^-Gamma_C and Kb, tf32 (the tensor-core product through the chunk end);
-        //   1: [q^ X ; k^ X] and k^ Y, fp32 (block references);
+        //   0: [Qs ; Ks] and Kb 2^-Gamma_C = k^ 2^-Gamma_i, tf32 (one tensor-core product; the
+        //      second factor is at most 2^kSafeLog2 at this level);
+        //   1: [q^ X ; k^ X] (fp32) and k^ Y (tf32) (block references);
         //   2: [q^ ; k^] and Gamma, fp32.
         // A warp stores four whole 128-byte rows of the image at a time.
         int level = 0;
@@ -370,40 +372,42 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
                 rho1 = cc.rho[1];
                 rho2 = cc.rho[2];
                 rho3 = cc.rho[3];
-                inv = ex2x4(make_float4(fminf(-gc.x, 126.f), fminf(-gc.y, 126.f), fminf(-gc.z, 126.f),
-                                        fminf(-gc.w, 126.f)));
-                es = ex2x4(bprev);
-                ef = ex2x4(sub4(gc, bcur));
+                if (lvl == 0) {
+                    inv = ex2x4(make_float4(-gc.x, -gc.y, -gc.z, -gc.w));
+                } else if (lvl == 1) {
+                    es = ex2x4(bprev);
+                    ef = ex2x4(sub4(gc, bcur));
+                }
             };
             prep_chunk_rows(smem + P_KB, smem + P_KB + kC * kD * 2, greg, xch, L, scale, l2norm != 0, setup,
                             [&](int r, int kbi, int ch, float4 qn, float4 kn, float4 gr) {
-                float4 qs, ks, kb, xq, xk, y;
+                float4 q4, k4, b4, xq, xk, y;
                 if (level == 1) {
                     const float4 X = ex2x4(sub4(gr, bprev)), Y = ex2x4(sub4(bcur, gr));
                     xq = mul4(qn, X);
                     xk = mul4(kn, X);
-                    y = mul4(kn, Y);
-                    qs = mul4(xq, es);
-                    ks = mul4(xk, es);
-                    kb = mul4(y, ef);
+                    const float4 ky = mul4(kn, Y);
+                    y = tf32x4(ky.x, ky.y, ky.z, ky.w);
+                    const float4 qs = mul4(xq, es), ks = mul4(xk, es), kb = mul4(ky, ef);
+                    q4 = tf32x4(qs.x, qs.y, qs.z, qs.w);
+                    k4 = tf32x4(ks.x, ks.y, ks.z, ks.w);
+                    b4 = tf32x4(kb.x, kb.y, kb.z, kb.w);
                 } else {
                     const float4 e0 = ex2x4(gr), f = ex2x4(sub4(gc, gr));
-                    qs = mul4(qn, e0);
-                    ks = mul4(kn, e0);
-                    kb = mul4(kn, f);
+                    const float4 qs = mul4(qn, e0), ks = mul4(kn, e0), kb = mul4(kn, f);
+                    q4 = tf32x4(qs.x, qs.y, qs.z, qs.w);
+                    k4 = tf32x4(ks.x, ks.y, ks.z, ks.w);
+                    b4 = tf32x4(kb.x, kb.y, kb.z, kb.w);
                     if (level == 0) {
-                        xq = tf32x4(qs.x * inv.x, qs.y * inv.y, qs.z * inv.z, qs.w * inv.w);
-                        xk = tf32x4(ks.x * inv.x, ks.y * inv.y, ks.z * inv.z, ks.w * inv.w);
-                        y = tf32x4(kb.x, kb.y, kb.z, kb.w);
+                        xq = q4;
+                        xk = k4;
+                        y = tf32x4(kb.x * inv.x, kb.y * inv.y, kb.z * inv.z, kb.w * inv.w);
                     } else {
                         xq = qn;
                         xk = kn;
                         y = gr;
                     }
                 }
-                const float4 q4 = tf32x4(qs.x, qs.y, qs.z, qs.w);
-                const float4 k4 = tf32x4(ks.x, ks.y, ks.z, ks.w);
-                const float4 b4 = tf32x4(kb.x, kb.y, kb.z, kb.w);
                 *reinterpret_cast<float4*>(smem + P_X + kbi * KB_B1 + sw128_off(r, ch)) = xq;
                 *reinterpret_cast<float4*>(smem + P_X + kbi * KB_B1 + sw128_off(64 + r, ch)) = xk;
                 *reinterpret_cast<float4*>(smem + P_KB + kbi * P_KB_KB + sw128_off(r, ch)) = y;
@@ -420,7 +424,7 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
         tc_fence_before();
         __syncthreads();
 
-        // ============== [P ; A]: level 0 by one tensor-core product [Qs ; Ks] 2^-Gamma_C x Kb^T
+        // ============== [P ; A]: level 0 by one tensor-core product [Qs ; Ks] x (Kb 2^-Gamma_C)^T
         // (P in lanes 0-63, A in lanes 64-127 of TP_AP), levels 1 and 2 on CUDA cores and
         // mma.sync (gram_exact), staged into the same tensor-memory columns
         if (level == 0 && tid == 0) {
@@ -612,8 +616,8 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
             bulk_store(im + IMG_U, smem + P_V, 4 * IMG_BLK);
             bulk_commit();
             if (RING) {
-                pub_flag = ready_flag(ring, cur.h, cur.c);
-                pub_val = cur.c + 1;
+                pub_flag = ready_flag(ring, cur.h, static_cast<int>(cur.gc));
+                pub_val = static_cast<int32_t>(cur.gc) + 1;
             }
         }
         cur = nxt;
@@ -677,7 +681,7 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
                                            const int32_t* __restrict__ chunk_off, const int32_t* __restrict__ cu,
                                            int64_t total_T, int H, int64_t max_total, const float* s0, float* sT,
                                            float* __restrict__ o, uint32_t* err, const int32_t* __restrict__ slots,
-                                           int num_slots, int n, int h, Ring ring) {
+                                           int num_slots, int n_begin, int n_end, int h, Ring ring) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sb = smem_u32(smem);
@@ -692,30 +696,6 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quarter = warp & 3, half = warp >> 2;
     const int e = 32 * quarter + lane;   // value column of this thread's TMEM lane
-
-    int64_t bos, eos;
-    if (!seq_bounds(cu, n, total_T, bos, eos)) return;   // flagged by the index kernel
-    const int64_t sidx = slots ? static_cast<int64_t>(slots[n]) : static_cast<int64_t>(n);
-    if (slots && (sidx < 0 || sidx >= num_slots)) {
-        if (tid == 0 && h == 0) set_error(err, 4u);
-        return;
-    }
-    const int nch = static_cast<int>((eos - bos + kC - 1) / kC);
-    const int64_t gc0 = chunk_off[n];
-    if (gc0 + nch > max_total) return;   // overlapping sequences overflowed the scratch: flagged above
-    auto image = [&](int c) {
-        const size_t slot = RING ? static_cast<size_t>(h) * kRing + (c & (kRing - 1))
-                                 : static_cast<size_t>(gc0 + c) * H + h;
-        return img + slot * IMG_BYTES;
-    };
-    // ring mode: chunk c's image must be complete before its first copy is issued
-    auto await_image = [&](int c) -> bool {
-        if (!RING) return true;
-        const bool good = wait_flag_ge(ready_flag(ring, h, c), c + 1);
-        fence_proxy_async_global();
-        return good;
-    };
-    bool img_ok = true;   // thread 0: the image wait did not give up (checked at the next barrier)
 
     if (warp == 0) {
         tmem_alloc(tmem_slot, TS_COLS);
@@ -732,6 +712,64 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // state carried across the sequences of this CTA: mbarrier phases follow the
+    // running chunk count `base` (one B1, one B2 and one MMA2b phase per chunk,
+    // two phases of bar_mma), and the in-flight copies and products with the
+    // running chunk index they belong to
+    uint32_t base = 0, mma_phase = 0;
+    bool ok = true, img_ok = true;   // img_ok: thread 0's image waits did not give up
+    bool b1_pending = false, b2_pending = false, mma_pending = false, o_pending = false;
+    int b1_chunk = 0, b2_chunk = 0;
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
+        return !__syncthreads_or(!mbar_wait_bounded(bar, parity));
+    };
+    auto zcol = [](int c) { return TS_Z + 256u * static_cast<uint32_t>(c & 1); };   // Z of chunk c; Y follows
+
+    for (int n = n_begin; ok && n < n_end; ++n) {
+    __syncthreads();   // the previous sequence's final state has left tensor memory
+    int64_t bos, eos;
+    if (!seq_bounds(cu, n, total_T, bos, eos)) continue;   // flagged by the index kernel
+    const int64_t sidx = slots ? static_cast<int64_t>(slots[n]) : static_cast<int64_t>(n);
+    const int nch = static_cast<int>((eos - bos + kC - 1) / kC);
+    const int64_t gc0 = chunk_off[n];
+    // a sequence skipped below still has its chunks' images made by the prep role (as far
+    // as the scratch reaches); in ring mode they are handed back unread, so that the
+    // producers waiting for those slots go on
+    auto drain = [&]() -> bool {
+        bool good = true;
+        if (RING && tid == kOutThread) {
+            const int64_t last = gc0 + nch < max_total ? gc0 + nch : max_total;
+            for (int64_t gcx = gc0; good && gcx < last; ++gcx) {
+                good = wait_flag_ge(ready_flag(ring, h, static_cast<int>(gcx)), static_cast<int>(gcx + 1));
+                if (good) st_relaxed_gpu(done_flag(ring, h), static_cast<int>(gcx + 1));
+            }
+        }
+        return !__syncthreads_or(!good);
+    };
+    if (slots && (sidx < 0 || sidx >= num_slots)) {
+        if (tid == 0 && h == 0) set_error(err, 4u);
+        if (!(ok = drain())) break;
+        continue;
+    }
+    if (gc0 + nch > max_total) {   // overlapping sequences overflowed the scratch: flagged above
+        if (!(ok = drain())) break;
+        continue;
+    }
+    auto image = [&](int c) {
+        const size_t slot = RING ? static_cast<size_t>(h) * kRing + ((gc0 + c) & (kRing - 1))
+                                 : static_cast<size_t>(gc0 + c) * H + h;
+        return img + slot * IMG_BYTES;
+    };
+    // ring mode: chunk c's image must be complete before its first copy is issued
+    auto await_image = [&](int c) -> bool {
+        if (!RING) return true;
+        const bool good = wait_flag_ge(ready_flag(ring, h, static_cast<int>(gc0 + c)), static_cast<int>(gc0 + c + 1));
+        fence_proxy_async_global();
+        return good;
+    };
+    img_ok = true;
+
+
     const size_t state_off = ((size_t)sidx * H + h) * kD * kD;
 
     // initial state, transposed: lane e = value column, columns = key rows 64*half ..
@@ -774,15 +812,10 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
             load_b2(0);
         }
     }
-    // in-flight copies and products: pending flag and the chunk (parity) they belong to
-    bool ok = !__syncthreads_or(!img_ok);
-    bool b1_pending = ok && nch > 0, b2_pending = ok && nch > 0, mma_pending = false, o_pending = false;
-    int b1_chunk = 0, b2_chunk = 0;
-    uint32_t mma_phase = 0;
-    auto wait_all = [&](uint64_t* bar, uint32_t parity) -> bool {
-        return !__syncthreads_or(!mbar_wait_bounded(bar, parity));
-    };
-    auto zcol = [](int c) { return TS_Z + 256u * static_cast<uint32_t>(c & 1); };   // Z of chunk c; Y follows
+    ok = !__syncthreads_or(!img_ok);
+    if (!ok) break;
+    b1_pending = b2_pending = nch > 0;
+    b1_chunk = b2_chunk = static_cast<int>(base);
     if (!RING && tid == kOutThread && nch > 1) prefetch_l2(image(1), IMG_BYTES);
 
     int64_t t_prev = bos;
@@ -798,13 +831,13 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
             tc_fence_after();
             if (tid == 0) load_b2_kb_u(c);
             b2_pending = true;
-            b2_chunk = c;
+            b2_chunk = static_cast<int>(base) + c;
         }
         if (!RING && tid == kOutThread && c + 2 < nch) prefetch_l2(image(c + 2), IMG_BYTES);
         if (tid == kOutThread) bulk_wait_read();   // the O staging tile is rewritten below
         // [Qs ; W] and 2^Gamma_C of chunk c have landed; 2^Gamma_C is kept aside for
         // the decay after MMA1 (the next chunk's copy lands on top of it before then)
-        const bool b1_ok = mbar_wait_bounded(bar_b1, c & 1);
+        const bool b1_ok = mbar_wait_bounded(bar_b1, (base + c) & 1);
         if (b1_ok && tid < kD / 4)
             reinterpret_cast<float4*>(dc_keep)[tid] = reinterpret_cast<const float4*>(dc_s)[tid];
         tc_fence_before();
@@ -830,7 +863,7 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
         // tile; its product MMA2b also read P, so chunk c's copy of P waits for it
         bool o_ok = true;
         if (c > 0 && half == 1) {
-            o_ok = mbar_wait_bounded(bar_o, (c - 1) & 1);
+            o_ok = mbar_wait_bounded(bar_o, (base + c - 1) & 1);
             if (o_ok) {
                 tc_fence_after();
                 if (tid == kOutThread) load_b2_p(c);
@@ -858,7 +891,7 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
         }
         if (tid == kImgThread && c + 1 < nch && img_ok) load_b1(c + 1);
         b1_pending = c + 1 < nch;
-        b1_chunk = c + 1;
+        b1_chunk = static_cast<int>(base) + c + 1;
 
         // ---- decay: S <- Diag(2^Gamma_C) S in place (fp32; MMA1, its last reader, is
         // done), key channels 64 * half .. of value column e;
@@ -881,7 +914,7 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
                 tmem_st32(tm_lane(tmem, quarter, TS_S + c0), st[part]);
             }
         }
-        const bool b2_ok = mbar_wait_bounded(bar_b2, c & 1);
+        const bool b2_ok = mbar_wait_bounded(bar_b2, (base + c) & 1);
         if (b2_ok) {
             float y[32];
             tmem_ld32(tm_lane(tmem, quarter, zcol(c) + 64 + 32 * half), y);
@@ -909,7 +942,7 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
         b2_pending = false;
         // chunk c's slot is read: both copies have landed (their mbarriers
         // completed), so the slot can be handed back with a plain store
-        if (RING && tid == kOutThread) st_relaxed_gpu(done_flag(ring, h), c + 1);
+        if (RING && tid == kOutThread) st_relaxed_gpu(done_flag(ring, h), static_cast<int>(gc0 + c + 1));
 
         // ---- MMA2a: S^T += delta^T Kb (thread 0);  MMA2b: Z_k^T += delta^T P^T,
         // O of chunk c (kOutThread, so that neither issuing thread is held up
@@ -934,8 +967,9 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
         t_prev = t0;
         if (c + 1 == nch) {   // last chunk: O straight to o once MMA2b is done
             if (!(ok = wait_all(bar_mma, mma_phase))) break;
+            mma_phase ^= 1;   // the next sequence's products continue the phase count
             mma_pending = false;
-            if (!(ok = wait_all(bar_o, c & 1))) break;
+            if (!(ok = wait_all(bar_o, (base + c) & 1))) break;
             o_pending = false;
             tc_fence_after();
             float acc[32];
@@ -948,19 +982,21 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
             }
         }
     }
-    if (ok) {
-        if (sT) {
-            float acc[32];
+    if (!ok) break;
+    if (sT) {
+        float acc[32];
 #pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                const int c0 = 64 * half + 32 * part;
-                tmem_ld32(tm_lane(tmem, quarter, TS_S + c0), acc);
-                tmem_wait_ld();
+        for (int part = 0; part < 2; ++part) {
+            const int c0 = 64 * half + 32 * part;
+            tmem_ld32(tm_lane(tmem, quarter, TS_S + c0), acc);
+            tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) sT[state_off + (size_t)(c0 + j) * kD + e] = acc[j];
-            }
+            for (int j = 0; j < 32; ++j) sT[state_off + (size_t)(c0 + j) * kD + e] = acc[j];
         }
-    } else if (tid == 0) {
+    }
+    base += static_cast<uint32_t>(nch);
+    }   // sequences
+    if (!ok && tid == 0) {
         // a bounded wait gave up: report, give outstanding copies and MMAs a
         // last bounded chance to land, then release tensor memory
         set_error(err, 2u);
@@ -995,27 +1031,30 @@ kda_chunk_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t* 
                        int64_t max_total, const float* s0, float* sT, float* __restrict__ o, uint32_t* err,
                        const int32_t* __restrict__ slots, int num_slots) {
     state_role<false>(&tm_o, img, chunk_off, cu, total_T, H, max_total, s0, sT, o, err, slots, num_slots,
-                      blockIdx.x / H, blockIdx.x % H, Ring{nullptr, nullptr});
+                      blockIdx.x / H, blockIdx.x / H + 1, blockIdx.x % H, Ring{nullptr, nullptr});
 }
 
-// One sequence, both passes in one cooperative launch (all CTAs resident):
-// CTAs 0 .. H-1 carry the states of the H heads, the others prepare chunks
-// ahead of them through the ring.
+// Both passes in one cooperative launch (all CTAs resident): CTAs 0 .. H-1
+// carry the states of the H heads -- CTA h walks (sequence 0, head h),
+// (sequence 1, head h), ... in order, so every head has the same amount of
+// work -- and the others prepare chunks ahead of them through the ring, in
+// the global chunk order (chunk-major over heads).  A head's ring slot and
+// flags follow the global chunk index, which runs on across sequences.
 __global__ void __launch_bounds__(kThreads, 1)
 kda_chunk_overlap_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                          const __grid_constant__ CUtensorMap tm_o,
                          const float* __restrict__ g, const float* __restrict__ beta, const int32_t* __restrict__ cu,
-                         const int32_t* __restrict__ chunk_off, int H, int64_t total_T, int64_t max_total,
+                         const int32_t* __restrict__ chunk_off, int N, int H, int64_t total_T, int64_t max_total,
                          float scale, int l2norm, int scalar_g, uint8_t* __restrict__ img, const float* s0,
                          float* sT, float* __restrict__ o, uint32_t* err, const int32_t* __restrict__ slots,
                          int num_slots, Ring ring) {
     if (static_cast<int>(blockIdx.x) < H)
-        state_role<true>(&tm_o, img, chunk_off, cu, total_T, H, max_total, s0, sT, o, err, slots, num_slots, 0,
+        state_role<true>(&tm_o, img, chunk_off, cu, total_T, H, max_total, s0, sT, o, err, slots, num_slots, 0, N,
                          blockIdx.x, ring);
     else
-        prep_role<true>(&tm_q, &tm_k, &tm_v, &tm_g, g, beta, cu, chunk_off, 1, H, max_total, scale, l2norm, scalar_g, img,
-                        err, blockIdx.x - H, gridDim.x - H, ring);
+        prep_role<true>(&tm_q, &tm_k, &tm_v, &tm_g, g, beta, cu, chunk_off, N, H, max_total, scale, l2norm, scalar_g,
+                        img, err, blockIdx.x - H, gridDim.x - H, ring);
 }
 
 int num_sms() {
@@ -1027,10 +1066,11 @@ int num_sms() {
 size_t max_chunks(int32_t N, int64_t total_T) { return static_cast<size_t>((total_T + 63 * (int64_t)N) / kC); }
 size_t index_bytes(int32_t N) { return (static_cast<size_t>(N + 1) * 4 + 1023) & ~size_t(1023); }
 
-// Overlapped mode: one sequence, and enough SMs left for the prep role.
+// Overlapped mode: at most 96 heads (one state CTA each, with enough SMs left
+// for the prep role), any number of sequences.
 constexpr int kMinPrepCtas = 16;
 constexpr int kMaxRingHeads = 96;
-bool ring_eligible(int32_t N, int32_t H) { return N == 1 && H <= kMaxRingHeads; }
+bool ring_eligible(int32_t N, int32_t H) { return N >= 1 && H <= kMaxRingHeads; }
 size_t ring_flag_bytes(int32_t H) { return (static_cast<size_t>(H) * 2 * kFlagStride * 4 + 1023) & ~size_t(1023); }
 
 template <class K>
@@ -1051,12 +1091,12 @@ cudaError_t launch_chunk_two_pass(const PrefillArgs& a, void* scratch, cudaStrea
     if (a.N == 0 || a.H == 0) return cudaSuccess;
     if (a.total_T <= 0) return cudaErrorInvalidValue;   // callers route empty batches elsewhere
     constexpr uint32_t O_SMEM = P_SMEM > S_SMEM ? P_SMEM : S_SMEM;
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = set_smem(kda_chunk_prep_kernel, P_SMEM);
-        if (attr_err == cudaSuccess) attr_err = set_smem(kda_chunk_state_kernel, S_SMEM);
-        if (attr_err == cudaSuccess) attr_err = set_smem(kda_chunk_overlap_kernel, O_SMEM);
+    static PerDeviceOnce attr_once;
+    const cudaError_t attr_err = attr_once.run([] {
+        cudaError_t e = set_smem(kda_chunk_prep_kernel, P_SMEM);
+        if (e == cudaSuccess) e = set_smem(kda_chunk_state_kernel, S_SMEM);
+        if (e == cudaSuccess) e = set_smem(kda_chunk_overlap_kernel, O_SMEM);
+        return e;
     });
     if (attr_err != cudaSuccess) return attr_err;
     CUtensorMap mq, mk, mv, mg, mo;
@@ -1077,13 +1117,14 @@ cudaError_t launch_chunk_two_pass(const PrefillArgs& a, void* scratch, cudaStrea
             cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess ||
             cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kda_chunk_overlap_kernel, kThreads, O_SMEM) !=
                 cudaSuccess)
-            return cudaGetLastError();
+            return cudaErrorUnknown;
         if (!coop || per_sm < 1 || a.H + kMinPrepCtas > sms) return cudaErrorNotSupported;
         uint8_t* flags = static_cast<uint8_t*>(scratch) + index_bytes(a.N);
         Ring ring{reinterpret_cast<int32_t*>(flags), reinterpret_cast<int32_t*>(flags) + a.H * kFlagStride};
         uint8_t* img = flags + ring_flag_bytes(a.H);
-        kda_chunk_index_kernel<<<1, 1024, 0, stream>>>(a.cu_seqlens, a.N, a.total_T, max_total, chunk_off, a.err,
-                                                       ring.ready, a.H * 2 * kFlagStride);
+        cudaError_t e = launch_kernel(kda_chunk_index_kernel, dim3(1), dim3(1024), 0, stream, a.cu_seqlens, a.N,
+                                      a.total_T, max_total, chunk_off, a.err, ring.ready, a.H * 2 * kFlagStride);
+        if (e != cudaSuccess) return e;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(static_cast<unsigned>(sms));
         cfg.blockDim = dim3(kThreads);
@@ -1094,28 +1135,32 @@ cudaError_t launch_chunk_two_pass(const PrefillArgs& a, void* scratch, cudaStrea
         attr[0].val.cooperative = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        const cudaError_t e = cudaLaunchKernelEx(
+        e = cudaLaunchKernelEx(
             &cfg, kda_chunk_overlap_kernel, mq, mk, mv, mg, mo, a.g, a.beta, a.cu_seqlens,
-            static_cast<const int32_t*>(chunk_off), static_cast<int>(a.H), a.total_T, max_total, a.scale,
+            static_cast<const int32_t*>(chunk_off), static_cast<int>(a.N), static_cast<int>(a.H), a.total_T,
+            max_total, a.scale,
             a.l2norm ? 1 : 0, a.scalar_decay ? 1 : 0, img, a.initial_state, a.final_state, a.o, a.err, a.slots,
             static_cast<int>(a.num_slots), ring);
-        return e != cudaSuccess ? e : cudaGetLastError();
+        return e;
     }
 
     uint8_t* img = static_cast<uint8_t*>(scratch) + index_bytes(a.N);
-    kda_chunk_index_kernel<<<1, 1024, 0, stream>>>(a.cu_seqlens, a.N, a.total_T, max_total, chunk_off, a.err,
-                                                   nullptr, 0);
+    cudaError_t e = launch_kernel(kda_chunk_index_kernel, dim3(1), dim3(1024), 0, stream, a.cu_seqlens, a.N,
+                                  a.total_T, max_total, chunk_off, a.err, static_cast<int32_t*>(nullptr), 0);
+    if (e != cudaSuccess) return e;
     const size_t items_ub = max_chunks(a.N, a.total_T) * static_cast<size_t>(a.H);
     const size_t grid1 = items_ub < static_cast<size_t>(sms) ? items_ub : static_cast<size_t>(sms);
-    if (grid1 > 0)
-        kda_chunk_prep_kernel<<<static_cast<unsigned>(grid1), kThreads, P_SMEM, stream>>>(
-            mq, mk, mv, mg, a.g, a.beta, a.cu_seqlens, chunk_off, a.N, a.H, max_total, a.scale, a.l2norm ? 1 : 0,
-            a.scalar_decay ? 1 : 0, img, a.err);
+    if (grid1 > 0) {
+        e = launch_kernel(kda_chunk_prep_kernel, dim3(static_cast<unsigned>(grid1)), dim3(kThreads), P_SMEM, stream,
+                          mq, mk, mv, mg, a.g, a.beta, a.cu_seqlens, static_cast<const int32_t*>(chunk_off), a.N, a.H,
+                          max_total, a.scale, a.l2norm ? 1 : 0, a.scalar_decay ? 1 : 0, img, a.err);
+        if (e != cudaSuccess) return e;
+    }
     const long long blocks = (long long)a.N * a.H;
-    kda_chunk_state_kernel<<<static_cast<unsigned>(blocks), kThreads, S_SMEM, stream>>>(
-        mo, img, chunk_off, a.cu_seqlens, a.total_T, a.H, max_total, a.initial_state, a.final_state, a.o, a.err,
-        a.slots, a.num_slots);
-    return cudaGetLastError();
+    return launch_kernel(kda_chunk_state_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kThreads), S_SMEM, stream,
+                         mo, static_cast<const uint8_t*>(img), static_cast<const int32_t*>(chunk_off), a.cu_seqlens,
+                         a.total_T, a.H, max_total, a.initial_state, a.final_state, a.o, a.err, a.slots,
+                         static_cast<int>(a.num_slots));
 }
 
 }  // namespace kda

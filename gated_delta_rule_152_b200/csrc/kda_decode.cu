@@ -40,7 +40,10 @@ kda_decode_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __r
     size_t sp = static_cast<size_t>(p);
     if (slots) {
         const int n = p / H, h = p - n * H, slot = slots[n];
-        if (slot < 0 || slot >= num_slots) return;   // out-of-range slot: sequence skipped
+        if (slot < 0 || slot >= num_slots) {   // out-of-range slot: sequence skipped, its o marked NaN
+            if (warp == 0) reinterpret_cast<float4*>(o + (size_t)p * kD)[lane] = make_float4(NAN, NAN, NAN, NAN);
+            return;
+        }
         sp = static_cast<size_t>(slot) * H + h;
     }
     float4* S = reinterpret_cast<float4*>(state + sp * kD * kD);
@@ -138,16 +141,15 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
     const long long pairs = (long long)a.N * a.H;
     if (pairs == 0) return cudaSuccess;
     if (a.bf16)
-        kda_decode_kernel<__nv_bfloat16><<<(unsigned)pairs, kThreads, 0, stream>>>(
-            static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
-            static_cast<const __nv_bfloat16*>(a.v), a.g, a.beta, a.state, a.o, a.scale,
-            a.l2norm ? 1 : 0, a.scalar_decay ? 1 : 0, a.H, a.slots, a.num_slots);
-    else
-        kda_decode_kernel<float><<<(unsigned)pairs, kThreads, 0, stream>>>(
-            static_cast<const float*>(a.q), static_cast<const float*>(a.k),
-            static_cast<const float*>(a.v), a.g, a.beta, a.state, a.o, a.scale, a.l2norm ? 1 : 0,
-            a.scalar_decay ? 1 : 0, a.H, a.slots, a.num_slots);
-    return cudaGetLastError();
+        return launch_kernel(kda_decode_kernel<__nv_bfloat16>, dim3((unsigned)pairs), dim3(kThreads), 0, stream,
+                             static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
+                             static_cast<const __nv_bfloat16*>(a.v), a.g, a.beta, a.state, a.o, a.scale,
+                             a.l2norm ? 1 : 0, a.scalar_decay ? 1 : 0, static_cast<int>(a.H), a.slots,
+                             static_cast<int>(a.num_slots));
+    return launch_kernel(kda_decode_kernel<float>, dim3((unsigned)pairs), dim3(kThreads), 0, stream,
+                         static_cast<const float*>(a.q), static_cast<const float*>(a.k),
+                         static_cast<const float*>(a.v), a.g, a.beta, a.state, a.o, a.scale, a.l2norm ? 1 : 0,
+                         a.scalar_decay ? 1 : 0, static_cast<int>(a.H), a.slots, static_cast<int>(a.num_slots));
 }
 
 }  // namespace kda

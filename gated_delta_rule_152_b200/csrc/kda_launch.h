@@ -1,10 +1,51 @@
 // kda_launch.h -- host-side launchers of the KDA kernels (internal to libkda).
 #pragma once
 #include <cstdint>
+#include <mutex>
+#include <utility>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace kda {
+
+// Launch `kernel` with an explicit configuration and return this launch's own
+// status (cudaLaunchKernelEx's return value), so that an unrelated earlier
+// error left on the calling thread by other code is neither reported as ours
+// nor cleared.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                          Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// One-time set-up that CUDA keeps per device (a kernel's dynamic shared-memory
+// limit, for instance): run() calls fn once for each device that is current
+// when it is called, and returns that first outcome on every later call.
+class PerDeviceOnce {
+  public:
+    template <class Fn>
+    cudaError_t run(Fn fn) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+        std::lock_guard<std::mutex> lock(mu_);
+        if (!done_[dev]) {
+            err_[dev] = fn();
+            done_[dev] = true;
+        }
+        return err_[dev];
+    }
+
+  private:
+    static constexpr int kMaxDevices = 64;
+    std::mutex mu_;
+    bool done_[kMaxDevices] = {};
+    cudaError_t err_[kMaxDevices] = {};
+};
 
 struct PrefillArgs {
     const void* q;

@@ -55,18 +55,17 @@ kda_recurrent_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* 
 cudaError_t launch_recurrent(const PrefillArgs& a, cudaStream_t stream) {
     const unsigned grid = static_cast<unsigned>((long long)a.N * a.H * (kD / kSerialSlice));
     if (a.bf16)
-        kda_recurrent_kernel<__nv_bfloat16><<<grid, kThreads, 0, stream>>>(
-            static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
-            static_cast<const __nv_bfloat16*>(a.v), a.g, a.beta, a.cu_seqlens, a.total_T, a.H,
-            a.scale, a.l2norm ? 1 : 0, a.scalar_decay ? 1 : 0, a.initial_state, a.final_state, a.o, a.err,
-            a.slots, a.num_slots, a.snapshots);
-    else
-        kda_recurrent_kernel<float><<<grid, kThreads, 0, stream>>>(
-            static_cast<const float*>(a.q), static_cast<const float*>(a.k),
-            static_cast<const float*>(a.v), a.g, a.beta, a.cu_seqlens, a.total_T, a.H, a.scale,
-            a.l2norm ? 1 : 0, a.scalar_decay ? 1 : 0, a.initial_state, a.final_state, a.o, a.err, a.slots,
-            a.num_slots, a.snapshots);
-    return cudaGetLastError();
+        return launch_kernel(kda_recurrent_kernel<__nv_bfloat16>, dim3(grid), dim3(kThreads), 0, stream,
+                             static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
+                             static_cast<const __nv_bfloat16*>(a.v), a.g, a.beta, a.cu_seqlens, a.total_T,
+                             static_cast<int>(a.H), a.scale, a.l2norm ? 1 : 0, a.scalar_decay ? 1 : 0,
+                             a.initial_state, a.final_state, a.o, a.err, a.slots, static_cast<int>(a.num_slots),
+                             a.snapshots);
+    return launch_kernel(kda_recurrent_kernel<float>, dim3(grid), dim3(kThreads), 0, stream,
+                         static_cast<const float*>(a.q), static_cast<const float*>(a.k),
+                         static_cast<const float*>(a.v), a.g, a.beta, a.cu_seqlens, a.total_T, static_cast<int>(a.H),
+                         a.scale, a.l2norm ? 1 : 0, a.scalar_decay ? 1 : 0, a.initial_state, a.final_state, a.o,
+                         a.err, a.slots, static_cast<int>(a.num_slots), a.snapshots);
 }
 
 }  // namespace kda

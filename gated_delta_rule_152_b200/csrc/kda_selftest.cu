@@ -8,6 +8,7 @@
 
 #include "../../include/kda.h"
 #include "kda_common.cuh"
+#include "kda_launch.h"
 #include "sm100.cuh"
 
 namespace kda {
@@ -35,6 +36,8 @@ extern "C" KDA_API int kda_selftest_bounded_waits(void* workspace, size_t worksp
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (cudaMemsetAsync(workspace, 0, 8, s) != cudaSuccess) return KDA_ERR_CUDA;
     uint32_t* err = static_cast<uint32_t*>(workspace);
-    kda::kda_selftest_kernel<<<1, 32, 0, s>>>(err, reinterpret_cast<const int32_t*>(err + 1), polls);
-    return cudaGetLastError() == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    return kda::launch_kernel(kda::kda_selftest_kernel, dim3(1), dim3(32), 0, s, err,
+                              reinterpret_cast<const int32_t*>(err + 1), polls) == cudaSuccess
+               ? KDA_OK
+               : KDA_ERR_CUDA;
 }

@@ -307,7 +307,7 @@ __device__ __forceinline__ float4 sub4(float4 a, float4 b) {
 // tiles as the emit wrote them):
 //   xt  128 rows: rows 0-63 Q-side, rows 64-127 K-side;
 //   yt  64 rows;
-// level 1: xt = [q^ X ; k^ X], yt = k^ Y (block references, see above);
+// level 1: xt = [q^ X ; k^ X], yt = k^ Y rounded to tf32 (block references, see above);
 // level 2: xt = [q^ ; k^], yt = Gamma (log2), converted here in place to the
 //          level-1 tiles once the in-block pairs are done;
 // rho: [4][128] block-end Gammas (shared memory);  ztab: [10][128] scratch.
@@ -372,63 +372,87 @@ __device__ __forceinline__ void gram_exact(uint8_t* xt, uint32_t kbx, uint8_t* y
             const float4 X = ex2x4(sub4(g, prev)), Y = ex2x4(sub4(cur, g));
             *qp = mul4(q, X);
             *kp = mul4(kk, X);
-            *yp = mul4(kk, Y);
+            const float4 ky = mul4(kk, Y);
+            *yp = tf32x4(ky.x, ky.y, ky.z, ky.w);
         }
         __syncthreads();
     }
-    // block pairs on mma.sync (tf32, fp32 accumulation): unit u = 2 p + m is
-    // block pair p, matrix m (0: P from the Q-side rows, 1: A from the K-side
-    // rows); at level 2 only pairs of different blocks
+    // block pairs on mma.sync (tf32, fp32 accumulation): warp w takes the pairs
+    // w and w + 8 of the list (gram_pair), both matrices of each (P from the
+    // Q-side rows, A from the K-side rows), which share the K-side columns and
+    // the Z factors.  Every row a lane reads has (row mod 8) = lane / 4, so
+    // the swizzled chunk offsets are per-lane constants.
     const int gq = lane >> 2, tq = lane & 3;
-    float d[3][2][4];
-    int units[3];
-    const int nunits = level == 2 ? 12 : 20;
+    const int npairs = level == 2 ? 6 : 10;
+    float d[2][2][2][4];   // [pair slot][matrix][column half][fragment]
+    int pairs[2];
+    uint32_t swz[8];
 #pragma unroll
-    for (int s = 0; s < 3; ++s) {
-        const int u = warp + 8 * s;
-        units[s] = u < nunits ? u : -1;
-        if (units[s] < 0) continue;
-        const int p = gram_pair(u, level);
+    for (int j = 0; j < 8; ++j) swz[j] = (static_cast<uint32_t>(j ^ gq) << 4) + 4u * tq;
+#pragma unroll
+    for (int sl = 0; sl < 2; ++sl) {
+        const int q = warp + 8 * sl;
+        pairs[sl] = q < npairs ? gram_pair(2 * q, level) : -1;
+        if (pairs[sl] < 0) continue;
+        const int p = pairs[sl];
         const int a = (p >= 1) + (p >= 3) + (p >= 6), b = p - a * (a + 1) / 2;
-        const int m = u & 1, row0 = 64 * m + 16 * a;
         const float* z = ztab + p * kD;
+        const uint8_t* pq = xt + (16 * a + gq) * 128;          // Q-side row gq of block a
+        const uint8_t* pk = xt + (64 + 16 * a + gq) * 128;     // K-side row
+        const uint8_t* py = yt + (16 * b + gq) * 128;          // column rows of block b
 #pragma unroll
-        for (int nh = 0; nh < 2; ++nh)
+        for (int m = 0; m < 2; ++m)
 #pragma unroll
-            for (int x = 0; x < 4; ++x) d[s][nh][x] = 0.f;
-#pragma unroll 4
-        for (int k0 = 0; k0 < kD; k0 += 8) {
-            const float z0 = z[k0 + tq], z1 = z[k0 + tq + 4];
-            uint32_t fa[4];
-            fa[0] = tf32_bits(*K_at(xt, 0, kbx, row0 + gq, k0 + tq) * z0);
-            fa[1] = tf32_bits(*K_at(xt, 0, kbx, row0 + gq + 8, k0 + tq) * z0);
-            fa[2] = tf32_bits(*K_at(xt, 0, kbx, row0 + gq, k0 + tq + 4) * z1);
-            fa[3] = tf32_bits(*K_at(xt, 0, kbx, row0 + gq + 8, k0 + tq + 4) * z1);
+            for (int nh = 0; nh < 2; ++nh)
 #pragma unroll
-            for (int nh = 0; nh < 2; ++nh) {
-                const int col = 16 * b + 8 * nh + gq;
-                uint32_t fb[2];
-                fb[0] = tf32_bits(*K_at(yt, 0, kby, col, k0 + tq));
-                fb[1] = tf32_bits(*K_at(yt, 0, kby, col, k0 + tq + 4));
-                mma_m16n8k8_tf32(d[s][nh], fa, fb);
+                for (int x = 0; x < 4; ++x) d[sl][m][nh][x] = 0.f;
+#pragma unroll 1
+        for (int kbi = 0; kbi < 4; ++kbi) {
+            const uint8_t* bq = pq + kbi * kbx;
+            const uint8_t* bk = pk + kbi * kbx;
+            const uint8_t* by = py + kbi * kby;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int k0 = 32 * kbi + 8 * j;
+                const float z0 = z[k0 + tq], z1 = z[k0 + tq + 4];
+                const uint32_t o0 = swz[2 * j], o1 = swz[2 * j + 1];
+                uint32_t fa[2][4], fb[2][2];
+#pragma unroll
+                for (int m = 0; m < 2; ++m) {
+                    const uint8_t* r = m ? bk : bq;
+                    fa[m][0] = tf32_bits(*reinterpret_cast<const float*>(r + o0) * z0);
+                    fa[m][1] = tf32_bits(*reinterpret_cast<const float*>(r + 8 * 128 + o0) * z0);
+                    fa[m][2] = tf32_bits(*reinterpret_cast<const float*>(r + o1) * z1);
+                    fa[m][3] = tf32_bits(*reinterpret_cast<const float*>(r + 8 * 128 + o1) * z1);
+                }
+#pragma unroll
+                for (int nh = 0; nh < 2; ++nh) {   // the K-side tile is stored already rounded to tf32
+                    fb[nh][0] = *reinterpret_cast<const uint32_t*>(by + nh * 8 * 128 + o0);
+                    fb[nh][1] = *reinterpret_cast<const uint32_t*>(by + nh * 8 * 128 + o1);
+                }
+#pragma unroll
+                for (int m = 0; m < 2; ++m)
+#pragma unroll
+                    for (int nh = 0; nh < 2; ++nh) mma_m16n8k8_tf32(d[sl][m][nh], fa[m], fb[nh]);
             }
         }
     }
     __syncthreads();   // every input read
     mid();
 #pragma unroll
-    for (int s = 0; s < 3; ++s) {
-        if (units[s] < 0) continue;
-        const int u = units[s];
-        const int p = gram_pair(u, level);
+    for (int sl = 0; sl < 2; ++sl) {
+        if (pairs[sl] < 0) continue;
+        const int p = pairs[sl];
         const int a = (p >= 1) + (p >= 3) + (p >= 6), b = p - a * (a + 1) / 2;
-        const int row0 = 64 * (u & 1) + 16 * a;
 #pragma unroll
-        for (int nh = 0; nh < 2; ++nh) {
-            const int col = 16 * b + 8 * nh + 2 * tq;
-            *reinterpret_cast<float2*>(st + (row0 + gq) * kStLd + col) = make_float2(d[s][nh][0], d[s][nh][1]);
-            *reinterpret_cast<float2*>(st + (row0 + gq + 8) * kStLd + col) = make_float2(d[s][nh][2], d[s][nh][3]);
-        }
+        for (int m = 0; m < 2; ++m)
+#pragma unroll
+            for (int nh = 0; nh < 2; ++nh) {
+                const int row = 64 * m + 16 * a + gq, col = 16 * b + 8 * nh + 2 * tq;
+                *reinterpret_cast<float2*>(st + row * kStLd + col) = make_float2(d[sl][m][nh][0], d[sl][m][nh][1]);
+                *reinterpret_cast<float2*>(st + (row + 8) * kStLd + col) =
+                    make_float2(d[sl][m][nh][2], d[sl][m][nh][3]);
+            }
     }
     if (level == 2 && pcol <= prow) {
         *reinterpret_cast<float4*>(st + prow * kStLd + pcol) = make_float4(dq[0], dq[1], dq[2], dq[3]);

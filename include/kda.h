@@ -97,11 +97,11 @@ enum {
  * Bytes of device workspace with which kda_chunk_fwd (and _slots) runs its
  * fastest path for these sizes: the error word, a chunk index, and room for
  * the state-independent tensor-core operands of the (64-token chunk, head)
- * pairs, 145 KiB per pair.  One sequence with at most 96 heads needs a ring
- * of 8 such slots per head plus one 128-byte flag line per head and
- * direction (32 heads: about 38 MB, whatever the length); otherwise every
- * pair has its own slot (2 x 8192 tokens x 32 heads: about 613 MB).
- * Returns 0 for invalid sizes.
+ * pairs, 145 KiB per pair.  With at most 96 heads that is a ring of 8 such
+ * slots per head plus one 128-byte flag line per head and direction,
+ * whatever the number and lengths of the sequences (32 heads: about 38 MB);
+ * with more heads every pair has its own slot (2 x 8192 tokens x 100 heads:
+ * about 1.9 GB).  Returns 0 for invalid sizes.
  */
 KDA_API size_t kda_chunk_fwd_workspace_size(int32_t N, int64_t total_T, int32_t H, int32_t d,
                                     kda_dtype dt);
@@ -217,7 +217,9 @@ KDA_API int kda_chunk_fwd_slots(const void *q, const void *k, const void *v, con
 /*
  * kda_decode_step_slots: as kda_decode_step with state = state_pool[slots[n]],
  * updated in place.  A sequence whose slot is outside [0, num_slots) is
- * skipped (its state and o rows are left untouched).
+ * skipped: no state is read or written for it, and its o rows are set to NaN
+ * so that the skip shows in the output (decode has no workspace to report it
+ * in).
  */
 KDA_API int kda_decode_step_slots(const void *q, const void *k, const void *v, const float *g,
                           const float *beta, float *state_pool, const int32_t *slots,
@@ -263,6 +265,43 @@ KDA_API int kda_workspace_error(const void *workspace, uint32_t *out, kda_stream
  */
 KDA_API int kda_selftest_bounded_waits(void *workspace, size_t workspace_bytes, uint32_t polls,
                                        kda_stream_t stream);
+
+/*
+ * kda_topk_indices -- the selection step of the lightning indexer (page
+ * "GLM-5.3-FLASH", dimsnsums.com, section "How can a layer search the whole
+ * history selectively?": every past token gets a relevance score and the
+ * 2,048 highest are kept for full attention).  The page defines neither the
+ * score nor ties, so the scores are the caller's and the ranking is stated
+ * here: a higher score ranks higher; equal scores (-0 == +0) rank the lower
+ * index higher, which makes the kept set unique.
+ *
+ *   scores       [rows, ld] fp32 DEVICE array, 16-byte aligned, ld a multiple
+ *                of 4 and >= n; row r's scores are scores[r * ld + 0 .. n_r - 1].
+ *                NaN is not a score: a row holding NaN gets an unspecified
+ *                selection.
+ *   rows         query rows, 0 .. 65535.
+ *   n            tokens per row, < 2^31.
+ *   k            kept per row, 1 .. KDA_TOPK_MAX_K (2,048 on the page).
+ *   row_lengths  [rows] int32 DEVICE array or NULL: n_r = clamp(row_lengths[r],
+ *                0, n) (e.g. a causal prefill, where query r sees fewer
+ *                tokens); NULL: n_r = n.
+ *   indices      [rows, k] int32 out: the kept indices best first (descending
+ *                score, then ascending index); slots past n_r hold -1.
+ *   values       [rows, k] fp32 out or NULL: the kept scores in the same order
+ *                (-inf in the empty slots).
+ *   workspace    device scratch of kda_topk_workspace_size(rows, n, k) bytes,
+ *                256-byte aligned; its first word is cleared by the call.
+ * Returns KDA_OK once the kernels are enqueued, KDA_ERR_INVALID_ARG /
+ * _UNSUPPORTED / _MISALIGNED / _WORKSPACE for bad arguments (nothing is
+ * launched then).  The scores are read twice when the cut falls in a part of
+ * the score range that holds at most 16,384 of the row's tokens (the usual
+ * case), and a few more times otherwise.
+ */
+#define KDA_TOPK_MAX_K 4096
+KDA_API size_t kda_topk_workspace_size(int32_t rows, int64_t n, int32_t k);
+KDA_API int kda_topk_indices(const float *scores, int64_t ld, int32_t rows, int64_t n, int32_t k,
+                             const int32_t *row_lengths, int32_t *indices, float *values,
+                             void *workspace, size_t workspace_bytes, kda_stream_t stream);
 
 /* Static English description of a kda_status value. */
 KDA_API const char *kda_status_string(int status);

@@ -56,10 +56,14 @@ def test_workspace_size_ring_and_per_pair_scratch(lib):
     one = lib.kda_chunk_fwd_workspace_size(1, 8192, 32, 128, 0)
     assert 32 * 8 * slot <= one < 64 << 20           # one sequence: a ring of 8 slots per head
     assert lib.kda_chunk_fwd_workspace_size(1, 131072, 32, 128, 0) == one   # independent of length
+    # several sequences share each head's ring: the size hardly depends on their number
+    # or lengths (16 sequences of up to 16K tokens: under 40 MB, not 9.5 GB)
     two = lib.kda_chunk_fwd_workspace_size(2, 8192, 32, 128, 0)
-    assert two >= 128 * 32 * slot                    # several sequences: a slot per pair
+    sixteen = lib.kda_chunk_fwd_workspace_size(16, 135168, 32, 128, 0)
+    assert one <= two <= sixteen < 40 << 20
     many_heads = lib.kda_chunk_fwd_workspace_size(1, 8192, 100, 128, 0)
-    assert many_heads >= 128 * 100 * slot            # too many heads for the ring
+    assert many_heads >= 128 * 100 * slot            # too many heads for the ring: a slot per pair
+    assert lib.kda_chunk_fwd_workspace_size(2, 8192, 100, 128, 0) >= (128 + 1) * 100 * slot
     assert lib.kda_chunk_fwd_workspace_size_min(1, 8192, 32, 128, 0) < 4096
 
 
@@ -144,3 +148,28 @@ def test_selftest_rejects_bad_workspace(lib):
     assert lib.kda_selftest_bounded_waits(None, 256, 16, None) == kda.KDA_ERR_WORKSPACE
     assert lib.kda_selftest_bounded_waits(P(A), 64, 16, None) == kda.KDA_ERR_WORKSPACE
     assert lib.kda_selftest_bounded_waits(P(MIS), 256, 16, None) == kda.KDA_ERR_MISALIGNED
+
+
+def test_topk_host_validation(lib):
+    P = ctypes.c_void_p
+    ws = kda.kda_topk_workspace_size(4, 1000, 2048)
+    assert ws > 0 and kda.kda_topk_workspace_size(4, 1000, kda.KDA_TOPK_MAX_K + 1) == 0
+    assert kda.kda_topk_workspace_size(4, 1000, 0) == 0
+    # grows with rows and k
+    assert kda.kda_topk_workspace_size(8, 1000, 2048) > ws > kda.kda_topk_workspace_size(4, 1000, 64)
+    W = 0x100000          # fake 256-byte-aligned workspace
+    call = lambda scores, ld, rows, n, k, idx, ws_ptr=W, ws_bytes=ws, lengths=None, vals=None: \
+        lib.kda_topk_indices(P(scores) if scores else None, ld, rows, n, k, P(lengths) if lengths else None,
+                             P(idx) if idx else None, P(vals) if vals else None, P(ws_ptr) if ws_ptr else None,
+                             ws_bytes, None)
+    assert call(A, 1000, 4, 1000, 0, A) == kda.KDA_ERR_UNSUPPORTED              # k = 0
+    assert call(A, 1000, 4, 1000, 4097, A) == kda.KDA_ERR_UNSUPPORTED           # k above the maximum
+    assert call(A, 996, 4, 1000, 16, A) == kda.KDA_ERR_INVALID_ARG              # ld < n
+    assert call(A, 1000, 70000, 1000, 16, A) == kda.KDA_ERR_INVALID_ARG         # too many rows
+    assert call(A, 1000, 4, 1000, 16, None) == kda.KDA_ERR_INVALID_ARG          # no output
+    assert call(MIS, 1000, 4, 1000, 16, A) == kda.KDA_ERR_MISALIGNED            # scores not 16-byte aligned
+    assert call(A, 1002, 4, 1000, 16, A) == kda.KDA_ERR_MISALIGNED              # row stride not a multiple of 4
+    assert call(A, 1000, 4, 1000, 16, A, ws_ptr=None) == kda.KDA_ERR_WORKSPACE
+    assert call(A, 1000, 4, 1000, 16, A, ws_ptr=W + 16) == kda.KDA_ERR_WORKSPACE   # not 256-byte aligned
+    assert call(A, 1000, 4, 1000, 2048, A, ws_bytes=ws - 1) == kda.KDA_ERR_WORKSPACE
+    assert call(A, 1000, 0, 1000, 16, None) == kda.KDA_OK                       # nothing to do

@@ -58,11 +58,18 @@ def small_workspace(x: kin.PrefillInputs, dev):
 def run_both(x: kin.PrefillInputs, recurrent=False, scale=1.0, l2norm=True, heads=None, path="two_pass"):
     dev = torch.device("cuda")
     xd = x.to(dev)
-    ws = small_workspace(x, dev) if path == "fused" else None
+    T, H, _ = x.q.shape
+    N = x.cu_seqlens.numel() - 1
+    if path == "fused":
+        ws = small_workspace(x, dev)
+    else:
+        ws = torch.zeros(max(kda.kda_chunk_fwd_workspace_size(N, T, H, dtype=x.q.dtype), 256), dtype=torch.uint8,
+                         device=dev)
     o, sT = kda.kda_chunk_fwd(xd.q, xd.k, xd.v, xd.g, xd.beta, xd.cu_seqlens, scale=scale,
                               l2norm=l2norm, initial_state=xd.initial_state, recurrent=recurrent,
                               workspace=ws)
     torch.cuda.synchronize()
+    assert kda.kda_workspace_error(ws) == 0, "a kernel reported an error"
     sel = slice(None) if heads is None else list(heads)
     s0 = None if x.initial_state is None else x.initial_state[:, sel].contiguous()
     o_ref, s_ref = oracle.kda_forward(x.q[:, sel].contiguous(), x.k[:, sel].contiguous(),
@@ -381,6 +388,40 @@ def test_single_sequence_state_pool_overlapped_path():
     assert torch.equal(pool_d[[0, 1, 3]].cpu(), pool[[0, 1, 3]])
 
 
+def test_packed_sequences_with_many_heads_take_the_two_launch_path():
+    # more heads than the overlapped launch takes: the separate prep and state
+    # launches over several sequences, an empty one and a ragged tail included
+    x = kin.make_custom_prefill(55, [130, 0, 300, 7], heads=100, init_state_std=0.02)
+    o, s, o_ref, s_ref = run_both(x, heads=[0, 41, 99])
+    assert_close(o, o_ref, TOL_BF16, "o")
+    assert_close(s, s_ref, TOL_BF16, "final state")
+    assert torch.equal(s[1].cpu(), x.initial_state[1][[0, 41, 99]])   # the empty sequence
+
+
+def test_ring_with_a_bad_slot_hands_its_chunks_back():
+    # several sequences through the overlapped launch (state pool): the middle
+    # sequence's slot is out of range, so it is skipped, but the images made for
+    # it must still be handed back for the prep role to go on to the third one
+    dev = torch.device("cuda")
+    x = kin.make_custom_prefill(56, [700, 900, 650], heads=4, init_state_std=0.02)
+    xd = x.to(dev)
+    pool = torch.zeros(4, 4, 128, 128)
+    pool[0], pool[3] = x.initial_state[0], x.initial_state[2]
+    pool_d = pool.to(dev)
+    T, H = x.total_T, x.heads
+    ws = torch.zeros(kda.kda_chunk_fwd_workspace_size(3, T, H), dtype=torch.uint8, device=dev)
+    kda.kda_chunk_fwd_slots(xd.q, xd.k, xd.v, xd.g, xd.beta, xd.cu_seqlens, pool_d,
+                            torch.tensor([0, 9, 3], dtype=torch.int32, device=dev), workspace=ws)
+    err = kda.kda_workspace_error(ws)
+    assert err & kda.KDA_DEVERR_SLOT and not err & kda.KDA_DEVERR_TIMEOUT
+    for n, slot in ((0, 0), (2, 3)):
+        cu = x.cu_seqlens.tolist()
+        sl = slice(cu[n], cu[n + 1])
+        _, s_ref = oracle.kda_forward(x.q[sl], x.k[sl], x.v[sl], x.g[sl], x.beta[sl], [0, cu[n + 1] - cu[n]],
+                                      x.initial_state[n:n + 1])
+        assert_close(pool_d[slot:slot + 1], s_ref, TOL_BF16, f"pooled final state of sequence {n}")
+
+
 def test_single_sequence_with_many_heads_takes_the_two_launch_path():
     # more heads than the overlapped launch gives state CTAs to: one sequence
     # through the separate prep and state launches
@@ -428,13 +469,14 @@ def test_decode_with_state_pool():
     assert_close(pool_d[slots], s_ref, TOL_FP32, "pooled states")
     untouched = [i for i in range(10) if i not in slots]
     assert torch.equal(pool_d[untouched].cpu(), pool[untouched])
-    # an out-of-range slot skips that sequence and touches nothing
+    # an out-of-range slot skips that sequence: no state is touched and its o rows are NaN
     o2 = torch.full((4, 3, 128), 5.0, device=dev)
     before = pool_d.clone()
     kda.kda_decode_step_slots(td.q, td.k, td.v, td.g, td.beta, pool_d,
                               torch.tensor([7, -1, 9, 10], dtype=torch.int32, device=dev), o=o2)
     torch.cuda.synchronize()
-    assert torch.all(o2[1] == 5.0) and torch.all(o2[3] == 5.0)
+    assert torch.isnan(o2[1]).all() and torch.isnan(o2[3]).all()
+    assert torch.isfinite(o2[0]).all() and torch.isfinite(o2[2]).all()
     assert torch.equal(pool_d[[2, 0]], before[[2, 0]])
 
 
@@ -477,8 +519,8 @@ def test_bounded_waits_give_up_with_an_error_and_the_context_survives():
 
 @pytest.mark.parametrize("lengths", [[700], [300, 450]])
 def test_prefill_replays_from_a_cuda_graph(lengths):
-    # the overlapped (one sequence) and two-launch (two sequences) paths,
-    # captured once and replayed: the same bits as the eager call
+    # the overlapped launch for one and for two sequences, captured once and
+    # replayed: the same bits as the eager call
     dev = torch.device("cuda")
     x = kin.make_custom_prefill(61, lengths, heads=4, init_state_std=0.02).to(dev)
     T, H, d = x.q.shape
