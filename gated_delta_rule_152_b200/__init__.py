@@ -16,6 +16,8 @@ from .kda import (  # noqa: F401
     kda_decode_step_slots,
     kda_selftest_bounded_waits,
     kda_status_string,
+    kda_topk_indices,
+    kda_topk_workspace_size,
     kda_verify_fwd,
     kda_workspace_error,
     load_library,

@@ -1,0 +1,457 @@
+// kda_topk.cu -- the selection step of the lightning indexer: per query row,
+// the k highest of n per-token relevance scores (page "GLM-5.3-FLASH",
+// dimsnsums.com, section "How can a layer search the whole history
+// selectively?": every past token is scored and the 2,048 highest are kept).
+//
+// Order of tokens: a higher score ranks higher; equal scores (-0 == +0) rank
+// the lower index higher, so the kept set is unique.  The output lists the
+// kept indices best first; -1 fills the slots past n when n < k.
+//
+// Scores become 32-bit keys whose unsigned order is the float order (sign
+// bit set for positives, all bits inverted for negatives), and the cut is
+// found by radix selection on the keys, most significant digit first:
+//   1. hist0 (many CTAs per row): histogram of the top 11 key bits;
+//   2. pick0 (one CTA per row): the top-digit bin b holding the k-th best key;
+//   3. split (many CTAs per row): keys above bin b are kept outright, keys in
+//      bin b become candidates (when there are at most kTopkCap of them);
+//   4. finish (one CTA per row): the remaining digits (and, for equal keys at
+//      the cut, the index digits) among the candidates -- or over the whole
+//      row when bin b holds more than kTopkCap keys -- then a bitonic sort of
+//      the k kept (key, index) pairs, best first.
+// HBM traffic in the common case: the scores are read twice (steps 1 and 3).
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/kda.h"
+#include "kda_common.cuh"
+#include "kda_launch.h"
+
+namespace kda {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kBins = 2048;               // 11-bit digits
+constexpr int kSeg = 16384;               // scores per CTA in the row-parallel passes
+constexpr int kTopkMaxK = 4096;
+constexpr int kTopkCap = 16384;           // candidates kept per row for the finish step
+
+struct RowState {
+    int32_t n;        // tokens in the row
+    int32_t need;     // keys still to take from bin b
+    uint32_t b;       // top-digit bin of the cut
+    int32_t cnt_b;    // keys in bin b
+    int32_t nsel;     // kept pairs written to the row's buffer
+    int32_t ncand;    // candidates written
+    int32_t mode;     // 0: n <= k, keep all; 1: candidates; 2: bin b too full, the finish step scans the row
+    int32_t pad[9];
+};
+static_assert(sizeof(RowState) == 64, "row state");
+
+// Workspace (after the 256-byte header with the error word): per row its
+// state, then [rows][kBins] histogram counts, [rows][k] kept pairs and
+// [rows][kTopkCap] candidates.
+struct Layout {
+    RowState* st;
+    uint32_t* hist;
+    unsigned long long* kept;
+    unsigned long long* cand;
+};
+__host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+__host__ __device__ inline Layout layout(void* ws, int rows, int k) {
+    uint8_t* p = static_cast<uint8_t*>(ws) + 256;
+    Layout l;
+    l.st = reinterpret_cast<RowState*>(p);
+    p += align256(sizeof(RowState) * static_cast<size_t>(rows));
+    l.hist = reinterpret_cast<uint32_t*>(p);
+    p += align256(sizeof(uint32_t) * kBins * static_cast<size_t>(rows));
+    l.kept = reinterpret_cast<unsigned long long*>(p);
+    p += align256(sizeof(unsigned long long) * static_cast<size_t>(k) * rows);
+    l.cand = reinterpret_cast<unsigned long long*>(p);
+    return l;
+}
+inline size_t workspace_bytes(int rows, int k) {
+    return 256 + align256(sizeof(RowState) * static_cast<size_t>(rows)) +
+           align256(sizeof(uint32_t) * kBins * static_cast<size_t>(rows)) +
+           align256(sizeof(unsigned long long) * static_cast<size_t>(k) * rows) +
+           sizeof(unsigned long long) * static_cast<size_t>(kTopkCap) * rows;
+}
+
+// Order-preserving key of a score; -0 and +0 get the same key.
+__device__ __forceinline__ uint32_t score_key(float x) {
+    uint32_t u = __float_as_uint(x);
+    if ((u << 1) == 0u) u = 0u;
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_score(uint32_t key) {
+    return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+// A kept (key, index) pair as one 64-bit value whose unsigned order is the
+// ranking: the key, then the lower index first.
+__device__ __forceinline__ unsigned long long pair_of(uint32_t key, int32_t idx) {
+    return (static_cast<unsigned long long>(key) << 32) | static_cast<uint32_t>(~idx);
+}
+
+__device__ __forceinline__ int row_len(const int32_t* lengths, int r, int64_t n) {
+    if (!lengths) return static_cast<int>(n);
+    const int64_t l = lengths[r];
+    return static_cast<int>(l < 0 ? 0 : (l > n ? n : l));
+}
+
+// First index >= lo whose score sits on a 16-byte boundary (rows need only be
+// 4-byte aligned, so the row stride may be any number of scores).
+__device__ __forceinline__ int aligned_from(const float* row, int lo) {
+    const int mis = static_cast<int>((reinterpret_cast<uintptr_t>(row + lo) >> 2) & 3u);
+    return lo + ((4 - mis) & 3);
+}
+
+// Visit the scores [lo, hi) of one row as (index, key), 4 at a time where aligned.
+template <class F>
+__device__ __forceinline__ void for_keys(const float* row, int lo, int hi, int t, int nt, F f) {
+    const int lo4 = aligned_from(row, lo), hi4 = lo4 + ((hi - lo4) & ~3);
+    if (lo4 >= hi) {
+        for (int i = lo + t; i < hi; i += nt) f(i, score_key(__ldg(row + i)));
+        return;
+    }
+    for (int i = lo + t; i < lo4; i += nt) f(i, score_key(__ldg(row + i)));
+#pragma unroll 4
+    for (int i = lo4 + 4 * t; i < hi4; i += 4 * nt) {
+        const float4 v = __ldcs(reinterpret_cast<const float4*>(row + i));
+        f(i, score_key(v.x));
+        f(i + 1, score_key(v.y));
+        f(i + 2, score_key(v.z));
+        f(i + 3, score_key(v.w));
+    }
+    for (int i = hi4 + t; i < hi; i += nt) f(i, score_key(__ldg(row + i)));
+}
+
+// Warp-aggregated append of (key, idx) to a per-row buffer with a shared counter.
+__device__ __forceinline__ void append(bool take, unsigned long long v, int32_t* counter,
+                                       unsigned long long* buf, int cap) {
+    const unsigned m = __ballot_sync(0xffffffffu, take);
+    if (!m) return;
+    const int lane = threadIdx.x & 31, leader = __ffs(m) - 1;
+    int base = 0;
+    if (lane == leader) base = atomicAdd(counter, __popc(m));
+    base = __shfl_sync(0xffffffffu, base, leader);
+    if (take) {
+        const int pos = base + __popc(m & ((1u << lane) - 1u));
+        if (pos < cap) buf[pos] = v;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads) kda_topk_init_kernel(const int32_t* lengths, int64_t n, int k, Layout L) {
+    const int r = blockIdx.x;
+    if (threadIdx.x == 0) {
+        RowState s = {};
+        s.n = row_len(lengths, r, n);
+        s.mode = s.n <= k ? 0 : 1;
+        L.st[r] = s;
+    }
+    for (int i = threadIdx.x; i < kBins; i += kThreads) L.hist[static_cast<size_t>(r) * kBins + i] = 0u;
+}
+
+// Histogram of the top 11 key bits of one segment of one row (counts of each
+// pair of warps in shared memory, then one global add per non-empty bin).
+constexpr int kSubHists = kThreads / 64;
+__global__ void __launch_bounds__(kThreads) kda_topk_hist0_kernel(const float* __restrict__ scores, int64_t ld,
+                                                                  Layout L) {
+    __shared__ uint32_t h[kSubHists][kBins];
+    const int r = blockIdx.y;
+    const RowState s = L.st[r];
+    const int lo = blockIdx.x * kSeg, hi = min(s.n, lo + kSeg);
+    if (s.mode == 0 || lo >= hi) return;
+    const int sub = threadIdx.x >> 6;
+    for (int i = threadIdx.x; i < kSubHists * kBins; i += kThreads) (&h[0][0])[i] = 0u;
+    __syncthreads();
+    for_keys(scores + r * ld, lo, hi, threadIdx.x, kThreads,
+             [&](int, uint32_t key) { atomicAdd(&h[sub][key >> 21], 1u); });
+    __syncthreads();
+    for (int b = threadIdx.x; b < kBins; b += kThreads) {
+        uint32_t c = 0;
+#pragma unroll
+        for (int w = 0; w < kSubHists; ++w) c += h[w][b];
+        if (c) atomicAdd(&L.hist[static_cast<size_t>(r) * kBins + b], c);
+    }
+}
+
+// Block-wide search over a 2048-bin histogram `h` (shared memory) for the bin
+// that holds the `need`-th element counted from the top (from_top) or from
+// the bottom.  Returns the bin; *before receives the count of the bins
+// passed over first.  All threads call it; two block barriers inside.
+__device__ __forceinline__ int find_bin(const uint32_t* h, int need, bool from_top, int* before, int* scratch) {
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    constexpr int per = kBins / kThreads;   // 8 bins per thread, thread 0 first in visiting order
+    if (t == 0) scratch[32] = scratch[33] = 0;
+    uint32_t c[per], sum = 0;
+#pragma unroll
+    for (int j = 0; j < per; ++j) {
+        const int b = from_top ? kBins - 1 - (per * t + j) : per * t + j;
+        c[j] = h[b];
+        sum += c[j];
+    }
+    // exclusive scan of the per-thread sums in visiting order
+    uint32_t x = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) scratch[warp] = static_cast<int>(x);
+    __syncthreads();
+    uint32_t woff = 0;
+    for (int w = 0; w < warp; ++w) woff += static_cast<uint32_t>(scratch[w]);
+    uint32_t run = woff + x - sum;
+    if (run < static_cast<uint32_t>(need) && run + sum >= static_cast<uint32_t>(need)) {
+#pragma unroll
+        for (int j = 0; j < per; ++j) {
+            if (run + c[j] >= static_cast<uint32_t>(need)) {
+                scratch[32] = from_top ? kBins - 1 - (per * t + j) : per * t + j;
+                scratch[33] = static_cast<int>(run);
+                break;
+            }
+            run += c[j];
+        }
+    }
+    __syncthreads();
+    *before = scratch[33];
+    return scratch[32];
+}
+
+__global__ void __launch_bounds__(kThreads) kda_topk_pick0_kernel(int k, Layout L) {
+    __shared__ uint32_t h[kBins];
+    __shared__ int scratch[40];
+    const int r = blockIdx.x;
+    RowState s = L.st[r];
+    if (s.mode == 0) return;
+    for (int i = threadIdx.x; i < kBins; i += kThreads) h[i] = L.hist[static_cast<size_t>(r) * kBins + i];
+    __syncthreads();
+    int above = 0;
+    const int b = find_bin(h, k, true, &above, scratch);
+    if (threadIdx.x == 0) {
+        s.b = static_cast<uint32_t>(b);
+        s.need = k - above;
+        s.cnt_b = static_cast<int>(h[b]);
+        s.mode = s.cnt_b <= kTopkCap ? 1 : 2;
+        L.st[r] = s;
+    }
+}
+
+// Keys above bin b are kept, keys in bin b are candidates (mode 1); every key
+// is kept when the row has at most k tokens (mode 0).
+__global__ void __launch_bounds__(kThreads) kda_topk_split_kernel(const float* __restrict__ scores, int64_t ld,
+                                                                  int k, Layout L) {
+    const int r = blockIdx.y;
+    RowState* sp = L.st + r;
+    const RowState s = *sp;
+    const int lo = blockIdx.x * kSeg, hi = min(s.n, lo + kSeg);
+    if (s.mode == 2) return;
+    unsigned long long* kept = L.kept + static_cast<size_t>(r) * k;
+    unsigned long long* cand = L.cand + static_cast<size_t>(r) * kTopkCap;
+    // whole warps iterate together so that the warp-wide append sees every lane;
+    // four scores per thread and step between 16-byte boundaries
+    const float* row = scores + r * ld;
+    auto visit = [&](int i, uint32_t key, bool live) {
+        const uint32_t top = key >> 21;
+        append(live && (s.mode == 0 || top > s.b), pair_of(key, i), &sp->nsel, kept, k);
+        if (s.mode == 1) append(live && top == s.b, pair_of(key, i), &sp->ncand, cand, kTopkCap);
+    };
+    if (hi <= lo) return;
+    const int lo4 = min(aligned_from(row, lo), hi), hi4 = lo4 + ((hi - lo4) & ~3);
+    if (threadIdx.x < 32) {   // up to three scores before the first 16-byte boundary: one warp
+        const int i = lo + static_cast<int>(threadIdx.x);
+        const bool live = i < lo4;
+        visit(i, live ? score_key(row[i]) : 0u, live);
+    }
+    for (int base = lo4; base < hi4; base += 4 * kThreads) {
+        const int i = base + 4 * static_cast<int>(threadIdx.x);
+        const bool live = i < hi4;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (live) v = __ldcs(reinterpret_cast<const float4*>(row + i));
+        visit(i, score_key(v.x), live);
+        visit(i + 1, score_key(v.y), live);
+        visit(i + 2, score_key(v.z), live);
+        visit(i + 3, score_key(v.w), live);
+    }
+    if (threadIdx.x < 32) {   // up to three scores after the last boundary: one warp
+        const int i = hi4 + static_cast<int>(threadIdx.x);
+        const bool live = i < hi;
+        visit(i, live ? score_key(row[i]) : 0u, live);
+    }
+}
+
+// One CTA per row: the rest of the cut, the kept set, and the sorted output.
+__global__ void __launch_bounds__(kThreads) kda_topk_finish_kernel(const float* __restrict__ scores, int64_t ld,
+                                                                   int k, Layout L, int32_t* __restrict__ out_idx,
+                                                                   float* __restrict__ out_val) {
+    __shared__ uint32_t h[kBins];
+    __shared__ int scratch[40];
+    __shared__ unsigned long long sorted[kTopkMaxK];
+    const int r = blockIdx.x, t = threadIdx.x;
+    RowState* sp = L.st + r;
+    const RowState s = *sp;
+    unsigned long long* kept = L.kept + static_cast<size_t>(r) * k;
+    const unsigned long long* cand = L.cand + static_cast<size_t>(r) * kTopkCap;
+    const float* row = scores + r * ld;
+
+    if (s.mode != 0) {
+        // the source of the remaining selection: the candidates (mode 1) or the whole row (mode 2);
+        // visit(f) calls f(key, idx) for every key of bin b (the caller filters further)
+        auto visit = [&](auto f) {
+            if (s.mode == 1) {
+                for (int i = t; i < s.cnt_b; i += kThreads) {
+                    const unsigned long long v = cand[i];
+                    f(static_cast<uint32_t>(v >> 32), static_cast<int32_t>(~static_cast<uint32_t>(v)));
+                }
+            } else {
+                for_keys(row, 0, s.n, t, kThreads, [&](int i, uint32_t key) {
+                    if ((key >> 21) == s.b) f(key, i);
+                });
+            }
+        };
+        // remaining key digits: bits 20..10, then 9..0
+        uint32_t prefix = s.b << 21, mask = 0xFFE00000u;
+        int need = s.need, eq_total = 0;
+        for (int pass = 0; pass < 2; ++pass) {
+            const int shift = pass == 0 ? 10 : 0;
+            const uint32_t dmask = pass == 0 ? 0x7FFu : 0x3FFu;
+            for (int i = t; i < kBins; i += kThreads) h[i] = 0u;
+            __syncthreads();
+            visit([&](uint32_t key, int32_t) {
+                if ((key & mask) == prefix) atomicAdd(&h[(key >> shift) & dmask], 1u);
+            });
+            __syncthreads();
+            int above = 0;
+            const int bin = find_bin(h, need, true, &above, scratch);
+            prefix |= static_cast<uint32_t>(bin) << shift;
+            mask |= dmask << shift;
+            need -= above;
+            eq_total = static_cast<int>(h[bin]);
+            __syncthreads();
+        }
+        const uint32_t T = prefix;   // the key at the cut; `need` of the eq_total keys equal to it are kept
+        // ties at the cut: the need-th smallest index among the keys equal to T (index bits 30..20, 19..10, 9..0)
+        int32_t last = 0x7FFFFFFF;
+        if (need < eq_total) {
+            uint32_t ip = 0, im = 0;
+            for (int pass = 0; pass < 3; ++pass) {
+                const int shift = pass == 0 ? 20 : (pass == 1 ? 10 : 0);
+                const uint32_t dmask = pass == 0 ? 0x7FFu : 0x3FFu;
+                for (int i = t; i < kBins; i += kThreads) h[i] = 0u;
+                __syncthreads();
+                visit([&](uint32_t key, int32_t idx) {
+                    const uint32_t u = static_cast<uint32_t>(idx);
+                    if (key == T && (u & im) == ip) atomicAdd(&h[(u >> shift) & dmask], 1u);
+                });
+                __syncthreads();
+                int below = 0;
+                const int bin = find_bin(h, need, false, &below, scratch);
+                ip |= static_cast<uint32_t>(bin) << shift;
+                im |= dmask << shift;
+                need -= below;
+                __syncthreads();
+            }
+            last = static_cast<int32_t>(ip);
+        }
+        // keep the keys above the cut and the equal keys up to index `last`
+        // (whole warps iterate together for the warp-wide append)
+        if (s.mode == 1) {
+            for (int base = 0; base < s.cnt_b; base += kThreads) {
+                const int i = base + t;
+                unsigned long long v = 0;
+                bool take = false;
+                if (i < s.cnt_b) {
+                    v = cand[i];
+                    const uint32_t key = static_cast<uint32_t>(v >> 32);
+                    const int32_t idx = static_cast<int32_t>(~static_cast<uint32_t>(v));
+                    take = key > T || (key == T && idx <= last);
+                }
+                append(take, v, &sp->nsel, kept, k);
+            }
+        } else {
+            for (int base = 0; base < s.n; base += kThreads) {
+                const int i = base + t;
+                bool take = false;
+                unsigned long long v = 0;
+                if (i < s.n) {
+                    const uint32_t key = score_key(row[i]);
+                    v = pair_of(key, i);
+                    take = key > T || (key == T && i <= last);
+                }
+                append(take, v, &sp->nsel, kept, k);
+            }
+        }
+        __syncthreads();
+    }
+    __threadfence_block();
+    // bitonic sort, best first, of the m kept pairs (padded with zeros, which rank last)
+    const int m = s.n < k ? s.n : k;
+    int P = 1;
+    while (P < m) P <<= 1;
+    for (int i = t; i < P; i += kThreads) sorted[i] = i < m ? kept[i] : 0ull;
+    __syncthreads();
+    for (int size = 2; size <= P; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int i = t; i < P / 2; i += kThreads) {
+                const int lo = 2 * i - (i & (stride - 1)), hi = lo + stride;
+                const bool desc = (lo & size) == 0;   // descending runs build the final descending order
+                const unsigned long long a = sorted[lo], b = sorted[hi];
+                if ((a < b) == desc) {
+                    sorted[lo] = b;
+                    sorted[hi] = a;
+                }
+            }
+            __syncthreads();
+        }
+    }
+    for (int i = t; i < k; i += kThreads) {
+        const bool live = i < m;
+        const unsigned long long v = live ? sorted[i] : 0ull;
+        out_idx[static_cast<size_t>(r) * k + i] = live ? static_cast<int32_t>(~static_cast<uint32_t>(v)) : -1;
+        if (out_val)
+            out_val[static_cast<size_t>(r) * k + i] = live ? key_score(static_cast<uint32_t>(v >> 32)) : -INFINITY;
+    }
+}
+
+}  // namespace
+}  // namespace kda
+
+extern "C" {
+
+size_t kda_topk_workspace_size(int32_t rows, int64_t n, int32_t k) {
+    if (rows < 0 || n < 0 || n >= (int64_t(1) << 31) || k < 1 || k > kda::kTopkMaxK) return 0;
+    return kda::workspace_bytes(rows, k);
+}
+
+int kda_topk_indices(const float* scores, int64_t ld, int32_t rows, int64_t n, int32_t k,
+                     const int32_t* row_lengths, int32_t* indices, float* values, void* workspace,
+                     size_t workspace_bytes, kda_stream_t stream) {
+    using namespace kda;
+    if (rows < 0 || n < 0 || n >= (int64_t(1) << 31) || ld < n || rows > 65535) return KDA_ERR_INVALID_ARG;
+    if (k < 1 || k > kTopkMaxK) return KDA_ERR_UNSUPPORTED;
+    if (rows == 0) return KDA_OK;
+    if (!indices || (n > 0 && !scores)) return KDA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(scores) & 3u) || (reinterpret_cast<uintptr_t>(indices) & 3u) ||
+        (reinterpret_cast<uintptr_t>(values) & 3u) || (reinterpret_cast<uintptr_t>(row_lengths) & 3u))
+        return KDA_ERR_MISALIGNED;
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < kda_topk_workspace_size(rows, n, k))
+        return KDA_ERR_WORKSPACE;
+    int dev = 0, major = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    if (major != 10) return KDA_ERR_UNSUPPORTED;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const Layout L = layout(workspace, rows, k);
+    const unsigned segs = static_cast<unsigned>((n + kSeg - 1) / kSeg > 0 ? (n + kSeg - 1) / kSeg : 1);
+    const dim3 grid2(segs, static_cast<unsigned>(rows));
+    cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(uint32_t), s);
+    if (e == cudaSuccess) e = launch_kernel(kda_topk_init_kernel, dim3(rows), dim3(kThreads), 0, s, row_lengths, n, k, L);
+    if (e == cudaSuccess) e = launch_kernel(kda_topk_hist0_kernel, grid2, dim3(kThreads), 0, s, scores, ld, L);
+    if (e == cudaSuccess) e = launch_kernel(kda_topk_pick0_kernel, dim3(rows), dim3(kThreads), 0, s, k, L);
+    if (e == cudaSuccess) e = launch_kernel(kda_topk_split_kernel, grid2, dim3(kThreads), 0, s, scores, ld, k, L);
+    if (e == cudaSuccess)
+        e = launch_kernel(kda_topk_finish_kernel, dim3(rows), dim3(kThreads), 0, s, scores, ld, k, L, indices, values);
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+}  // extern "C"

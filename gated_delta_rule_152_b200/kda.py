@@ -37,8 +37,9 @@ KDA_DEVERR_SLOT = 4
 EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd_workspace_size_min", "kda_chunk_fwd",
             "kda_chunk_fwd_noalloc", "kda_decode_step",
             "kda_chunk_fwd_slots", "kda_decode_step_slots", "kda_verify_fwd", "kda_workspace_error",
-            "kda_selftest_bounded_waits",
+            "kda_selftest_bounded_waits", "kda_topk_workspace_size", "kda_topk_indices",
             "kda_status_string")
+KDA_TOPK_MAX_K = 4096
 
 _lock = threading.Lock()
 _lib = None
@@ -87,6 +88,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         lib.kda_workspace_error.restype = ctypes.c_int
         lib.kda_selftest_bounded_waits.argtypes = [P, SZ, U32, P]
         lib.kda_selftest_bounded_waits.restype = ctypes.c_int
+        lib.kda_topk_workspace_size.argtypes = [I32, I64, I32]
+        lib.kda_topk_workspace_size.restype = SZ
+        lib.kda_topk_indices.argtypes = [P, I64, I32, I64, I32, P, P, P, P, SZ, P]
+        lib.kda_topk_indices.restype = ctypes.c_int
         lib.kda_status_string.argtypes = [ctypes.c_int]
         lib.kda_status_string.restype = ctypes.c_char_p
         _lib = lib
@@ -397,3 +402,47 @@ def kda_workspace_error(workspace: torch.Tensor, stream=None) -> int:
     if st != KDA_OK:
         raise KdaError(st, "kda_workspace_error")
     return int(out.value)
+
+
+def kda_topk_workspace_size(rows: int, n: int, k: int = 2048) -> int:
+    return int(load_library().kda_topk_workspace_size(rows, n, k))
+
+
+def kda_topk_indices(scores, k: int = 2048, *, row_lengths: Optional[torch.Tensor] = None,
+                     indices: Optional[torch.Tensor] = None, values=False,
+                     workspace: Optional[torch.Tensor] = None, stream=None):
+    """The lightning indexer's selection: per row of ``scores`` ([rows, n]
+    fp32 CUDA tensor whose rows are contiguous, any row stride), the indices
+    of the k highest scores, best first, ties to the lower index, -1 past the
+    row's length.  ``row_lengths``: optional [rows] int32 tokens per row.
+    Returns ``indices`` [rows, k] int32 (and the kept scores [rows, k] fp32 if
+    ``values`` is True or a tensor)."""
+    lib = load_library()
+    if scores.device.type != "cuda" or scores.dtype != torch.float32 or scores.dim() != 2:
+        raise ValueError("scores must be a 2-D float32 CUDA tensor")
+    if scores.stride(1) != 1:
+        raise ValueError("scores rows must be contiguous")
+    rows, n = scores.shape
+    ld = scores.stride(0) if rows > 1 else n
+    dev = scores.device
+    if row_lengths is not None:
+        _check(row_lengths, "row_lengths", (rows,), torch.int32, dev)
+    if indices is None:
+        indices = torch.empty((rows, k), dtype=torch.int32, device=dev)
+    _check(indices, "indices", (rows, k), torch.int32, dev)
+    vals = None
+    if values is True:
+        vals = torch.empty((rows, k), dtype=torch.float32, device=dev)
+    elif isinstance(values, torch.Tensor):
+        vals = values
+        _check(vals, "values", (rows, k), torch.float32, dev)
+    need = int(lib.kda_topk_workspace_size(rows, n, k))
+    if need == 0:
+        raise ValueError("unsupported sizes for kda_topk_indices")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    st = lib.kda_topk_indices(_ptr(scores), ld, rows, n, k, _ptr(row_lengths), _ptr(indices), _ptr(vals),
+                              _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_topk_indices")
+    return (indices, vals) if vals is not None else indices

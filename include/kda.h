@@ -275,8 +275,8 @@ KDA_API int kda_selftest_bounded_waits(void *workspace, size_t workspace_bytes, 
  * here: a higher score ranks higher; equal scores (-0 == +0) rank the lower
  * index higher, which makes the kept set unique.
  *
- *   scores       [rows, ld] fp32 DEVICE array, 16-byte aligned, ld a multiple
- *                of 4 and >= n; row r's scores are scores[r * ld + 0 .. n_r - 1].
+ *   scores       [rows, ld] fp32 DEVICE array, 4-byte aligned, ld >= n (any
+ *                row stride); row r's scores are scores[r * ld + 0 .. n_r - 1].
  *                NaN is not a score: a row holding NaN gets an unspecified
  *                selection.
  *   rows         query rows, 0 .. 65535.
@@ -289,6 +289,7 @@ KDA_API int kda_selftest_bounded_waits(void *workspace, size_t workspace_bytes, 
  *                score, then ascending index); slots past n_r hold -1.
  *   values       [rows, k] fp32 out or NULL: the kept scores in the same order
  *                (-inf in the empty slots).
+ *   indices / values / row_lengths: 4-byte aligned.
  *   workspace    device scratch of kda_topk_workspace_size(rows, n, k) bytes,
  *                256-byte aligned; its first word is cleared by the call.
  * Returns KDA_OK once the kernels are enqueued, KDA_ERR_INVALID_ARG /

@@ -167,8 +167,8 @@ def test_topk_host_validation(lib):
     assert call(A, 996, 4, 1000, 16, A) == kda.KDA_ERR_INVALID_ARG              # ld < n
     assert call(A, 1000, 70000, 1000, 16, A) == kda.KDA_ERR_INVALID_ARG         # too many rows
     assert call(A, 1000, 4, 1000, 16, None) == kda.KDA_ERR_INVALID_ARG          # no output
-    assert call(MIS, 1000, 4, 1000, 16, A) == kda.KDA_ERR_MISALIGNED            # scores not 16-byte aligned
-    assert call(A, 1002, 4, 1000, 16, A) == kda.KDA_ERR_MISALIGNED              # row stride not a multiple of 4
+    assert call(A + 2, 1000, 4, 1000, 16, A) == kda.KDA_ERR_MISALIGNED          # scores not 4-byte aligned
+    assert call(A, 1000, 4, 1000, 16, A + 1) == kda.KDA_ERR_MISALIGNED          # indices not 4-byte aligned
     assert call(A, 1000, 4, 1000, 16, A, ws_ptr=None) == kda.KDA_ERR_WORKSPACE
     assert call(A, 1000, 4, 1000, 16, A, ws_ptr=W + 16) == kda.KDA_ERR_WORKSPACE   # not 256-byte aligned
     assert call(A, 1000, 4, 1000, 2048, A, ws_bytes=ws - 1) == kda.KDA_ERR_WORKSPACE
