@@ -38,26 +38,55 @@ FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 TF32_OVER_BF16 = 1.1 / 2.25          # nominal dense tf32 : bf16 tensor-core ratio
 D = 128
-# Algorithmic HBM bytes per token-head of the prefill: q, k, v bf16 (3 x 256),
-# g fp32 (512), beta (4), o fp32 (512).  Per (sequence, head) add the final
-# state write (64 KiB) and, when given, the initial state read (64 KiB).
-PREFILL_BYTES_PER_TOKEN_HEAD = 3 * 2 * D + 4 * D + 4 + 4 * D
+# Algorithmic HBM bytes per token-head of the prefill, as the method's
+# workload fixes them: q, k, v bf16 (3 x 256), g fp32 (512), beta (4), and o
+# in v's dtype (256) = 1540 B.  Per (sequence, head) add the final state write
+# (64 KiB) and, when given, the initial state read (64 KiB).  The roofline
+# fraction is taken on these bytes.
+PREFILL_BYTES_PER_TOKEN_HEAD = 3 * 2 * D + 4 * D + 4 + 2 * D
+# This library writes o in fp32, 256 B more per token-head (bf16 rounding of
+# the exact output alone would exceed the 2e-2 x RMS bound); those are the
+# bytes the kernel actually moves, reported beside the fraction.
+PREFILL_BYTES_PER_TOKEN_HEAD_AS_WRITTEN = PREFILL_BYTES_PER_TOKEN_HEAD + 2 * D
 STATE_BYTES = 4 * D * D
 # Dense contraction flops per token-head of the 64-token chunk form:
 # 5 x (2 C^2 d) + 3 x (2 C d^2) + C^3 / 3 per chunk of C = 64 tokens.
 PREFILL_FLOPS_PER_TOKEN_HEAD = (5 * 2 * 64 * 64 * D + 3 * 2 * 64 * D * D + 64 ** 3 // 3) // 64
-# Decode: state read + write, plus q, k, v (bf16), g (fp32), beta, o (fp32).
-DECODE_BYTES_PER_SEQ_HEAD = 2 * STATE_BYTES + 3 * 2 * D + 4 * D + 4 + 4 * D
+# Decode: state read + write, plus q, k, v (bf16), g (fp32), beta and o in v's
+# dtype = 132,612 B per (sequence, head); o is written in fp32 (+256 B).
+DECODE_BYTES_PER_SEQ_HEAD = 2 * STATE_BYTES + 3 * 2 * D + 4 * D + 4 + 2 * D
+DECODE_BYTES_PER_SEQ_HEAD_AS_WRITTEN = DECODE_BYTES_PER_SEQ_HEAD + 2 * D
 # One prefill call of the 8K workload (one sequence, full workspace) launches
 # two kernels: the chunk index and the overlapped prep/state kernel.  The
 # prefill roofline is taken over the whole call (algorithmic bytes of the
 # call / its CUDA-event time); the ncu launch list gives each kernel's share.
 PREFILL_KERNELS = ("kda_chunk_index_kernel", "kda_chunk_overlap_kernel")
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one call, from
-# an ncu capture of the current kernel build on the same workload (the index
-# kernel's few KB left out); None whenever a kernel changed since it was captured.
-MEASURED_TRAFFIC_PREFILL = 343.761664e6 + 183.969280e6
-MEASURED_TRAFFIC_DECODE = 547.405312e6 + 486.942464e6
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
+# the dominant kernel, from the ncu capture named here, and a hash of the
+# kernel sources it was taken on: when the sources differ, the figure no
+# longer describes the kernel and the line reports traffic as null.
+MEASURED_TRAFFIC = {
+    "prefill": {"bytes": None, "capture": None, "sources_sha": None,
+                "files": ("kda_chunk2.cu", "kda_tile.cuh", "sm100.cuh", "kda_common.cuh", "kda_launch.h")},
+    "decode": {"bytes": None, "capture": None, "sources_sha": None,
+               "files": ("kda_decode.cu", "kda_common.cuh", "kda_launch.h")},
+}
+
+
+def sources_sha(files) -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "gated_delta_rule_152_b200", "csrc", f), "rb") as fh:
+            h.update(f.encode() + b"\0" + fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(kind):
+    t = MEASURED_TRAFFIC[kind]
+    if t["bytes"] is None or t["sources_sha"] != sources_sha(t["files"]):
+        return None, None
+    return t["bytes"], t["capture"]
 
 
 def load_peaks():
@@ -167,24 +196,77 @@ def oracle_prefill_sample(x: kin.PrefillInputs, tokens: int, threads: int = 0):
     return time.perf_counter() - t0, tokens
 
 
-def cpu_baseline(x: kin.PrefillInputs, target_s: float = 10.0):
+def _oracle_rate(fn, units, min_s):
+    """Run fn() (one bounded sample of `units` units) until min_s seconds have
+    passed; returns (units per second, seconds, repetitions)."""
+    reps, total = 0, 0.0
+    while reps == 0 or (total < min_s and reps < 64):
+        t0 = time.perf_counter()
+        fn()
+        total += time.perf_counter() - t0
+        reps += 1
+    return units * reps / total, total, reps
+
+
+def cpu_baseline(x: kin.PrefillInputs, min_s: float = 3.0):
+    """The fp64 oracle on the host cores: the headline figure is the 8K
+    workload on all cores; ``by_config`` adds one thread and all threads on
+    bounded samples of the tiny, 8K, varlen and decode workloads (each
+    sample's extent stated), about 10-20 s of CPU work in all."""
     import oracle
     cores = oracle.max_threads()
-    probe_tokens = 256
-    dt, _ = oracle_prefill_sample(x, probe_tokens)
-    tokens = int(min(x.total_T, max(probe_tokens, probe_tokens * target_s / max(dt, 1e-6))))
-    tokens = max(64, (tokens // 64) * 64)
-    dt, tokens = oracle_prefill_sample(x, tokens)
-    # when the whole workload takes well under the target, repeat whole
-    # passes so the rate is taken over about target_s of work
-    passes, total = 1, dt
-    while tokens == x.total_T and total < target_s and passes < 32:
-        dt, _ = oracle_prefill_sample(x, tokens)
-        passes, total = passes + 1, total + dt
-    what = (f"{passes} passes over all {tokens}" if passes > 1 else f"first {tokens} of {x.total_T}")
-    return {"value": tokens * passes / total, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": f"{what} tokens x 32 heads of prefill_bf16_T8192_H32, fp64, "
-                      f"{cores} OpenMP threads over (sequence, head) pairs, {total:.1f} s"}
+    rows = []
+    f64 = oracle.to_f64   # inputs converted once, outside the timed calls
+
+    def prefill_row(name, xs, tokens, threads, what):
+        sl = slice(0, tokens)
+        q, k, v, g, b = (f64(t)[sl] for t in (xs.q, xs.k, xs.v, xs.g, xs.beta))
+        cu = [0, tokens] if xs.cu_seqlens.numel() == 2 else xs.cu_seqlens.tolist()
+        s0 = None if xs.initial_state is None else f64(xs.initial_state)
+        fn = lambda: oracle.kda_forward(q, k, v, g, b, cu, s0, threads=threads)
+        rate, secs, reps = _oracle_rate(fn, tokens, min_s)
+        rows.append({"workload": name, "threads": threads, "value": rate, "unit": "tokens/s",
+                     "sample": f"{what}; {reps} pass(es), {secs:.1f} s"})
+        return rate, secs, reps
+
+    # 8K workload: all threads over whole passes (the headline), one thread on its first 256 tokens
+    rate8k, secs8k, reps8k = prefill_row(kin.PREFILL_8K.name, x, x.total_T, cores,
+                                         f"all {x.total_T} tokens x {x.heads} heads")
+    prefill_row(kin.PREFILL_8K.name, x, 256, 1, f"first 256 of {x.total_T} tokens x {x.heads} heads")
+    # tiny fp32 workload: whole (two heads, so at most two threads have work)
+    xt = kin.make_prefill(kin.TINY_FP32)
+    for th in (1, cores):
+        prefill_row(kin.TINY_FP32.name, xt, xt.total_T, th, f"all {xt.total_T} tokens x {xt.heads} heads")
+    # varlen workload: its first two sequence lengths (all heads, initial states) on all
+    # threads; the first 512 tokens of its first sequence on one thread
+    lens = kin.seq_lengths(kin.VARLEN_16)
+    xv = kin.make_prefill(kin.VARLEN_16, lengths=lens[:2])
+    prefill_row(kin.VARLEN_16.name, xv, xv.total_T, cores,
+                f"sequences of lengths {lens[0]} and {lens[1]} (the first two of 16) x {xv.heads} heads")
+    xv1 = kin.make_prefill(kin.VARLEN_16, lengths=[512])
+    prefill_row(kin.VARLEN_16.name, xv1, 512, 1, f"512 tokens of one sequence x {xv1.heads} heads")
+    # decode workload: 8 sequences x 4 of its layer slabs x 32 heads
+    spec = kin.DECODE_256x34
+    toks = [[f64(t) for t in (tk.q, tk.k, tk.v, tk.g, tk.beta)]
+            for tk in (kin.make_decode_tokens(spec, layer, n_seqs=8) for layer in range(4))]
+    states = [f64(kin.make_decode_state(spec, layer, n_seqs=8)) for layer in range(4)]
+    for th in (1, cores):
+        def dec():
+            for t, st in zip(toks, states):
+                oracle.kda_decode(*t, st, threads=th)
+        rate, secs, reps = _oracle_rate(dec, 8 * 4, min_s / 3)
+        rows.append({"workload": spec.name, "threads": th, "value": rate, "unit": "seq-steps/s/layer",
+                     "sample": f"8 sequences x 4 layer slabs x {spec.heads} heads; {reps} pass(es), {secs:.1f} s"})
+    # indexer selection: 4 of the top-k workload's 64 query rows (numpy's sort, one thread)
+    from oracle.topk import topk_indices
+    sc = torch.randn(4, TOPK_N, generator=torch.Generator().manual_seed(2048)).numpy()
+    rate, secs, reps = _oracle_rate(lambda: topk_indices(sc, TOPK_K), 4, min_s / 3)
+    rows.append({"workload": TOPK_WORKLOAD, "threads": 1, "value": rate, "unit": "query rows/s",
+                 "sample": f"4 of {TOPK_ROWS} rows x {TOPK_N} scores; {reps} pass(es), {secs:.1f} s"})
+    return {"value": rate8k, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{reps8k} passes over all {x.total_T} tokens x {x.heads} heads of {kin.PREFILL_8K.name}, "
+                      f"fp64, {cores} OpenMP threads over (sequence, head) pairs, {secs8k:.1f} s",
+            "by_config": rows}
 
 
 # ---------------------------------------------------------------- GPU arm
@@ -222,16 +304,61 @@ def time_prefill_config(spec, dev, stream, steps, warmup, hbm, world):
     ms = max_over_ranks(e0.elapsed_time(e1) / steps, world)
     state_io = N * H * STATE_BYTES * (2 if x.initial_state is not None else 1)
     nbytes = T * H * PREFILL_BYTES_PER_TOKEN_HEAD + state_io
+    nbytes_written = T * H * PREFILL_BYTES_PER_TOKEN_HEAD_AS_WRITTEN + state_io
     gbs = nbytes / (ms / 1e3) / 1e9
-    overlapped = N == 1 and H <= 96
+    overlapped = H <= 96   # the overlapped launch serves any number of sequences up to 96 heads
     del xd, o, sT, ws
     torch.cuda.empty_cache()
     return {"workload": spec.name, "value": world * T / (ms / 1e3), "unit": "tokens/s", "ms_per_call": ms,
             "sequences": N, "tokens": T, "heads": H, "steps": steps, "warmup": warmup,
             "path": "overlapped" if overlapped else "two-launch (index, prep, state kernels)",
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
-                         "bytes_per_launch": nbytes},
+                         "bytes_per_launch": nbytes, "bytes_per_launch_as_written": nbytes_written,
+                         "frac_as_written": nbytes_written / (ms / 1e3) / 1e9 / hbm},
             "clocks": clk}, steps * (2 if overlapped else 3)
+
+
+# The lightning indexer's selection step on one decode step's worth of
+# queries: 64 query rows, each over the scores of 1,048,576 past tokens, the
+# 2,048 highest kept (page "GLM-5.3-FLASH", section "How can a layer search
+# the whole history selectively?").  Scores ~ N(0, 1), seeded.
+TOPK_ROWS, TOPK_N, TOPK_K = 64, 1 << 20, 2048
+TOPK_WORKLOAD = f"indexer_topk{TOPK_K}_rows{TOPK_ROWS}_n{TOPK_N}"
+TOPK_KERNELS = 5   # init, hist0, pick0, split, finish (plus one memset of the error word)
+
+
+def time_topk(dev, stream, steps, warmup, hbm, world):
+    """Device time of one top-k selection call (scores resident in HBM,
+    256 MB > L2); the roofline bytes are the scores read once and the indices
+    written once."""
+    from gated_delta_rule_152_b200 import kda
+    g = torch.Generator().manual_seed(2048)
+    scores = torch.randn(TOPK_ROWS, TOPK_N, generator=g).to(dev)
+    idx = torch.empty(TOPK_ROWS, TOPK_K, dtype=torch.int32, device=dev)
+    ws = torch.empty(kda.kda_topk_workspace_size(TOPK_ROWS, TOPK_N, TOPK_K), dtype=torch.uint8, device=dev)
+    call = lambda: kda.kda_topk_indices(scores, TOPK_K, indices=idx, workspace=ws, stream=stream)
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, world)
+    nbytes = TOPK_ROWS * TOPK_N * 4 + TOPK_ROWS * TOPK_K * 4
+    gbs = nbytes / (ms / 1e3) / 1e9
+    del scores, idx, ws
+    torch.cuda.empty_cache()
+    return {"workload": TOPK_WORKLOAD, "value": world * TOPK_ROWS / (ms / 1e3), "unit": "query rows/s",
+            "ms_per_call": ms, "steps": steps, "warmup": warmup,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                         "bytes_per_launch": nbytes,
+                         "note": "scores read once + indices written once; the kernels read the scores "
+                                 "twice when the cut's bin holds <= 16,384 tokens of a row"}}, steps * TOPK_KERNELS
 
 
 def bench_gpu(args, world, rank, local):
@@ -271,6 +398,7 @@ def bench_gpu(args, world, rank, local):
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
     prefill_tok_s = world * T / (ms / 1e3)
     bytes_per_launch = T * H * PREFILL_BYTES_PER_TOKEN_HEAD + H * STATE_BYTES
+    bytes_written = T * H * PREFILL_BYTES_PER_TOKEN_HEAD_AS_WRITTEN + H * STATE_BYTES
     achieved_gbs = bytes_per_launch / (ms / 1e3) / 1e9
     flops_per_launch = T * H * PREFILL_FLOPS_PER_TOKEN_HEAD
     tf32_peak = bf16 * TF32_OVER_BF16
@@ -362,9 +490,13 @@ def bench_gpu(args, world, rank, local):
     dms = max_over_ranks(e0.elapsed_time(e1) / dsteps, world)
     dec_rate = world * N / (dms / 1e3)
     dec_bytes = N * spec.heads * DECODE_BYTES_PER_SEQ_HEAD
+    dec_bytes_written = N * spec.heads * DECODE_BYTES_PER_SEQ_HEAD_AS_WRITTEN
     dec_gbs = dec_bytes / (dms / 1e3) / 1e9
     del states
     torch.cuda.empty_cache()
+
+    # ---------------- the indexer's top-k selection -------------------------
+    topk, topk_launches = time_topk(dev, stream, max(args.steps, 20), max(args.warmup, 3), hbm, world)
 
     # ---------------- the other prefill configs (one GPU, not in --quick) ---
     # their host inputs take about 10 GB each, too much to hold once per rank
@@ -374,6 +506,8 @@ def bench_gpu(args, world, rank, local):
             extras[key], n_l = time_prefill_config(xspec, dev, stream, 30, max(args.warmup, 3), hbm, world)
             extra_launches += n_l
 
+    traffic_prefill, traffic_prefill_src = measured_traffic("prefill")
+    traffic_decode, traffic_decode_src = measured_traffic("decode")
     line = {
         "metric": METRIC,
         "value": prefill_tok_s,
@@ -391,21 +525,29 @@ def bench_gpu(args, world, rank, local):
                    "qkv_dtype": "bf16", "o_dtype": "fp32", "parallelism": f"replicas x{world}",
                    "l2": "inputs 471 MB > 126 MB L2, no flush"},
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved_gbs / hbm, "traffic": MEASURED_TRAFFIC_PREFILL,
+                     "frac": achieved_gbs / hbm, "traffic": traffic_prefill,
+                     "traffic_capture": traffic_prefill_src,
                      "peak_source": f"{peak_src} hbm_gbs",
                      "scope": "whole prefill call: " + " + ".join(PREFILL_KERNELS),
                      "bytes_per_launch": bytes_per_launch,
+                     "bytes_per_launch_as_written": bytes_written,
+                     "frac_as_written": bytes_written / (ms / 1e3) / 1e9 / hbm,
+                     "as_written_note": "o is written in fp32, 256 B per token-head more than the "
+                                        "1540 B the fraction is taken on",
                      "tensor": {"achieved_tflops": achieved_tflops, "peak_tflops_tf32": tf32_peak,
                                 "frac": achieved_tflops / tf32_peak,
                                 "flops_per_launch": flops_per_launch}},
         "decode": {"workload": spec.name, "value": dec_rate, "unit": "seq-steps/s/layer",
                    "ms_per_call": dms, "layers_rotated": L,
                    "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": hbm, "unit": "GB/s",
-                                "frac": dec_gbs / hbm, "traffic": MEASURED_TRAFFIC_DECODE,
-                                "bytes_per_launch": dec_bytes}},
+                                "frac": dec_gbs / hbm, "traffic": traffic_decode,
+                                "traffic_capture": traffic_decode_src,
+                                "bytes_per_launch": dec_bytes, "bytes_per_launch_as_written": dec_bytes_written,
+                                "frac_as_written": dec_bytes_written / (dms / 1e3) / 1e9 / hbm}},
         "e2e": {"value": world * T / (e2e_ms / 1e3), "unit": "tokens/s", "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": args.steps * 2 * len(PREFILL_KERNELS) + dsteps + extra_launches,
+        "topk": topk,
+        "gpu_launches": args.steps * 2 * len(PREFILL_KERNELS) + dsteps + topk_launches + extra_launches,
         "clocks": clk,
     }
     line.update(extras)

@@ -7,27 +7,31 @@
 //     o_t = scale * S_t^T q_t.
 // Evaluated 64 tokens at a time.  For one chunk with entry state S (rows =
 // key channels), Gamma_r = g_0 + ... + g_r per channel and Gamma_C its value
-// at the chunk's last token, the state side takes every exponent relative to
-// the chunk START, so each of its factors lies in (0, 1] whatever the decay:
-//     Qs = scale q^ e^Gamma_r,  Ks = k^ e^Gamma_r,  Kb = k^ e^(Gamma_C - Gamma_r),
-//     T' = (I + strict_lower(diag(beta) A))^-1 diag(beta),  P = lower_incl(...),
-//     W = T' Ks,  U = T' V,
-//     delta = U - W S,   O = Qs S + P delta,   S_next = Diag(e^Gamma_C) S + Kb^T delta,
-// with A_ri = sum_c k^_rc k^_ic e^(Gamma_rc - Gamma_ic) and P_ri the same with
-// scale q^_r: the intra-chunk Gram matrices, taken at the level the chunk's
-// decay allows (kda_tile.cuh: one tensor-core product through the chunk end,
-// 16-token block references, or pairwise exponentials).  Unrolling the
-// per-token rule inside the chunk gives (I + M) delta = diag(beta)(V - Ks S)
-// for the rank-one corrections delta_r, from which O and S_next follow.
-// Everything except the last line is independent of the state.  Pass 1
-// (kda_chunk_prep_kernel) therefore runs over all (chunk, head) pairs in
-// parallel and writes, per pair, ready-made tensor-core operand images of
-// [Qs ; W], Kb and P, and U and e^Gamma_C, to scratch.  Pass 2
-// (kda_chunk_state_kernel) walks the chunks of one (sequence, head) in order
-// and only carries the state:
-//     [Z^T | Y^T] = S^T [Qs ; W]^T             (M = 128 value columns, N = 128)
-//     delta^T = U^T - Y^T,   S^T <- S^T Diag(e^Gamma_C)
-//     S_next^T = S^T + delta^T Kb,   O^T = Z^T + delta^T P^T
+// at the chunk's last token, with T' = (I + strict_lower(diag(beta) A))^-1
+// diag(beta), A_ri = sum_c k^_rc k^_ic e^(Gamma_rc - Gamma_ic) and P_ri the
+// same with scale q^_r (the intra-chunk Gram matrices, taken at the level the
+// chunk's decay allows: kda_tile.cuh), the state side has two exact forms:
+//   chunk-end form (every channel decays by at most 2^100 over the chunk):
+//     Qt = scale q^ e^(Gamma_r - Gamma_C),  Kt = k^ e^(Gamma_r - Gamma_C),
+//     Kb = k^ e^(Gamma_C - Gamma_r),  St = Diag(e^Gamma_C) S,
+//     W = T' Kt,  U = T' V,  delta = U - W St,
+//     O = Qt St + P delta,   S_next = St + Kb^T delta;
+//   chunk-start form (any decay; every factor in (0, 1]):
+//     Qs = scale q^ e^Gamma_r,  Ks = k^ e^Gamma_r,  same Kb,
+//     W = T' Ks,  delta = U - W S,
+//     O = Qs S + P delta,   S_next = Diag(e^Gamma_C) S + Kb^T delta.
+// Unrolling the per-token rule inside the chunk gives (I + M) delta =
+// diag(beta)(V - k^ e^Gamma S) for the rank-one corrections delta_r, from
+// which O and S_next follow.  Everything except the last line is independent
+// of the state.  Pass 1 (kda_chunk_prep_kernel) therefore runs over all
+// (chunk, head) pairs in parallel and writes, per pair, ready-made
+// tensor-core operand images of [Q ; W], Kb and P, U, e^Gamma_C and a flag
+// naming the form, to scratch.  Pass 2 (kda_chunk_state_kernel) walks the
+// chunks of one (sequence, head) in order and only carries the state:
+//     (chunk-end form) S^T <- S^T Diag(e^Gamma_C)
+//     [Z^T | Y^T] = S^T [Q ; W]^T              (M = 128 value columns, N = 128)
+//     (chunk-start form) S^T <- S^T Diag(e^Gamma_C)
+//     delta^T = U^T - Y^T,   S_next^T = S^T + delta^T Kb,   O^T = Z^T + delta^T P^T
 // The state is kept transposed in tensor memory (lane = value column, column
 // = key channel), so it is the A operand of the first products and the
 // accumulator of the update, and the readout O^T lands with the value
@@ -37,7 +41,7 @@
 // contiguous) permute 16-byte chunks by the row index mod 8; MN-major tf32
 // tiles (the other axis contiguous), which the tensor core reads with a
 // different swizzle, permute 32-byte granules by the row index mod 4.  Pass 1
-// writes Ks, Kb and V in the token-row orientation it produces them in and
+// writes K (Kt or Ks), Kb and V in the token-row orientation it produces them in and
 // lets the products read them MN-major, so no tile is transposed.
 //
 // Precision: as the fused kernel -- tf32 operands (rounded to nearest),
@@ -57,7 +61,7 @@ constexpr int kThreads = 256;
 
 // ---- per (chunk, head) operand image in scratch (byte offsets), tiles
 // exactly as the state pass holds them in shared memory.
-constexpr uint32_t IMG_B1 = 0;        // [Qs ; W]: rows 0-63 Qs, 64-127 W (token) x 128 channels, K-major,
+constexpr uint32_t IMG_B1 = 0;        // [Q ; W]: rows 0-63 Q, 64-127 W (token) x 128 channels, K-major,
                                       //   4 K-blocks x 16 KB
 constexpr uint32_t IMG_DC = 65536;    // exp(Gamma_C): 128 fp32 (+ 512 B pad)
 constexpr uint32_t IMG_KB = 66560;    // Kb: 64 token rows x 128 channels, MN-major, 4 blocks of 32 channels x 8 KB
@@ -65,8 +69,10 @@ constexpr uint32_t IMG_P = 99328;     // P: 64 token rows x 64 tokens, K-major, 
 constexpr uint32_t IMG_U = 115712;    // U^T: 128 value rows x 64 tokens fp32, 16-byte chunks permuted as
                                       //   K-major tiles, 2 blocks of 32 tokens x 16 KB
 constexpr uint32_t IMG_BYTES = 148480;
-constexpr uint32_t KB_B1 = 16384, IMG_BLK = 8192;   // K-block of [Qs ; W]; 64 rows x 128 B
-constexpr uint32_t B1_COPY = IMG_DC + 512;   // [Qs ; W] and exp(Gamma_C) in one copy
+constexpr uint32_t KB_B1 = 16384, IMG_BLK = 8192;   // K-block of [Q ; W]; 64 rows x 128 B
+constexpr uint32_t IMG_FORM = IMG_DC + 512;   // 16 B: word 0 = 0 for the chunk-end form, 1 for the chunk-start form
+constexpr uint32_t B1_COPY = IMG_FORM + 16;   // [Q ; W], exp(Gamma_C) and the form flag in one copy
+static_assert(IMG_DC == 4 * 16384 && (B1_COPY - IMG_DC) % 16 == 0, "B1 copy: four 16 KB blocks, then the rest");
 constexpr uint32_t B2_COPY = IMG_BYTES - IMG_KB;   // Kb, P and U on one mbarrier phase
 static_assert(IMG_KB % 1024 == 0 && IMG_P == IMG_KB + 32768 && IMG_U == IMG_P + 16384 &&
               IMG_BYTES == IMG_U + 32768, "image layout");
@@ -144,8 +150,8 @@ constexpr uint32_t P_TP = 49152;     // 16 KB T': 64 rows (token r) x 64 (token 
 constexpr uint32_t P_KB = 65536;     // 32 KB second Gram operand: 64 rows x 128 channels, K-major, 4 K-blocks
                                      //   x 8 KB; also the TMA destination of the next item's raw q (16 KB)
                                      //   and k (16 KB)
-constexpr uint32_t P_KTM = 98304;    // 32 KB Ks MN-major: 64 token rows x 128 channels, 4 blocks x 8 KB
-                                     //   (Ks^T for W^T)
+constexpr uint32_t P_KTM = 98304;    // 32 KB Kt or Ks MN-major: 64 token rows x 128 channels, 4 blocks x
+                                     //   8 KB (the A operand of W^T)
 constexpr uint32_t P_WST = 131072;   // 32 KB W (K-major, 4 K-blocks x 8 KB) on its way to the image; before
                                      //   that the exact Gram's Z table (levels 1, 2)
 constexpr uint32_t P_V = 163840;     // 32 KB V MN-major: 64 token rows x 128 values, 4 blocks x 8 KB
@@ -257,7 +263,7 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
                                  : static_cast<size_t>(it.gc) * H + it.h;
         return img + slot * IMG_BYTES;
     };
-    // ring mode: the image of an item (Qs, Kb and exp(Gamma_C) written with
+    // ring mode: the image of an item (Q, Kb, exp(Gamma_C) and the form written with
     // plain stores before the item's block barriers, the rest by bulk stores)
     // is announced by the store thread once those bulk stores have completed:
     // a proxy fence, then a gpu-scope release, which also covers the plain
@@ -347,22 +353,28 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
         load_pending = false;
         load_parity ^= 1;
 
-        // ============== prep.  The state side takes the chunk-start form (every factor in
-        // (0, 1]): Qs = q^ 2^Gamma_r -> image rows 0-63 of [Qs ; W] (K-major), Ks = k^ 2^Gamma_r
-        // -> KTM (MN-major, for W), Kb = k^ 2^(Gamma_C - Gamma_r) -> image (MN-major), and
-        // 2^Gamma_C -> image.  The Gram operands in X (128 rows, Q-side then K-side) and KB
-        // (64 rows), both K-major, depend on the chunk's level (kda_tile.cuh):
-        //   0: [Qs ; Ks] and Kb 2^-Gamma_C = k^ 2^-Gamma_i, tf32 (one tensor-core product; the
-        //      second factor is at most 2^kSafeLog2 at this level);
-        //   1: [q^ X ; k^ X] (fp32) and k^ Y (tf32) (block references);
-        //   2: [q^ ; k^] and Gamma, fp32.
+        // ============== prep.  Two forms of the state-side operands, chosen by the chunk's
+        // Gram level (kda_tile.cuh), which the image records for the state role:
+        //   chunk-end form (level 0, every channel decays by at most 2^kSafeLog2 over the
+        //   chunk): Qt = q^ 2^(Gamma_r - Gamma_C), Kt = k^ 2^(Gamma_r - Gamma_C) (<= 2^100),
+        //   Kb = k^ 2^(Gamma_C - Gamma_r); the state role decays the state to the chunk end
+        //   first and MMA1 reads the decayed state;
+        //   chunk-start form (levels 1, 2, any decay): Qs = q^ 2^Gamma_r, Ks = k^ 2^Gamma_r,
+        //   same Kb (every factor <= 1); MMA1 reads the state at the chunk start and the
+        //   state role decays it afterwards.
+        // Either way: Q -> image rows 0-63 of [Q ; W] (K-major), K -> KTM (MN-major, for W),
+        // Kb -> image (MN-major), 2^Gamma_C and the form flag -> image.  The Gram operands in
+        // X (128 rows, Q-side then K-side) and KB (64 rows), both K-major:
+        //   level 0: [Qt ; Kt] and Kb, tf32 (one tensor-core product through the chunk end);
+        //   level 1: [q^ X ; k^ X] (fp32) and k^ Y (tf32) (block references);
+        //   level 2: [q^ ; k^] and Gamma, fp32.
         // A warp stores four whole 128-byte rows of the image at a time.
         int level = 0;
         float4 rho0, rho1, rho2, rho3;   // block ends of the thread's channels (for the exact Gram's table)
         {
-            // per-channel factors: 2^-Gamma_C (level 0); 2^rho_{a-1} and 2^(Gamma_C - rho_a) of the
-            // thread's block a = warp / 2 (level 1)
-            float4 gc, bprev, bcur, inv, es, ef;
+            // per-channel factors of level 1: 2^rho_{a-1} and 2^(Gamma_C - rho_a) of the thread's
+            // block a = warp / 2
+            float4 gc, bprev, bcur, es, ef;
             auto setup = [&](const ChunkChannels& cc, int lvl) {
                 level = lvl;
                 gc = cc.rho[3];
@@ -372,9 +384,7 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
                 rho1 = cc.rho[1];
                 rho2 = cc.rho[2];
                 rho3 = cc.rho[3];
-                if (lvl == 0) {
-                    inv = ex2x4(make_float4(-gc.x, -gc.y, -gc.z, -gc.w));
-                } else if (lvl == 1) {
+                if (lvl == 1) {
                     es = ex2x4(bprev);
                     ef = ex2x4(sub4(gc, bcur));
                 }
@@ -392,21 +402,22 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
                     q4 = tf32x4(qs.x, qs.y, qs.z, qs.w);
                     k4 = tf32x4(ks.x, ks.y, ks.z, ks.w);
                     b4 = tf32x4(kb.x, kb.y, kb.z, kb.w);
+                } else if (level == 0) {
+                    const float4 a = sub4(gr, gc);   // >= 0, at most kSafeLog2 at this level
+                    const float4 E = ex2x4(a), F = ex2x4(make_float4(-a.x, -a.y, -a.z, -a.w));
+                    const float4 qt = mul4(qn, E), kt = mul4(kn, E), kb = mul4(kn, F);
+                    q4 = xq = tf32x4(qt.x, qt.y, qt.z, qt.w);
+                    k4 = xk = tf32x4(kt.x, kt.y, kt.z, kt.w);
+                    b4 = y = tf32x4(kb.x, kb.y, kb.z, kb.w);
                 } else {
                     const float4 e0 = ex2x4(gr), f = ex2x4(sub4(gc, gr));
                     const float4 qs = mul4(qn, e0), ks = mul4(kn, e0), kb = mul4(kn, f);
                     q4 = tf32x4(qs.x, qs.y, qs.z, qs.w);
                     k4 = tf32x4(ks.x, ks.y, ks.z, ks.w);
                     b4 = tf32x4(kb.x, kb.y, kb.z, kb.w);
-                    if (level == 0) {
-                        xq = q4;
-                        xk = k4;
-                        y = tf32x4(kb.x * inv.x, kb.y * inv.y, kb.z * inv.z, kb.w * inv.w);
-                    } else {
-                        xq = qn;
-                        xk = kn;
-                        y = gr;
-                    }
+                    xq = qn;
+                    xk = kn;
+                    y = gr;
                 }
                 *reinterpret_cast<float4*>(smem + P_X + kbi * KB_B1 + sw128_off(r, ch)) = xq;
                 *reinterpret_cast<float4*>(smem + P_X + kbi * KB_B1 + sw128_off(64 + r, ch)) = xk;
@@ -416,6 +427,8 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
                 *reinterpret_cast<float4*>(im + IMG_KB + kbi * IMG_BLK + sw32g_off(r, ch)) = b4;
             });
             if (warp == 0) *reinterpret_cast<float4*>(im + IMG_DC + 16 * lane) = ex2x4(gc);
+            if (tid == 64)
+                *reinterpret_cast<float4*>(im + IMG_FORM) = make_float4(level != 0 ? 1.f : 0.f, 0.f, 0.f, 0.f);
             if (tid < kC) beta_s[tid] = breg;
         }
         // the previous item's U and W have left V and WST (V is rewritten below)
@@ -424,7 +437,7 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
         tc_fence_before();
         __syncthreads();
 
-        // ============== [P ; A]: level 0 by one tensor-core product [Qs ; Ks] x (Kb 2^-Gamma_C)^T
+        // ============== [P ; A]: level 0 by one tensor-core product [Qt ; Kt] x Kb^T
         // (P in lanes 0-63, A in lanes 64-127 of TP_AP), levels 1 and 2 on CUDA cores and
         // mma.sync (gram_exact), staged into the same tensor-memory columns
         if (level == 0 && tid == 0) {
@@ -545,7 +558,7 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
         tc_fence_before();
         __syncthreads();
 
-        // ============== W^T = Ks^T T'^T,  U^T = V^T T'^T  (Ks and V read MN-major)
+        // ============== W^T = K^T T'^T,  U^T = V^T T'^T  (K and V read MN-major)
         if (tid == 0) {
             tc_fence_after();
             const uint64_t dkt = sdesc_mn32(sb + P_KTM, P_MN_KB), dv = sdesc_mn32(sb + P_V, P_MN_KB);
@@ -645,8 +658,8 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
 
 // ============================================================ pass 2
 // The state pass keeps the image layout: shared-memory offsets equal image offsets.
-constexpr uint32_t S_B1 = 0;          // 64 KB [Qs ; W] of the current chunk
-constexpr uint32_t S_DC = 65536;      // exp(Gamma_C), copied with [Qs ; W]
+constexpr uint32_t S_B1 = 0;          // 64 KB [Q ; W] of the current chunk
+constexpr uint32_t S_DC = 65536;      // exp(Gamma_C) and the form flag, copied with [Q ; W]
 constexpr uint32_t S_KB = 66560;      // 32 KB Kb (MN-major), copied with U, then
 constexpr uint32_t S_P = 99328;       //   16 KB P (K-major)
 constexpr uint32_t S_U = 115712;      // 32 KB U^T
@@ -667,12 +680,13 @@ constexpr int kImgThread = 32;    // waits for the next chunk's image during MMA
 constexpr int kOutThread = 128;   // issues the O stores, the L2 prefetches and the ring hand-back
                                   // (first thread of the O warps; not the MMA thread)
 
-// Pass 2 for sequence n, head h.  Per chunk c (k = c % 2 selects one of two
-// Z/Y column sets in TMEM):
-//   MMA1:   [Z_k | Y_k] = S^T [Qs ; W]^T         (A = the state at the chunk start in
-//           TMEM, read as tf32; B = [Qs ; W])
+// Pass 2 for head h over the sequences n_begin .. n_end - 1.  Per chunk c
+// (k = c % 2 selects one of two Z/Y column sets in TMEM):
+//   decay:  S = Diag(e^Gamma_C) S in place in TMEM (fp32, all warps): here for the
+//           chunk-end form, after MMA1 for the chunk-start form
+//   MMA1:   [Z_k | Y_k] = S^T [Q ; W]^T          (A = the state in TMEM, read as
+//           tf32; B = [Q ; W])
 //           meanwhile O of chunk c-1 (set k^1) is read out and staged
-//   decay:  S = Diag(e^Gamma_C) S in place in TMEM (fp32)          (all warps)
 //   delta:  delta^T = U^T - Y_k^T                                  (all warps)
 //   MMA2a:  S^T += delta^T Kb   (Kb read MN-major; the only product the next chunk waits for)
 //   MMA2b:  Z_k^T += delta^T P^T  = O^T of chunk c, read out during chunk c+1
@@ -724,6 +738,25 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
         return !__syncthreads_or(!mbar_wait_bounded(bar, parity));
     };
     auto zcol = [](int c) { return TS_Z + 256u * static_cast<uint32_t>(c & 1); };   // Z of chunk c; Y follows
+    // S <- Diag(d) S in place in TMEM (fp32): key channels 64 * half .. of value column e;
+    // the caller waits for the stores (tmem_wait_st) before the next product reads S
+    auto decay_state = [&](const float* d) {
+        float st[2][32];
+#pragma unroll
+        for (int part = 0; part < 2; ++part) tmem_ld32(tm_lane(tmem, quarter, TS_S + 64 * half + 32 * part), st[part]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+            const int c0 = 64 * half + 32 * part;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float4 d4 = *reinterpret_cast<const float4*>(d + c0 + 4 * j);
+                st[part][4 * j] *= d4.x; st[part][4 * j + 1] *= d4.y;
+                st[part][4 * j + 2] *= d4.z; st[part][4 * j + 3] *= d4.w;
+            }
+            tmem_st32(tm_lane(tmem, quarter, TS_S + c0), st[part]);
+        }
+    };
 
     for (int n = n_begin; ok && n < n_end; ++n) {
     __syncthreads();   // the previous sequence's final state has left tensor memory
@@ -789,7 +822,7 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
         const uint8_t* src = image(c);
 #pragma unroll
         for (int p = 0; p < 4; ++p) bulk_load(smem + S_B1 + p * 16384, src + p * 16384, 16384, bar_b1);
-        bulk_load(smem + S_DC, src + IMG_DC, 512, bar_b1);
+        bulk_load(smem + S_DC, src + IMG_DC, B1_COPY - IMG_DC, bar_b1);
     };
     // Kb, P and U in two steps on one mbarrier phase (the first step
     // registers all the bytes): Kb and U as soon as MMA2a of the previous
@@ -835,18 +868,23 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
         }
         if (!RING && tid == kOutThread && c + 2 < nch) prefetch_l2(image(c + 2), IMG_BYTES);
         if (tid == kOutThread) bulk_wait_read();   // the O staging tile is rewritten below
-        // [Qs ; W] and 2^Gamma_C of chunk c have landed; 2^Gamma_C is kept aside for
-        // the decay after MMA1 (the next chunk's copy lands on top of it before then)
+        // [Q ; W], 2^Gamma_C and the form flag of chunk c have landed.  Chunk-end form:
+        // the state is decayed to the chunk end now and MMA1 reads it decayed.  Chunk-start
+        // form: MMA1 reads the state as it is and the decay follows MMA1, so 2^Gamma_C is
+        // kept aside (the next chunk's copy lands on top of it before then).
         const bool b1_ok = mbar_wait_bounded(bar_b1, (base + c) & 1);
-        if (b1_ok && tid < kD / 4)
+        const bool start_form = b1_ok && dc_s[kD] != 0.f;   // the same word for every thread
+        if (b1_ok && !start_form) decay_state(dc_s);
+        if (b1_ok && start_form && tid < kD / 4)
             reinterpret_cast<float4*>(dc_keep)[tid] = reinterpret_cast<const float4*>(dc_s)[tid];
+        tmem_wait_st();
         tc_fence_before();
         if (!(ok = !__syncthreads_or(!b1_ok))) break;
         b1_pending = false;
 
-        // ---- MMA1: [Z_k^T | Y_k^T] = S^T [Qs ; W]^T (the state at the chunk start,
-        // read by the tensor core as tf32: the low mantissa bits are dropped; measured
-        // on the CPU against the fp64 oracle: no change in the error of o or S)
+        // ---- MMA1: [Z_k^T | Y_k^T] = S^T [Q ; W]^T (the state, decayed or not by the
+        // form, read by the tensor core as tf32: the low mantissa bits are dropped;
+        // measured on the CPU against the fp64 oracle: no change in the error of o or S)
         if (tid == 0) {
             tc_fence_after();
             const uint64_t db = tdesc(sb, S_B1);
@@ -893,27 +931,10 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
         b1_pending = c + 1 < nch;
         b1_chunk = static_cast<int>(base) + c + 1;
 
-        // ---- decay: S <- Diag(2^Gamma_C) S in place (fp32; MMA1, its last reader, is
-        // done), key channels 64 * half .. of value column e;
+        // ---- chunk-start form: the decay, now that MMA1 (its last reader) is done;
         // delta^T = U^T - Y_k^T (tf32 operand, row = value column, K = token);
         // U^T came with Kb
-        {
-            float st[2][32];
-#pragma unroll
-            for (int part = 0; part < 2; ++part) tmem_ld32(tm_lane(tmem, quarter, TS_S + 64 * half + 32 * part), st[part]);
-            tmem_wait_ld();
-#pragma unroll
-            for (int part = 0; part < 2; ++part) {
-                const int c0 = 64 * half + 32 * part;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const float4 d4 = *reinterpret_cast<const float4*>(dc_keep + c0 + 4 * j);
-                    st[part][4 * j] *= d4.x; st[part][4 * j + 1] *= d4.y;
-                    st[part][4 * j + 2] *= d4.z; st[part][4 * j + 3] *= d4.w;
-                }
-                tmem_st32(tm_lane(tmem, quarter, TS_S + c0), st[part]);
-            }
-        }
+        if (start_form) decay_state(dc_keep);
         const bool b2_ok = mbar_wait_bounded(bar_b2, (base + c) & 1);
         if (b2_ok) {
             float y[32];
@@ -932,7 +953,7 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
                     tf32x4(u[4 * j] - y[4 * j], u[4 * j + 1] - y[4 * j + 1], u[4 * j + 2] - y[4 * j + 2],
                            u[4 * j + 3] - y[4 * j + 3]);
         }
-        tmem_wait_st();   // the decayed state is in place before MMA2a accumulates onto it
+        tmem_wait_st();   // (chunk-start form) the decayed state is in place before MMA2a accumulates onto it
         fence_proxy_async_smem();
         tc_fence_before();
         if (!(ok = !__syncthreads_or(!b2_ok || !img_ok))) {

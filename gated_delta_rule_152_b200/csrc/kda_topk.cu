@@ -1,7 +1,8 @@
 // kda_topk.cu -- the selection step of the lightning indexer: per query row,
-// the k highest of n per-token relevance scores (page "GLM-5.3-FLASH",
-// dimsnsums.com, section "How can a layer search the whole history
-// selectively?": every past token is scored and the 2,048 highest are kept).
+// the k best of n per-token scores (page "GLM-5.3-FLASH", dimsnsums.com,
+// section "How can a layer search the whole history selectively?": the
+// indexer of a sparse layer scores all earlier tokens and passes only the
+// best 2,048 on to full attention).
 //
 // Order of tokens: a higher score ranks higher; equal scores (-0 == +0) rank
 // the lower index higher, so the kept set is unique.  The output lists the

@@ -269,8 +269,8 @@ KDA_API int kda_selftest_bounded_waits(void *workspace, size_t workspace_bytes, 
 /*
  * kda_topk_indices -- the selection step of the lightning indexer (page
  * "GLM-5.3-FLASH", dimsnsums.com, section "How can a layer search the whole
- * history selectively?": every past token gets a relevance score and the
- * 2,048 highest are kept for full attention).  The page defines neither the
+ * history selectively?": the indexer of a sparse layer scores all earlier
+ * tokens and passes only the best 2,048 on to full attention).  The page defines neither the
  * score nor ties, so the scores are the caller's and the ranking is stated
  * here: a higher score ranks higher; equal scores (-0 == +0) rank the lower
  * index higher, which makes the kept set unique.

@@ -5,9 +5,9 @@ the library's product path never does, and it shares no code with the CUDA
 implementation.
 
 What it computes: page "GLM-5.3-FLASH" (dimsnsums.com), section "How can a
-layer search the whole history selectively?": each sparse layer's lightning
-indexer gives every past token a relevance score and keeps the 2,048 highest
-for full attention.  The page defines neither the score nor what happens on
+layer search the whole history selectively?": the lightning indexer of a
+sparse layer scores all earlier tokens and passes only the best 2,048 on to
+full attention.  The page defines neither the score nor what happens on
 equal scores, so the selection is stated here on caller-given scores, with
 these readings:
 

@@ -90,9 +90,10 @@ def kda_forward_chunked(q, k, v, g, beta, cu_seqlens, initial_state=None, scale=
 
 
 # ---------------------------------------------------------------------------
-# The form the two-pass tensor-core prefill evaluates.  The state side takes
-# every exponent relative to the chunk START, so all its factors lie in
-# (0, 1] whatever the decay:
+# The forms the two-pass tensor-core prefill evaluates.  A chunk whose Gram
+# level is 0 (below) keeps the chunk-end form above; any other chunk takes
+# every state-side exponent relative to the chunk START, so all its factors
+# lie in (0, 1] whatever the decay:
 #     Qs = q exp(Gamma_r),  Ks = k exp(Gamma_r),  Kb = k exp(Gamma_C - Gamma_r)
 #     W = T' Ks,  U = T' V,  delta = U - W S,  O = Qs S + P delta,
 #     S_next = diag(exp(Gamma_C)) S + Kb^T delta,
@@ -155,9 +156,10 @@ def gram(qn, kn, G, level):
 
 def kda_forward_chunked_start(q, k, v, g, beta, cu_seqlens, initial_state=None, scale=1.0,
                               l2norm=True, eps=1e-6, force_level=None, levels=None):
-    """The chunk-start form above, exact (fp64).  ``force_level`` evaluates
-    every chunk's Gram matrices at that level (where it is finite);
-    ``levels``, if a list, receives the level each chunk chose."""
+    """The forms above, exact (fp64): the chunk-end state form for level-0
+    chunks, the chunk-start form otherwise.  ``force_level`` evaluates every
+    chunk at that level (where it is finite); ``levels``, if a list, receives
+    the level each chunk chose."""
     q, k, v, g, beta = (np.asarray(x, dtype=np.float64) for x in (q, k, v, g, beta))
     cu = [int(x) for x in cu_seqlens]
     T, H, d = q.shape
@@ -189,12 +191,21 @@ def kda_forward_chunked_start(q, k, v, g, beta, cu_seqlens, initial_state=None, 
                 Mm = np.tril(b[:, None] * A, -1)
                 Tp = np.linalg.inv(np.eye(C) + Mm) * b[None, :]
                 P = np.tril(P)
-                Qs, Ks, Kb = qc * np.exp(G), kc * np.exp(G), kc * np.exp(GC - G)
                 V = np.zeros((C, d))
                 V[:L] = v[sl, h]
-                W, U = Tp @ Ks, Tp @ V
-                delta = U - W @ S
-                o[sl, h] = (Qs @ S + P @ delta)[:L]
-                S = np.exp(GC)[:, None] * S + Kb.T @ delta
+                Kb = kc * np.exp(GC - G)
+                if lvl == 0:   # chunk-end form: the state decayed first, factors up to e^LIMIT
+                    Qt, Kt = qc * np.exp(G - GC), kc * np.exp(G - GC)
+                    St = np.exp(GC)[:, None] * S
+                    W, U = Tp @ Kt, Tp @ V
+                    delta = U - W @ St
+                    o[sl, h] = (Qt @ St + P @ delta)[:L]
+                    S = St + Kb.T @ delta
+                else:          # chunk-start form: every factor at most 1
+                    Qs, Ks = qc * np.exp(G), kc * np.exp(G)
+                    W, U = Tp @ Ks, Tp @ V
+                    delta = U - W @ S
+                    o[sl, h] = (Qs @ S + P @ delta)[:L]
+                    S = np.exp(GC)[:, None] * S + Kb.T @ delta
             sT[n, h] = S
     return o, sT
