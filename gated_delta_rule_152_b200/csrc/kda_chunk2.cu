@@ -370,39 +370,20 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
         //   level 2: [q^ ; k^] and Gamma, fp32.
         // A warp stores four whole 128-byte rows of the image at a time.
         int level = 0;
-        float4 rho0, rho1, rho2, rho3;   // block ends of the thread's channels (for the exact Gram's table)
         {
-            // per-channel factors of level 1: 2^rho_{a-1} and 2^(Gamma_C - rho_a) of the thread's
-            // block a = warp / 2
-            float4 gc, bprev, bcur, es, ef;
+            // Gamma_C, and the block ends rho_{a-1}, rho_a of the thread's block a = warp / 2
+            // (level 1); the full block-end table is rebuilt from xch after the rows
+            float4 gc, bprev, bcur;
             auto setup = [&](const ChunkChannels& cc, int lvl) {
                 level = lvl;
                 gc = cc.rho[3];
                 bprev = cc.bstart;
                 bcur = cc.bend;
-                rho0 = cc.rho[0];
-                rho1 = cc.rho[1];
-                rho2 = cc.rho[2];
-                rho3 = cc.rho[3];
-                if (lvl == 1) {
-                    es = ex2x4(bprev);
-                    ef = ex2x4(sub4(gc, bcur));
-                }
             };
             prep_chunk_rows(smem + P_KB, smem + P_KB + kC * kD * 2, greg, xch, L, scale, l2norm != 0, setup,
                             [&](int r, int kbi, int ch, float4 qn, float4 kn, float4 gr) {
                 float4 q4, k4, b4, xq, xk, y;
-                if (level == 1) {
-                    const float4 X = ex2x4(sub4(gr, bprev)), Y = ex2x4(sub4(bcur, gr));
-                    xq = mul4(qn, X);
-                    xk = mul4(kn, X);
-                    const float4 ky = mul4(kn, Y);
-                    y = tf32x4(ky.x, ky.y, ky.z, ky.w);
-                    const float4 qs = mul4(xq, es), ks = mul4(xk, es), kb = mul4(ky, ef);
-                    q4 = tf32x4(qs.x, qs.y, qs.z, qs.w);
-                    k4 = tf32x4(ks.x, ks.y, ks.z, ks.w);
-                    b4 = tf32x4(kb.x, kb.y, kb.z, kb.w);
-                } else if (level == 0) {
+                if (level == 0) {
                     const float4 a = sub4(gr, gc);   // >= 0, at most kSafeLog2 at this level
                     const float4 E = ex2x4(a), F = ex2x4(make_float4(-a.x, -a.y, -a.z, -a.w));
                     const float4 qt = mul4(qn, E), kt = mul4(kn, E), kb = mul4(kn, F);
@@ -410,14 +391,23 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
                     k4 = xk = tf32x4(kt.x, kt.y, kt.z, kt.w);
                     b4 = y = tf32x4(kb.x, kb.y, kb.z, kb.w);
                 } else {
+                    // chunk-start form (every factor <= 1)
                     const float4 e0 = ex2x4(gr), f = ex2x4(sub4(gc, gr));
                     const float4 qs = mul4(qn, e0), ks = mul4(kn, e0), kb = mul4(kn, f);
                     q4 = tf32x4(qs.x, qs.y, qs.z, qs.w);
                     k4 = tf32x4(ks.x, ks.y, ks.z, ks.w);
                     b4 = tf32x4(kb.x, kb.y, kb.z, kb.w);
-                    xq = qn;
-                    xk = kn;
-                    y = gr;
+                    if (level == 1) {   // block references: X = 2^(Gamma_r - rho_{a-1}), Y = 2^(rho_a - Gamma_r)
+                        const float4 X = ex2x4(sub4(gr, bprev)), Y = ex2x4(sub4(bcur, gr));
+                        xq = mul4(qn, X);
+                        xk = mul4(kn, X);
+                        const float4 ky = mul4(kn, Y);
+                        y = tf32x4(ky.x, ky.y, ky.z, ky.w);
+                    } else {
+                        xq = qn;
+                        xk = kn;
+                        y = gr;
+                    }
                 }
                 *reinterpret_cast<float4*>(smem + P_X + kbi * KB_B1 + sw128_off(r, ch)) = xq;
                 *reinterpret_cast<float4*>(smem + P_X + kbi * KB_B1 + sw128_off(64 + r, ch)) = xk;
@@ -449,11 +439,19 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
             mma_commit(bar_mma);
         }
         if (level == 0) mma_pending = true;
-        if (level != 0 && warp == 0) {   // block ends of the thread's channels -> [4][128] table in xch
-            *reinterpret_cast<float4*>(xch + 0 * kD + 4 * lane) = rho0;
-            *reinterpret_cast<float4*>(xch + 1 * kD + 4 * lane) = rho1;
-            *reinterpret_cast<float4*>(xch + 2 * kD + 4 * lane) = rho2;
-            *reinterpret_cast<float4*>(xch + 3 * kD + 4 * lane) = rho3;
+        if (level != 0 && warp == 0) {
+            // block ends -> [4][128] table in xch, in place: xch row w holds the Gamma sum of
+            // warp w's 8 rows, and rho_a = the sum over warps 0 .. 2a + 1, added in the order
+            // (and so to the same floats) as in the rows' prefix
+            float4 t[8];
+#pragma unroll
+            for (int v = 0; v < 8; ++v) t[v] = *reinterpret_cast<const float4*>(xch + v * kD + 4 * lane);
+            float4 run = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+                run = make_float4(run.x + t[v].x, run.y + t[v].y, run.z + t[v].z, run.w + t[v].w);
+                if (v & 1) *reinterpret_cast<float4*>(xch + (v >> 1) * kD + 4 * lane) = run;
+            }
         }
         // ============== meanwhile: V (MN-major; bf16 is exact in tf32) from the raw
         // tile, rows past L zero; a 32-byte granule holds the 8 values of a raw chunk
