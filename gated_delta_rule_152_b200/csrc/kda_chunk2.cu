@@ -282,6 +282,8 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
     };
     // store thread: done[] of the item's head, read one item ahead
     int32_t done_seen = 0;
+    // q, k, v and g are read once: evict them first, ahead of the ring's images
+    const uint64_t stream_policy = l2_evict_first();
     float greg[8][4];
     float breg;
     auto prefetch = [&](const Item& it) {
@@ -294,7 +296,8 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
                     const float gs = __ldg(g + (size_t)(it.t0 + r) * H + it.h);
                     x = make_float4(gs, gs, gs, gs);
                 } else {
-                    x = __ldg(reinterpret_cast<const float4*>(g + ((size_t)(it.t0 + r) * H + it.h) * kD + 4 * lane));
+                    x = ldg_hint(reinterpret_cast<const float4*>(g + ((size_t)(it.t0 + r) * H + it.h) * kD + 4 * lane),
+                                 stream_policy);
                 }
             }
             greg[m][0] = x.x; greg[m][1] = x.y; greg[m][2] = x.z; greg[m][3] = x.w;
@@ -305,9 +308,9 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
     auto issue_load = [&](const Item& it) {
         mbar_arrive_expect_tx(bar_load, 3u * kC * kD * 2u);
         const int32_t t0 = static_cast<int32_t>(it.t0);
-        tma_load_3d(smem + P_KB, tm_q, bar_load, 0, it.h, t0);
-        tma_load_3d(smem + P_KB + kC * kD * 2, tm_k, bar_load, 0, it.h, t0);
-        tma_load_3d(smem + P_RV, tm_v, bar_load, 0, it.h, t0);
+        tma_load_3d_hint(smem + P_KB, tm_q, bar_load, 0, it.h, t0, stream_policy);
+        tma_load_3d_hint(smem + P_KB + kC * kD * 2, tm_k, bar_load, 0, it.h, t0, stream_policy);
+        tma_load_3d_hint(smem + P_RV, tm_v, bar_load, 0, it.h, t0, stream_policy);
     };
 
     bool ok = true;
@@ -922,7 +925,7 @@ __device__ __forceinline__ void state_role(const CUtensorMap* tm_o, const uint8_
         if (c > 0) o_pending = false;
         tc_fence_after();
         if (c > 0 && tid == kOutThread) {   // O of chunk c-1 leaves by one TMA store
-            tma_store_3d(tm_o, smem + S_OS, 0, h, static_cast<int32_t>(t_prev));
+            tma_store_3d_hint(tm_o, smem + S_OS, 0, h, static_cast<int32_t>(t_prev), l2_evict_first());
             bulk_commit();
         }
         if (tid == kImgThread && c + 1 < nch && img_ok) load_b1(c + 1);
