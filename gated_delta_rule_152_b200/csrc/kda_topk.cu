@@ -13,8 +13,8 @@
 // found by radix selection on the keys, most significant digit first:
 //   1. hist0 (many CTAs per row): histogram of the top 11 key bits;
 //   2. pick0 (one CTA per row): the top-digit bin b holding the k-th best key;
-//   3. split (many CTAs per row): keys above bin b are kept outright, keys in
-//      bin b become candidates (when there are at most kTopkCap of them);
+//   3. split (many CTAs per row): the keys of bin b and above become candidates
+//      (when bin b holds at most kTopkCap keys);
 //   4. finish (one CTA per row): the remaining digits (and, for equal keys at
 //      the cut, the index digits) among the candidates -- or over the whole
 //      row when bin b holds more than kTopkCap keys -- then a bitonic sort of
@@ -35,6 +35,8 @@ constexpr int kBins = 2048;               // 11-bit digits
 constexpr int kSeg = 16384;               // scores per CTA in the row-parallel passes
 constexpr int kTopkMaxK = 4096;
 constexpr int kTopkCap = 16384;           // candidates kept per row for the finish step
+constexpr int kCandCap = kTopkCap + kTopkMaxK;   // candidates: bin b and the keys above it
+constexpr int kSplitStage = 1024;         // pairs one split CTA stages in shared memory
 
 struct RowState {
     int32_t n;        // tokens in the row
@@ -42,7 +44,7 @@ struct RowState {
     uint32_t b;       // top-digit bin of the cut
     int32_t cnt_b;    // keys in bin b
     int32_t nsel;     // kept pairs written to the row's buffer
-    int32_t ncand;    // candidates written
+    int32_t ncand;    // candidates written (bin b and the keys above it)
     int32_t mode;     // 0: n <= k, keep all; 1: candidates; 2: bin b too full, the finish step scans the row
     int32_t pad[9];
 };
@@ -50,7 +52,7 @@ static_assert(sizeof(RowState) == 64, "row state");
 
 // Workspace (after the 256-byte header with the error word): per row its
 // state, then [rows][kBins] histogram counts, [rows][k] kept pairs and
-// [rows][kTopkCap] candidates.
+// [rows][kCandCap] candidates.
 struct Layout {
     RowState* st;
     uint32_t* hist;
@@ -74,14 +76,15 @@ inline size_t workspace_bytes(int rows, int k) {
     return 256 + align256(sizeof(RowState) * static_cast<size_t>(rows)) +
            align256(sizeof(uint32_t) * kBins * static_cast<size_t>(rows)) +
            align256(sizeof(unsigned long long) * static_cast<size_t>(k) * rows) +
-           sizeof(unsigned long long) * static_cast<size_t>(kTopkCap) * rows;
+           sizeof(unsigned long long) * static_cast<size_t>(kCandCap) * rows;
 }
 
-// Order-preserving key of a score; -0 and +0 get the same key.
+// Order-preserving key of a score; -0 and +0 get the same key (the IEEE sum
+// x + 0 turns -0 into +0 and leaves every other non-NaN score as it is).
+// Positives get the sign bit set, negatives all bits inverted.
 __device__ __forceinline__ uint32_t score_key(float x) {
-    uint32_t u = __float_as_uint(x);
-    if ((u << 1) == 0u) u = 0u;
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    const uint32_t u = __float_as_uint(x + 0.0f);
+    return u ^ (static_cast<uint32_t>(static_cast<int32_t>(u) >> 31) | 0x80000000u);
 }
 __device__ __forceinline__ float key_score(uint32_t key) {
     return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
@@ -140,6 +143,73 @@ __device__ __forceinline__ void append(bool take, unsigned long long v, int32_t*
     }
 }
 
+// The same append staged in shared memory: the pairs of one CTA collect in `sh`
+// (cap_sh of them; any further ones go straight to the row's buffer), and
+// flush_staged moves them out with one reservation on the row's counter.
+__device__ __forceinline__ void append_staged(bool take, unsigned long long v, int* sh_count,
+                                              unsigned long long* sh, int cap_sh, int32_t* counter,
+                                              unsigned long long* buf, int cap) {
+    const unsigned m = __ballot_sync(0xffffffffu, take);
+    if (!m) return;
+    const int lane = threadIdx.x & 31, leader = __ffs(m) - 1;
+    int base = 0;
+    if (lane == leader) base = atomicAdd(sh_count, __popc(m));
+    base = __shfl_sync(0xffffffffu, base, leader);
+    if (take) {
+        const int pos = base + __popc(m & ((1u << lane) - 1u));
+        if (pos < cap_sh) {
+            sh[pos] = v;
+        } else {
+            const int g = atomicAdd(counter, 1);
+            if (g < cap) buf[g] = v;
+        }
+    }
+}
+// append_staged for four pairs per lane at once (one shared-memory reservation
+// for the warp); all 32 lanes call it.
+__device__ __forceinline__ void append4_staged(const bool (&take)[4], const unsigned long long (&v)[4], int* sh_count,
+                                               unsigned long long* sh, int cap_sh, int32_t* counter,
+                                               unsigned long long* buf, int cap) {
+    unsigned m[4];
+    int tot = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        m[j] = __ballot_sync(0xffffffffu, take[j]);
+        tot += __popc(m[j]);
+    }
+    if (tot == 0) return;
+    const int lane = threadIdx.x & 31;
+    int base = 0;
+    if (lane == 0) base = atomicAdd(sh_count, tot);
+    base = __shfl_sync(0xffffffffu, base, 0);
+    const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        if (take[j]) {
+            const int pos = base + __popc(m[j] & lt);
+            if (pos < cap_sh) {
+                sh[pos] = v[j];
+            } else {
+                const int g = atomicAdd(counter, 1);
+                if (g < cap) buf[g] = v[j];
+            }
+        }
+        base += __popc(m[j]);
+    }
+}
+// All threads; a block barrier first.
+__device__ __forceinline__ void flush_staged(const int* sh_count, const unsigned long long* sh, int cap_sh,
+                                             int32_t* counter, unsigned long long* buf, int cap, int* sh_base) {
+    __syncthreads();
+    const int n = min(*sh_count, cap_sh);
+    if (threadIdx.x == 0 && n > 0) *sh_base = atomicAdd(counter, n);
+    __syncthreads();
+    if (n == 0) return;
+    const int g0 = *sh_base;
+    for (int i = threadIdx.x; i < n; i += blockDim.x)
+        if (g0 + i < cap) buf[g0 + i] = sh[i];
+}
+
 __global__ void __launch_bounds__(kThreads) kda_topk_init_kernel(const int32_t* lengths, int64_t n, int k, Layout L) {
     const int r = blockIdx.x;
     if (threadIdx.x == 0) {
@@ -179,9 +249,11 @@ __global__ void __launch_bounds__(kThreads) kda_topk_hist0_kernel(const float* _
 // that holds the `need`-th element counted from the top (from_top) or from
 // the bottom.  Returns the bin; *before receives the count of the bins
 // passed over first.  All threads call it; two block barriers inside.
+template <int NT>
 __device__ __forceinline__ int find_bin(const uint32_t* h, int need, bool from_top, int* before, int* scratch) {
+    static_assert(NT % 32 == 0 && NT <= 1024 && kBins % NT == 0, "find_bin: whole warps, at most 32");
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    constexpr int per = kBins / kThreads;   // 8 bins per thread, thread 0 first in visiting order
+    constexpr int per = kBins / NT;   // bins per thread, thread 0 first in visiting order
     if (t == 0) scratch[32] = scratch[33] = 0;
     uint32_t c[per], sum = 0;
 #pragma unroll
@@ -227,7 +299,7 @@ __global__ void __launch_bounds__(kThreads) kda_topk_pick0_kernel(int k, Layout 
     for (int i = threadIdx.x; i < kBins; i += kThreads) h[i] = L.hist[static_cast<size_t>(r) * kBins + i];
     __syncthreads();
     int above = 0;
-    const int b = find_bin(h, k, true, &above, scratch);
+    const int b = find_bin<kThreads>(h, k, true, &above, scratch);
     if (threadIdx.x == 0) {
         s.b = static_cast<uint32_t>(b);
         s.need = k - above;
@@ -237,8 +309,8 @@ __global__ void __launch_bounds__(kThreads) kda_topk_pick0_kernel(int k, Layout 
     }
 }
 
-// Keys above bin b are kept, keys in bin b are candidates (mode 1); every key
-// is kept when the row has at most k tokens (mode 0).
+// Keys in bin b or above are candidates (mode 1); every key is kept when the
+// row has at most k tokens (mode 0).
 __global__ void __launch_bounds__(kThreads) kda_topk_split_kernel(const float* __restrict__ scores, int64_t ld,
                                                                   int k, Layout L) {
     const int r = blockIdx.y;
@@ -246,17 +318,24 @@ __global__ void __launch_bounds__(kThreads) kda_topk_split_kernel(const float* _
     const RowState s = *sp;
     const int lo = blockIdx.x * kSeg, hi = min(s.n, lo + kSeg);
     if (s.mode == 2) return;
-    unsigned long long* kept = L.kept + static_cast<size_t>(r) * k;
-    unsigned long long* cand = L.cand + static_cast<size_t>(r) * kTopkCap;
+    // mode 0: every pair to the kept buffer; mode 1: the candidates
+    unsigned long long* buf =
+        s.mode == 0 ? L.kept + static_cast<size_t>(r) * k : L.cand + static_cast<size_t>(r) * kCandCap;
+    int32_t* counter = s.mode == 0 ? &sp->nsel : &sp->ncand;
+    const int cap = s.mode == 0 ? k : kCandCap;
     // whole warps iterate together so that the warp-wide append sees every lane;
     // four scores per thread and step between 16-byte boundaries
     const float* row = scores + r * ld;
+    // this CTA's pairs, staged in shared memory
+    __shared__ unsigned long long sh_buf[kSplitStage];
+    __shared__ int sh_n, sh_base;
     auto visit = [&](int i, uint32_t key, bool live) {
-        const uint32_t top = key >> 21;
-        append(live && (s.mode == 0 || top > s.b), pair_of(key, i), &sp->nsel, kept, k);
-        if (s.mode == 1) append(live && top == s.b, pair_of(key, i), &sp->ncand, cand, kTopkCap);
+        append_staged(live && (s.mode == 0 || (key >> 21) >= s.b), pair_of(key, i), &sh_n, sh_buf, kSplitStage,
+                      counter, buf, cap);
     };
     if (hi <= lo) return;
+    if (threadIdx.x == 0) sh_n = 0;
+    __syncthreads();
     const int lo4 = min(aligned_from(row, lo), hi), hi4 = lo4 + ((hi - lo4) & ~3);
     if (threadIdx.x < 32) {   // up to three scores before the first 16-byte boundary: one warp
         const int i = lo + static_cast<int>(threadIdx.x);
@@ -268,22 +347,29 @@ __global__ void __launch_bounds__(kThreads) kda_topk_split_kernel(const float* _
         const bool live = i < hi4;
         float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
         if (live) v = __ldcs(reinterpret_cast<const float4*>(row + i));
-        visit(i, score_key(v.x), live);
-        visit(i + 1, score_key(v.y), live);
-        visit(i + 2, score_key(v.z), live);
-        visit(i + 3, score_key(v.w), live);
+        const uint32_t k0 = score_key(v.x), k1 = score_key(v.y), k2 = score_key(v.z), k3 = score_key(v.w);
+        // most steps keep nothing: a warp whose keys all lie below bin b skips the appends
+        const uint32_t top = max(max(k0, k1), max(k2, k3)) >> 21;
+        if (!__any_sync(0xffffffffu, live && (s.mode == 0 || top >= s.b))) continue;
+        const bool take[4] = {live && (s.mode == 0 || (k0 >> 21) >= s.b), live && (s.mode == 0 || (k1 >> 21) >= s.b),
+                              live && (s.mode == 0 || (k2 >> 21) >= s.b), live && (s.mode == 0 || (k3 >> 21) >= s.b)};
+        const unsigned long long pv[4] = {pair_of(k0, i), pair_of(k1, i + 1), pair_of(k2, i + 2), pair_of(k3, i + 3)};
+        append4_staged(take, pv, &sh_n, sh_buf, kSplitStage, counter, buf, cap);
     }
     if (threadIdx.x < 32) {   // up to three scores after the last boundary: one warp
         const int i = hi4 + static_cast<int>(threadIdx.x);
         const bool live = i < hi;
         visit(i, live ? score_key(row[i]) : 0u, live);
     }
+    flush_staged(&sh_n, sh_buf, kSplitStage, counter, buf, cap, &sh_base);
 }
 
 // One CTA per row: the rest of the cut, the kept set, and the sorted output.
-__global__ void __launch_bounds__(kThreads) kda_topk_finish_kernel(const float* __restrict__ scores, int64_t ld,
-                                                                   int k, Layout L, int32_t* __restrict__ out_idx,
-                                                                   float* __restrict__ out_val) {
+constexpr int kFinishThreads = 1024;
+__global__ void __launch_bounds__(kFinishThreads) kda_topk_finish_kernel(const float* __restrict__ scores, int64_t ld,
+                                                                         int k, Layout L, int32_t* __restrict__ out_idx,
+                                                                         float* __restrict__ out_val) {
+    constexpr int NT = kFinishThreads;
     __shared__ uint32_t h[kBins];
     __shared__ int scratch[40];
     __shared__ unsigned long long sorted[kTopkMaxK];
@@ -291,7 +377,8 @@ __global__ void __launch_bounds__(kThreads) kda_topk_finish_kernel(const float* 
     RowState* sp = L.st + r;
     const RowState s = *sp;
     unsigned long long* kept = L.kept + static_cast<size_t>(r) * k;
-    const unsigned long long* cand = L.cand + static_cast<size_t>(r) * kTopkCap;
+    const unsigned long long* cand = L.cand + static_cast<size_t>(r) * kCandCap;
+    const int ncand = s.ncand < kCandCap ? s.ncand : kCandCap;
     const float* row = scores + r * ld;
 
     if (s.mode != 0) {
@@ -299,12 +386,12 @@ __global__ void __launch_bounds__(kThreads) kda_topk_finish_kernel(const float* 
         // visit(f) calls f(key, idx) for every key of bin b (the caller filters further)
         auto visit = [&](auto f) {
             if (s.mode == 1) {
-                for (int i = t; i < s.cnt_b; i += kThreads) {
+                for (int i = t; i < ncand; i += NT) {
                     const unsigned long long v = cand[i];
                     f(static_cast<uint32_t>(v >> 32), static_cast<int32_t>(~static_cast<uint32_t>(v)));
                 }
             } else {
-                for_keys(row, 0, s.n, t, kThreads, [&](int i, uint32_t key) {
+                for_keys(row, 0, s.n, t, NT, [&](int i, uint32_t key) {
                     if ((key >> 21) == s.b) f(key, i);
                 });
             }
@@ -315,14 +402,14 @@ __global__ void __launch_bounds__(kThreads) kda_topk_finish_kernel(const float* 
         for (int pass = 0; pass < 2; ++pass) {
             const int shift = pass == 0 ? 10 : 0;
             const uint32_t dmask = pass == 0 ? 0x7FFu : 0x3FFu;
-            for (int i = t; i < kBins; i += kThreads) h[i] = 0u;
+            for (int i = t; i < kBins; i += NT) h[i] = 0u;
             __syncthreads();
             visit([&](uint32_t key, int32_t) {
                 if ((key & mask) == prefix) atomicAdd(&h[(key >> shift) & dmask], 1u);
             });
             __syncthreads();
             int above = 0;
-            const int bin = find_bin(h, need, true, &above, scratch);
+            const int bin = find_bin<NT>(h, need, true, &above, scratch);
             prefix |= static_cast<uint32_t>(bin) << shift;
             mask |= dmask << shift;
             need -= above;
@@ -337,7 +424,7 @@ __global__ void __launch_bounds__(kThreads) kda_topk_finish_kernel(const float* 
             for (int pass = 0; pass < 3; ++pass) {
                 const int shift = pass == 0 ? 20 : (pass == 1 ? 10 : 0);
                 const uint32_t dmask = pass == 0 ? 0x7FFu : 0x3FFu;
-                for (int i = t; i < kBins; i += kThreads) h[i] = 0u;
+                for (int i = t; i < kBins; i += NT) h[i] = 0u;
                 __syncthreads();
                 visit([&](uint32_t key, int32_t idx) {
                     const uint32_t u = static_cast<uint32_t>(idx);
@@ -345,7 +432,7 @@ __global__ void __launch_bounds__(kThreads) kda_topk_finish_kernel(const float* 
                 });
                 __syncthreads();
                 int below = 0;
-                const int bin = find_bin(h, need, false, &below, scratch);
+                const int bin = find_bin<NT>(h, need, false, &below, scratch);
                 ip |= static_cast<uint32_t>(bin) << shift;
                 im |= dmask << shift;
                 need -= below;
@@ -356,11 +443,11 @@ __global__ void __launch_bounds__(kThreads) kda_topk_finish_kernel(const float* 
         // keep the keys above the cut and the equal keys up to index `last`
         // (whole warps iterate together for the warp-wide append)
         if (s.mode == 1) {
-            for (int base = 0; base < s.cnt_b; base += kThreads) {
+            for (int base = 0; base < ncand; base += NT) {
                 const int i = base + t;
                 unsigned long long v = 0;
                 bool take = false;
-                if (i < s.cnt_b) {
+                if (i < ncand) {
                     v = cand[i];
                     const uint32_t key = static_cast<uint32_t>(v >> 32);
                     const int32_t idx = static_cast<int32_t>(~static_cast<uint32_t>(v));
@@ -369,7 +456,7 @@ __global__ void __launch_bounds__(kThreads) kda_topk_finish_kernel(const float* 
                 append(take, v, &sp->nsel, kept, k);
             }
         } else {
-            for (int base = 0; base < s.n; base += kThreads) {
+            for (int base = 0; base < s.n; base += NT) {
                 const int i = base + t;
                 bool take = false;
                 unsigned long long v = 0;
@@ -388,11 +475,11 @@ __global__ void __launch_bounds__(kThreads) kda_topk_finish_kernel(const float* 
     const int m = s.n < k ? s.n : k;
     int P = 1;
     while (P < m) P <<= 1;
-    for (int i = t; i < P; i += kThreads) sorted[i] = i < m ? kept[i] : 0ull;
+    for (int i = t; i < P; i += NT) sorted[i] = i < m ? kept[i] : 0ull;
     __syncthreads();
     for (int size = 2; size <= P; size <<= 1) {
         for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            for (int i = t; i < P / 2; i += kThreads) {
+            for (int i = t; i < P / 2; i += NT) {
                 const int lo = 2 * i - (i & (stride - 1)), hi = lo + stride;
                 const bool desc = (lo & size) == 0;   // descending runs build the final descending order
                 const unsigned long long a = sorted[lo], b = sorted[hi];
@@ -404,7 +491,7 @@ __global__ void __launch_bounds__(kThreads) kda_topk_finish_kernel(const float* 
             __syncthreads();
         }
     }
-    for (int i = t; i < k; i += kThreads) {
+    for (int i = t; i < k; i += NT) {
         const bool live = i < m;
         const unsigned long long v = live ? sorted[i] : 0ull;
         out_idx[static_cast<size_t>(r) * k + i] = live ? static_cast<int32_t>(~static_cast<uint32_t>(v)) : -1;
@@ -451,7 +538,8 @@ int kda_topk_indices(const float* scores, int64_t ld, int32_t rows, int64_t n, i
     if (e == cudaSuccess) e = launch_kernel(kda_topk_pick0_kernel, dim3(rows), dim3(kThreads), 0, s, k, L);
     if (e == cudaSuccess) e = launch_kernel(kda_topk_split_kernel, grid2, dim3(kThreads), 0, s, scores, ld, k, L);
     if (e == cudaSuccess)
-        e = launch_kernel(kda_topk_finish_kernel, dim3(rows), dim3(kThreads), 0, s, scores, ld, k, L, indices, values);
+        e = launch_kernel(kda_topk_finish_kernel, dim3(rows), dim3(kFinishThreads), 0, s, scores, ld, k, L, indices,
+                          values);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
