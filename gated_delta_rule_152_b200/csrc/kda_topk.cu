@@ -128,9 +128,9 @@ __device__ __forceinline__ void for_keys(const float* row, int lo, int hi, int t
     for (int i = hi4 + t; i < hi; i += nt) f(i, score_key(__ldg(row + i)));
 }
 
-// Warp-aggregated append of (key, idx) to a per-row buffer with a shared counter.
-__device__ __forceinline__ void append(bool take, unsigned long long v, int32_t* counter,
-                                       unsigned long long* buf, int cap) {
+// Warp-aggregated append of (key, idx) to a buffer in shared memory.
+__device__ __forceinline__ void append_shared(bool take, unsigned long long v, int* counter, unsigned long long* buf,
+                                              int cap) {
     const unsigned m = __ballot_sync(0xffffffffu, take);
     if (!m) return;
     const int lane = threadIdx.x & 31, leader = __ffs(m) - 1;
@@ -142,7 +142,6 @@ __device__ __forceinline__ void append(bool take, unsigned long long v, int32_t*
         if (pos < cap) buf[pos] = v;
     }
 }
-
 // The same append staged in shared memory: the pairs of one CTA collect in `sh`
 // (cap_sh of them; any further ones go straight to the row's buffer), and
 // flush_staged moves them out with one reservation on the row's counter.
@@ -373,7 +372,9 @@ __global__ void __launch_bounds__(kFinishThreads) kda_topk_finish_kernel(const f
     __shared__ uint32_t h[kBins];
     __shared__ int scratch[40];
     __shared__ unsigned long long sorted[kTopkMaxK];
+    __shared__ int sh_nsel;   // kept pairs gathered into `sorted`
     const int r = blockIdx.x, t = threadIdx.x;
+    if (t == 0) sh_nsel = 0;
     RowState* sp = L.st + r;
     const RowState s = *sp;
     unsigned long long* kept = L.kept + static_cast<size_t>(r) * k;
@@ -453,7 +454,7 @@ __global__ void __launch_bounds__(kFinishThreads) kda_topk_finish_kernel(const f
                     const int32_t idx = static_cast<int32_t>(~static_cast<uint32_t>(v));
                     take = key > T || (key == T && idx <= last);
                 }
-                append(take, v, &sp->nsel, kept, k);
+                append_shared(take, v, &sh_nsel, sorted, kTopkMaxK);
             }
         } else {
             for (int base = 0; base < s.n; base += NT) {
@@ -465,17 +466,22 @@ __global__ void __launch_bounds__(kFinishThreads) kda_topk_finish_kernel(const f
                     v = pair_of(key, i);
                     take = key > T || (key == T && i <= last);
                 }
-                append(take, v, &sp->nsel, kept, k);
+                append_shared(take, v, &sh_nsel, sorted, kTopkMaxK);
             }
         }
         __syncthreads();
     }
-    __threadfence_block();
-    // bitonic sort, best first, of the m kept pairs (padded with zeros, which rank last)
+    // bitonic sort, best first, of the m kept pairs (padded with zeros, which rank last):
+    // gathered into `sorted` above, or written by the split step when the row has at
+    // most k tokens
     const int m = s.n < k ? s.n : k;
     int P = 1;
     while (P < m) P <<= 1;
-    for (int i = t; i < P; i += NT) sorted[i] = i < m ? kept[i] : 0ull;
+    if (s.mode == 0) {
+        for (int i = t; i < P; i += NT) sorted[i] = i < m ? kept[i] : 0ull;
+    } else {
+        for (int i = m + t; i < P; i += NT) sorted[i] = 0ull;
+    }
     __syncthreads();
     for (int size = 2; size <= P; size <<= 1) {
         for (int stride = size >> 1; stride > 0; stride >>= 1) {
