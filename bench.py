@@ -66,9 +66,15 @@ PREFILL_KERNELS = ("kda_chunk_index_kernel", "kda_chunk_overlap_kernel")
 # kernel sources it was taken on: when the sources differ, the figure no
 # longer describes the kernel and the line reports traffic as null.
 MEASURED_TRAFFIC = {
-    "prefill": {"bytes": None, "capture": None, "sources_sha": None,
+    # 336,992,256 B read + 120,929,024 B written (one-pass capture)
+    "prefill": {"bytes": 457921280,
+                "capture": "profiles/kda_chunk_overlap_kernel__prefill_bf16_T8192_H32.md",
+                "sources_sha": "38a0d28fafc61985",
                 "files": ("kda_chunk2.cu", "kda_tile.cuh", "sm100.cuh", "kda_common.cuh", "kda_launch.h")},
-    "decode": {"bytes": None, "capture": None, "sources_sha": None,
+    # 547,409,408 B read + 483,761,920 B written
+    "decode": {"bytes": 1031171328,
+               "capture": "profiles/kda_decode_kernel__decode_bf16_256seq_H32_one_layer.md",
+               "sources_sha": "db3decae6f041942",
                "files": ("kda_decode.cu", "kda_common.cuh", "kda_launch.h")},
 }
 
