@@ -383,42 +383,44 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
                 bprev = cc.bstart;
                 bcur = cc.bend;
             };
-            prep_chunk_rows(smem + P_KB, smem + P_KB + kC * kD * 2, greg, xch, L, scale, l2norm != 0, setup,
-                            [&](int r, int kbi, int ch, float4 qn, float4 kn, float4 gr) {
-                float4 q4, k4, b4, xq, xk, y;
-                if (level == 0) {
-                    const float4 a = sub4(gr, gc);   // >= 0, at most kSafeLog2 at this level
-                    const float4 E = ex2x4(a), F = ex2x4(make_float4(-a.x, -a.y, -a.z, -a.w));
-                    const float4 qt = mul4(qn, E), kt = mul4(kn, E), kb = mul4(kn, F);
-                    q4 = xq = tf32x4(qt.x, qt.y, qt.z, qt.w);
-                    k4 = xk = tf32x4(kt.x, kt.y, kt.z, kt.w);
-                    b4 = y = tf32x4(kb.x, kb.y, kb.z, kb.w);
-                } else {
-                    // chunk-start form (every factor <= 1)
-                    const float4 e0 = ex2x4(gr), f = ex2x4(sub4(gc, gr));
-                    const float4 qs = mul4(qn, e0), ks = mul4(kn, e0), kb = mul4(kn, f);
-                    q4 = tf32x4(qs.x, qs.y, qs.z, qs.w);
-                    k4 = tf32x4(ks.x, ks.y, ks.z, ks.w);
-                    b4 = tf32x4(kb.x, kb.y, kb.z, kb.w);
-                    if (level == 1) {   // block references: X = 2^(Gamma_r - rho_{a-1}), Y = 2^(rho_a - Gamma_r)
-                        const float4 X = ex2x4(sub4(gr, bprev)), Y = ex2x4(sub4(bcur, gr));
-                        xq = mul4(qn, X);
-                        xk = mul4(kn, X);
-                        const float4 ky = mul4(kn, Y);
-                        y = tf32x4(ky.x, ky.y, ky.z, ky.w);
-                    } else {
-                        xq = qn;
-                        xk = kn;
-                        y = gr;
-                    }
-                }
+            // the six stores of one row and 4 channels
+            auto put = [&](int r, int kbi, int ch, float4 xq, float4 xk, float4 y, float4 k4, float4 q4, float4 b4) {
                 *reinterpret_cast<float4*>(smem + P_X + kbi * KB_B1 + sw128_off(r, ch)) = xq;
                 *reinterpret_cast<float4*>(smem + P_X + kbi * KB_B1 + sw128_off(64 + r, ch)) = xk;
                 *reinterpret_cast<float4*>(smem + P_KB + kbi * P_KB_KB + sw128_off(r, ch)) = y;
                 *reinterpret_cast<float4*>(smem + P_KTM + kbi * P_MN_KB + sw32g_off(r, ch)) = k4;
                 *reinterpret_cast<float4*>(im + IMG_B1 + kbi * KB_B1 + sw128_off(r, ch)) = q4;
                 *reinterpret_cast<float4*>(im + IMG_KB + kbi * IMG_BLK + sw32g_off(r, ch)) = b4;
+            };
+            // level 0 (the common case) in a pass of its own, without the other levels'
+            // branches; a chunk of level 1 or 2 runs the rows again with the general emit
+            prep_chunk_rows<0>(smem + P_KB, smem + P_KB + kC * kD * 2, greg, xch, L, scale, l2norm != 0, setup,
+                               [&](int r, int kbi, int ch, float4 qn, float4 kn, float4 gr) {
+                const float4 a = sub4(gr, gc);   // >= 0, at most kSafeLog2 at this level
+                const float4 E = ex2x4(a), F = ex2x4(make_float4(-a.x, -a.y, -a.z, -a.w));
+                const float4 qt = mul4(qn, E), kt = mul4(kn, E), kb = mul4(kn, F);
+                const float4 q4 = tf32x4(qt.x, qt.y, qt.z, qt.w), k4 = tf32x4(kt.x, kt.y, kt.z, kt.w),
+                             b4 = tf32x4(kb.x, kb.y, kb.z, kb.w);
+                put(r, kbi, ch, q4, k4, b4, k4, q4, b4);
             });
+            if (level != 0) {
+                __syncthreads();   // every warp is past the first pass's reads of xch
+                prep_chunk_rows(smem + P_KB, smem + P_KB + kC * kD * 2, greg, xch, L, scale, l2norm != 0, setup,
+                                [&](int r, int kbi, int ch, float4 qn, float4 kn, float4 gr) {
+                    // chunk-start form (every factor <= 1)
+                    const float4 e0 = ex2x4(gr), f = ex2x4(sub4(gc, gr));
+                    const float4 qs = mul4(qn, e0), ks = mul4(kn, e0), kb = mul4(kn, f);
+                    const float4 q4 = tf32x4(qs.x, qs.y, qs.z, qs.w), k4 = tf32x4(ks.x, ks.y, ks.z, ks.w),
+                                 b4 = tf32x4(kb.x, kb.y, kb.z, kb.w);
+                    if (level == 1) {   // block references: X = 2^(Gamma_r - rho_{a-1}), Y = 2^(rho_a - Gamma_r)
+                        const float4 X = ex2x4(sub4(gr, bprev)), Y = ex2x4(sub4(bcur, gr));
+                        const float4 ky = mul4(kn, Y);
+                        put(r, kbi, ch, mul4(qn, X), mul4(kn, X), tf32x4(ky.x, ky.y, ky.z, ky.w), k4, q4, b4);
+                    } else {
+                        put(r, kbi, ch, qn, kn, gr, k4, q4, b4);
+                    }
+                });
+            }
             if (warp == 0) *reinterpret_cast<float4*>(im + IMG_DC + 16 * lane) = ex2x4(gc);
             if (tid == 64)
                 *reinterpret_cast<float4*>(im + IMG_FORM) = make_float4(level != 0 ? 1.f : 0.f, 0.f, 0.f, 0.f);

@@ -201,8 +201,10 @@ constexpr float kSafeLog2 = 100.f;
 // emit(r, kbi, ch, qn, kn, gr) with the fp32 q^, k^ and Gamma_r of row r for
 // the K-block kbi = lane / 8 and 16-byte chunk ch = lane % 8 of a K-major
 // tile.  Returns the level.  xch is a shared [8][128] exchange buffer.  All
-// 256 threads must call it.
-template <class Setup, class Emit>
+// 256 threads must call it.  With kMaxLevel < 2 and a chunk of a higher level,
+// it returns after setup without calling emit (the raw rows are then still in
+// place; a block barrier must separate this call from the next one).
+template <int kMaxLevel = 2, class Setup, class Emit>
 __device__ __forceinline__ int prep_chunk_rows(const uint8_t* rq, const uint8_t* rk, const float (&greg)[8][4],
                                                float* xch, int L, float scale, bool l2norm, Setup setup,
                                                Emit emit) {
@@ -258,6 +260,7 @@ __device__ __forceinline__ int prep_chunk_rows(const uint8_t* rq, const uint8_t*
                       : !__any_sync(0xffffffffu, block_decay > kSafeLog2) ? 1
                                                                           : 2;
     setup(cc, level);
+    if (kMaxLevel < 2 && level > kMaxLevel) return level;
 
     // unpack, mask rows past the sequence end, and L2-normalise all 8 rows
     float2 qv[8][2], kv[8][2];
