@@ -236,21 +236,29 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
     const uint32_t tmem = *tmem_slot;
 
     // work item w -> chunk gc = w / H of head h = w % H; sequence n = the last
-    // one whose first chunk is <= gc (sequences without chunks are skipped)
+    // one whose first chunk is <= gc (sequences without chunks are skipped).
+    // Items are decoded in increasing order, stride apart: (gc, h) advances by
+    // (stride / H, stride % H) with a carry, and the sequence search goes on
+    // from the previous item's sequence.
     struct Item {
         int64_t t0, gc;
         int L, h, c;   // c: chunk index inside its sequence
     };
-    auto decode = [&](int64_t w) {
-        Item it;
-        it.gc = w / H;
-        it.h = static_cast<int>(w - it.gc * H);
-        int lo = 0, hi = N;
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (chunk_off[mid] <= it.gc) lo = mid;
-            else hi = mid;
+    const int64_t step_gc = stride / H;
+    const int step_h = static_cast<int>(stride - step_gc * H);
+    int seq = 0;
+    auto advance = [&](Item p) {
+        p.gc += step_gc;
+        p.h += step_h;
+        if (p.h >= H) {
+            p.h -= H;
+            ++p.gc;
         }
+        return p;
+    };
+    auto decode = [&](Item it) {
+        while (seq + 1 < N && chunk_off[seq + 1] <= it.gc) ++seq;
+        const int lo = seq;
         it.c = static_cast<int>(it.gc - chunk_off[lo]);
         it.t0 = cu[lo] + static_cast<int64_t>(it.c) * kC;
         const int64_t rem = cu[lo + 1] - it.t0;
@@ -327,9 +335,14 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
     };
 
     int64_t w = first;
-    Item cur = decode(w);
-    Item nxt = w + stride < items ? decode(w + stride) : cur;
-    Item nxt2 = w + 2 * stride < items ? decode(w + 2 * stride) : cur;   // only for an L2 prefetch
+    Item pos2;   // position (gc, h) of the item two ahead
+    pos2.gc = first / H;
+    pos2.h = static_cast<int>(first - pos2.gc * H);
+    Item cur = decode(pos2);
+    pos2 = advance(pos2);
+    Item nxt = w + stride < items ? decode(pos2) : cur;
+    pos2 = advance(pos2);
+    Item nxt2 = w + 2 * stride < items ? decode(pos2) : cur;   // only for an L2 prefetch
     if (tid == 0) issue_load(cur);
     load_pending = true;
     prefetch(cur);
@@ -638,7 +651,8 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
         }
         cur = nxt;
         nxt = nxt2;
-        if (w2 + stride < items) nxt2 = decode(w2 + stride);
+        pos2 = advance(pos2);
+        if (w2 + stride < items) nxt2 = decode(pos2);
     }
 
     if (tid == kStoreThread) {
