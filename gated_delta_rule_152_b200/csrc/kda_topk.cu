@@ -341,15 +341,26 @@ __global__ void __launch_bounds__(kThreads) kda_topk_split_kernel(const float* _
         const bool live = i < lo4;
         visit(i, live ? score_key(row[i]) : 0u, live);
     }
+    // The filter below needs no keys when bin b's lowest key is that of a number fb:
+    // key(x) >= b << 21 exactly when x >= fb (the key order is the float order, -0
+    // and +0 alike); bins 0-3 and 2044-2047 begin among the NaN bit patterns
+    const bool by_float = s.mode == 1 && s.b >= 4u && s.b < 2044u;
+    const float fb = by_float ? key_score(s.b << 21) : 0.f;
     for (int base = lo4; base < hi4; base += 4 * kThreads) {
         const int i = base + 4 * static_cast<int>(threadIdx.x);
         const bool live = i < hi4;
         float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
         if (live) v = __ldcs(reinterpret_cast<const float4*>(row + i));
+        // most steps keep nothing: a warp whose scores all lie below bin b skips the appends
+        bool maybe;
+        if (by_float) {
+            maybe = live && fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)) >= fb;
+        } else {
+            const uint32_t top = max(max(score_key(v.x), score_key(v.y)), max(score_key(v.z), score_key(v.w))) >> 21;
+            maybe = live && (s.mode == 0 || top >= s.b);
+        }
+        if (!__any_sync(0xffffffffu, maybe)) continue;
         const uint32_t k0 = score_key(v.x), k1 = score_key(v.y), k2 = score_key(v.z), k3 = score_key(v.w);
-        // most steps keep nothing: a warp whose keys all lie below bin b skips the appends
-        const uint32_t top = max(max(k0, k1), max(k2, k3)) >> 21;
-        if (!__any_sync(0xffffffffu, live && (s.mode == 0 || top >= s.b))) continue;
         const bool take[4] = {live && (s.mode == 0 || (k0 >> 21) >= s.b), live && (s.mode == 0 || (k1 >> 21) >= s.b),
                               live && (s.mode == 0 || (k2 >> 21) >= s.b), live && (s.mode == 0 || (k3 >> 21) >= s.b)};
         const unsigned long long pv[4] = {pair_of(k0, i), pair_of(k1, i + 1), pair_of(k2, i + 2), pair_of(k3, i + 3)};
