@@ -563,6 +563,9 @@ STRONG = {
     "g_80_three": lambda g: g.__setitem__((Ellipsis, [3, 77, 100]), -80.0),   # ~5,000 nats per chunk
     "x40": lambda g: g.mul_(40.0),                         # ~270 nats per chunk on the fastest channel
     "spike": lambda g: g[100, :, 5].fill_(-150.0),         # one token, one channel
+    # chunks of all three levels in one sequence: level 1 on chunks 3-4, level 2 on
+    # chunk 7, level 0 around them (the state role switches forms chunk by chunk)
+    "mixed": lambda g: (g[192:320].fill_(-1.6), g[448:512, :, ::3].fill_(-8.0)),
 }
 
 
@@ -589,11 +592,13 @@ def _levels(x):
 
 @pytest.mark.parametrize("path", ["one_sequence", "two_sequences", "fused"])
 @pytest.mark.parametrize("kind,level", [("g_1.6_all", 1), ("g_8_third", 2), ("g_80_three", 2), ("x40", 2),
-                                        ("spike", 2)])
+                                        ("spike", 2), ("mixed", 2)])
 def test_prefill_strong_decay(kind, level, path):
     lengths = [640] if path != "two_sequences" else [300, 340]
     x = _strong_input(kind, lengths)
     assert max(_levels(x)) == level   # the case exercises the intended Gram level
+    if kind == "mixed" and path == "one_sequence":
+        assert _levels(x) == {0, 1, 2}
     o, s, o_ref, s_ref = run_both(x, path="fused" if path == "fused" else "two_pass")
     assert_close(o, o_ref, TOL_BF16, "o")
     assert_close(s, s_ref, TOL_BF16, "final state")
