@@ -411,30 +411,39 @@ def bench_gpu(args, world, rank, local):
     achieved_tflops = flops_per_launch / (ms / 1e3) / 1e12
 
     # end to end: pinned host inputs -> device, call, o + final state -> host,
-    # every step.  The result copies of step i run on a second stream while
-    # step i+1's inputs come in (PCIe is full duplex); outputs and their host
-    # copies are double-buffered so that no copy is overwritten in flight.
+    # every step.  Inputs, outputs and their host copies are double-buffered:
+    # step i+1's inputs come in on one copy stream while step i computes, and
+    # step i's results leave on another (PCIe is full duplex); an event orders
+    # every reuse of a buffer after its last reader.
     pin = lambda t: t.pin_memory()
-    hq, hk, hv, hg, hb, hcu = (pin(t) for t in (x.q, x.k, x.v, x.g, x.beta, x.cu_seqlens))
+    hins = [pin(t) for t in (x.q, x.k, x.v, x.g, x.beta, x.cu_seqlens)]
     ho = [torch.empty(T, H, D).pin_memory() for _ in range(2)]
     hs = [torch.empty(1, H, D, D).pin_memory() for _ in range(2)]
     do = [o, torch.empty(T, H, D, device=dev)]
     ds = [sT, torch.empty(1, H, D, D, device=dev)]
-    dq, dk, dv, dg, db, dcu = (torch.empty_like(t, device=dev) for t in (hq, hk, hv, hg, hb, hcu))
-    out_stream = torch.cuda.Stream(dev)
+    dins = [[torch.empty_like(t, device=dev) for t in hins] for _ in range(2)]
+    in_stream, out_stream = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    in_done = [torch.cuda.Event(), torch.cuda.Event()]
+    comp_done = [torch.cuda.Event(), torch.cuda.Event()]
     out_done = [torch.cuda.Event(), torch.cuda.Event()]
+    for ev in comp_done:
+        ev.record(stream)
     for ev in out_done:
         ev.record(out_stream)
 
     def e2e_step(i):
         b = i & 1
-        for d_, h_ in ((dq, hq), (dk, hk), (dv, hv), (dg, hg), (db, hb), (dcu, hcu)):
-            d_.copy_(h_, non_blocking=True)
-        stream.wait_event(out_done[b])   # step i-2's results have left buffer b
+        in_stream.wait_event(comp_done[b])   # step i-2's call has read input set b
+        with torch.cuda.stream(in_stream):
+            for d_, h_ in zip(dins[b], hins):
+                d_.copy_(h_, non_blocking=True)
+        in_done[b].record(in_stream)
+        stream.wait_event(in_done[b])
+        stream.wait_event(out_done[b])       # step i-2's results have left output set b
+        dq, dk, dv, dg, db, dcu = dins[b]
         kda.kda_chunk_fwd(dq, dk, dv, dg, db, dcu, final_state=ds[b], o=do[b], workspace=ws, stream=stream)
-        computed = torch.cuda.Event()
-        computed.record(stream)
-        out_stream.wait_event(computed)
+        comp_done[b].record(stream)
+        out_stream.wait_event(comp_done[b])
         with torch.cuda.stream(out_stream):
             ho[b].copy_(do[b], non_blocking=True)
             hs[b].copy_(ds[b], non_blocking=True)
@@ -446,6 +455,7 @@ def bench_gpu(args, world, rank, local):
     barrier(world)
     torch.cuda.synchronize(dev)
     e0.record(stream)
+    in_stream.wait_event(e0)   # the first timed copies start inside the timed region
     for i in range(args.steps):
         e2e_step(i)
     for ev in out_done:   # the last results are on the host
@@ -454,9 +464,9 @@ def bench_gpu(args, world, rank, local):
     torch.cuda.synchronize(dev)
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hg, hb, hcu))
+    h2d = sum(t.numel() * t.element_size() for t in hins)
     d2h = ho[0].numel() * 4 + hs[0].numel() * 4
-    del xd, dq, dk, dv, dg, db, do, ds
+    del xd, dins, do, ds
     torch.cuda.empty_cache()
 
     # ---------------- decode (256 seq x 34 layers) -------------------------
