@@ -276,8 +276,8 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
     // is announced by the store thread once those bulk stores have completed:
     // a proxy fence, then a gpu-scope release, which also covers the plain
     // stores of the other threads (ordered before it by the barriers).  That
-    // happens while the next item's W / U product runs, or before the store
-    // thread blocks on a slot.
+    // happens once the next item's rows are done, or before the store thread
+    // blocks on a slot.
     int32_t* pub_flag = nullptr;
     int32_t pub_val = 0;
     auto publish = [&]() {
@@ -439,8 +439,9 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
                 *reinterpret_cast<float4*>(im + IMG_FORM) = make_float4(level != 0 ? 1.f : 0.f, 0.f, 0.f, 0.f);
             if (tid < kC) beta_s[tid] = breg;
         }
-        // the previous item's U and W have left V and WST (V is rewritten below)
-        if (tid == kStoreThread) bulk_wait_read();
+        // the previous item's U and W have left V and WST (V is rewritten below); their
+        // bulk stores have completed by now, so the previous item's image is announced
+        if (tid == kStoreThread) publish();
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
@@ -589,7 +590,7 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
         mma_pending = true;
         if (has_next) prefetch(nxt);
         if (tid == kStoreThread) {
-            publish();   // the previous item's image (its stores are long complete)
+            publish();   // (announced already; the call only covers the last item of a loop exit)
             if (RING && has_next) done_seen = ld_relaxed_gpu(done_flag(ring, nxt.h));
         }
         // ============== meanwhile P (lower incl., tf32, K-major) from TMEM -> X (free
