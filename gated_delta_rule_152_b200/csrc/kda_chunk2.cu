@@ -276,8 +276,8 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
     // is announced by the store thread once those bulk stores have completed:
     // a proxy fence, then a gpu-scope release, which also covers the plain
     // stores of the other threads (ordered before it by the barriers).  That
-    // happens once the next item's rows are done, or before the store thread
-    // blocks on a slot.
+    // happens when the next item's rows reach their decay sums, or before the
+    // store thread blocks on a slot.
     int32_t* pub_flag = nullptr;
     int32_t pub_val = 0;
     auto publish = [&]() {
@@ -391,6 +391,9 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
             // (level 1); the full block-end table is rebuilt from xch after the rows
             float4 gc, bprev, bcur;
             auto setup = [&](const ChunkChannels& cc, int lvl) {
+                // the previous item's W and U bulk stores have had the row
+                // normalisation and the decay sums to complete: announce its image
+                if (tid == kStoreThread) publish();
                 level = lvl;
                 gc = cc.rho[3];
                 bprev = cc.bstart;
@@ -439,9 +442,6 @@ __device__ __forceinline__ void prep_role(const CUtensorMap* tm_q, const CUtenso
                 *reinterpret_cast<float4*>(im + IMG_FORM) = make_float4(level != 0 ? 1.f : 0.f, 0.f, 0.f, 0.f);
             if (tid < kC) beta_s[tid] = breg;
         }
-        // the previous item's U and W have left V and WST (V is rewritten below); their
-        // bulk stores have completed by now, so the previous item's image is announced
-        if (tid == kStoreThread) publish();
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
