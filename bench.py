@@ -66,10 +66,10 @@ PREFILL_KERNELS = ("kda_chunk_index_kernel", "kda_chunk_overlap_kernel")
 # kernel sources it was taken on: when the sources differ, the figure no
 # longer describes the kernel and the line reports traffic as null.
 MEASURED_TRAFFIC = {
-    # 336,965,120 B read + 120,091,904 B written (one-pass capture)
-    "prefill": {"bytes": 457057024,
+    # 336,875,008 B read + 121,080,576 B written (one-pass capture)
+    "prefill": {"bytes": 457955584,
                 "capture": "profiles/kda_chunk_overlap_kernel__prefill_bf16_T8192_H32.md",
-                "sources_sha": "210a0797ac24da83",
+                "sources_sha": "04e0894bf777ae0d",
                 "files": ("kda_chunk2.cu", "kda_tile.cuh", "sm100.cuh", "kda_common.cuh", "kda_launch.h")},
     # 547,409,408 B read + 483,761,920 B written
     "decode": {"bytes": 1031171328,
