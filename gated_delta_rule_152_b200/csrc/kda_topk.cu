@@ -374,6 +374,80 @@ __global__ void __launch_bounds__(kThreads) kda_topk_split_kernel(const float* _
     flush_staged(&sh_n, sh_buf, kSplitStage, counter, buf, cap, &sh_base);
 }
 
+// One compare-exchange stage in registers: stride s (< 64) of block size `size`.
+__device__ __forceinline__ void bitonic_reg_stage(ulonglong2& x, int v, int size, int s) {
+    const bool desc = ((2 * v) & size) == 0;
+    if (s == 1) {
+        if ((x.x < x.y) == desc) {
+            const unsigned long long tmp = x.x;
+            x.x = x.y;
+            x.y = tmp;
+        }
+    } else {
+        const int hs = s >> 1;
+        const unsigned long long y0 = __shfl_xor_sync(0xffffffffu, x.x, hs);
+        const unsigned long long y1 = __shfl_xor_sync(0xffffffffu, x.y, hs);
+        const bool keep_max = ((v & hs) == 0) == desc;   // the lower thread holds the lower index
+        x.x = keep_max ? (x.x > y0 ? x.x : y0) : (x.x < y0 ? x.x : y0);
+        x.y = keep_max ? (x.y > y1 ? x.y : y1) : (x.y < y1 ? x.y : y1);
+    }
+}
+
+// Bitonic sort, descending, of the P pairs in a (P a power of two, P <= 4 NT),
+// by all NT threads; ends with a block barrier.  Strides of 64 and more take
+// a shared-memory pass and a block barrier each; the strides below 64 of every
+// merge run in registers, elements 2v and 2v+1 in (virtual) thread v, with the
+// partner element of stride s >= 2 in thread v ^ (s / 2) of the same warp.
+// Descending runs (the compare direction of block `size` containing the pair)
+// build the final descending order.
+template <int NT>
+__device__ __forceinline__ void bitonic_desc(unsigned long long* a, int P) {
+    const int t = threadIdx.x, nv = P >> 1;
+    // whole warps over the virtual threads (for the shuffles); lanes past nv carry zeros
+    auto each_warp = [&](auto body) {
+        for (int v0 = t & ~31; v0 < nv; v0 += NT) {
+            const int v = v0 + (t & 31);
+            const bool live = v < nv;
+            ulonglong2 x = live ? *reinterpret_cast<const ulonglong2*>(a + 2 * v) : make_ulonglong2(0ull, 0ull);
+            body(x, v);
+            if (live) *reinterpret_cast<ulonglong2*>(a + 2 * v) = x;
+        }
+    };
+    if (P >= 64) {
+        each_warp([&](ulonglong2& x, int v) {
+#pragma unroll
+            for (int size = 2; size <= 64; size <<= 1)
+#pragma unroll
+                for (int st = size >> 1; st >= 1; st >>= 1) bitonic_reg_stage(x, v, size, st);
+        });
+    } else if (P >= 2) {
+        each_warp([&](ulonglong2& x, int v) {
+            for (int size = 2; size <= P; size <<= 1)
+                for (int st = size >> 1; st >= 1; st >>= 1) bitonic_reg_stage(x, v, size, st);
+        });
+    }
+    __syncthreads();
+    for (int size = 128; size <= P; size <<= 1) {
+        for (int stride = size >> 1; stride >= 64; stride >>= 1) {
+            for (int i = t; i < nv; i += NT) {
+                const int lo = 2 * i - (i & (stride - 1)), hi = lo + stride;
+                const bool desc = (lo & size) == 0;
+                const unsigned long long x = a[lo], y = a[hi];
+                if ((x < y) == desc) {
+                    a[lo] = y;
+                    a[hi] = x;
+                }
+            }
+            __syncthreads();
+        }
+        each_warp([&](ulonglong2& x, int v) {
+#pragma unroll
+            for (int st = 32; st >= 1; st >>= 1) bitonic_reg_stage(x, v, size, st);
+        });
+        __syncthreads();
+    }
+}
+
 // One CTA per row: the rest of the cut, the kept set, and the sorted output.
 constexpr int kFinishThreads = 1024;
 __global__ void __launch_bounds__(kFinishThreads) kda_topk_finish_kernel(const float* __restrict__ scores, int64_t ld,
@@ -382,7 +456,7 @@ __global__ void __launch_bounds__(kFinishThreads) kda_topk_finish_kernel(const f
     constexpr int NT = kFinishThreads;
     __shared__ uint32_t h[kBins];
     __shared__ int scratch[40];
-    __shared__ unsigned long long sorted[kTopkMaxK];
+    __shared__ __align__(16) unsigned long long sorted[kTopkMaxK];
     __shared__ int sh_nsel;   // kept pairs gathered into `sorted`
     const int r = blockIdx.x, t = threadIdx.x;
     if (t == 0) sh_nsel = 0;
@@ -494,20 +568,7 @@ __global__ void __launch_bounds__(kFinishThreads) kda_topk_finish_kernel(const f
         for (int i = m + t; i < P; i += NT) sorted[i] = 0ull;
     }
     __syncthreads();
-    for (int size = 2; size <= P; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            for (int i = t; i < P / 2; i += NT) {
-                const int lo = 2 * i - (i & (stride - 1)), hi = lo + stride;
-                const bool desc = (lo & size) == 0;   // descending runs build the final descending order
-                const unsigned long long a = sorted[lo], b = sorted[hi];
-                if ((a < b) == desc) {
-                    sorted[lo] = b;
-                    sorted[hi] = a;
-                }
-            }
-            __syncthreads();
-        }
-    }
+    bitonic_desc<NT>(sorted, P);
     for (int i = t; i < k; i += NT) {
         const bool live = i < m;
         const unsigned long long v = live ? sorted[i] : 0ull;
